@@ -1,0 +1,435 @@
+"""Benchmark of the CSA2 decode step over the FP4 KV cache (B200, sm_100a).
+
+Workload: the 64K-context decode batch -- 32 sequences of 65,536 tokens, 64
+query heads x 512 latent, FP4 KV in 64-token pages scattered over a 4 GiB
+pool, one decoder group Full + 3 Reuse then one group Reindex + 3 Reuse.  A
+step appends each sequence's newest token (csa2_kv_quant_append) and runs the
+8 layers (csa2_indexer_score_topk for Full / Reindex, csa2_sparse_attn for
+every layer).  Metric: layer-steps/s (one layer over the whole batch).
+
+Timing: W warm-up steps, then K timed steps; L2 is flushed (a 256 MiB write)
+before every step, outside the timed events; each step is bracketed by CUDA
+events on the launching stream and the step time is their sum; with N ranks
+(torchrun) every rank runs its own batch (weak scaling, no collective on the
+data path) and the reported time is the max over ranks.
+
+``--impl reference`` times the CPU oracle instead (bounded sample, host cores).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "CSA2 decode layer-steps/s at 64K ctx; achieved HBM GB/s vs B200 peak"
+UNIT = "layer-steps/s"
+CONFIG_ID = 1
+L2_FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def _config_json(w, n_gpus):
+    return {"workload": "decode B=32 x 65536-token context, 64 heads x 512 latent, 8 layers "
+                        "F,R,R,R,RI,R,R,R, 64-token pages in a 4 GiB pool",
+            "batch": w.batch, "context": w.lengths[0], "heads": w.heads, "layers": w.layers,
+            "l2": "flushed before every step (256 MiB write outside the timed events)",
+            "parallelism": f"dp{n_gpus} (independent batches per GPU)"}
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def _attended_rows(idx: np.ndarray, L: int) -> int:
+    w0 = max(0, L - 128)
+    sel = idx[(idx >= 0) & (idx < w0)]
+    return int(sel.size + (L - w0))
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import workload as wl
+    from fp4_kv_cache_decode_b200 import _build, csa2, synthetic
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not os.path.exists(_build.LIB):
+        raise SystemExit("libcsa2.so is not built: run `python -c 'import __graft_entry__ as g; g.build()'`")
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    w = wl.workload(CONFIG_ID)
+    if world > 1:
+        w.seed = w.seed + 1000 * rank          # every rank gets its own batch
+    torch.manual_seed(0)
+    cache = synthetic.new_cache(w)
+    synthetic.fill_decode_cache(w, cache)
+    step = synthetic.DecodeStep(w, cache)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    assert csa2.csa2_check_device_error(cache) == 0
+
+    calls = ["append"] + [f"L{i}:{m}" for i, m in enumerate(w.layers)]
+
+    def timed_step(ev):
+        ev[0].record(stream)
+        step.append()
+        ev[1].record(stream)
+        for i in range(len(w.layers)):
+            step.layer(i)
+            ev[2 + i].record(stream)
+
+    n_ev = 2 + len(w.layers)
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step.run()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)
+        timed_step(events[k])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+
+    per_call = np.zeros((args.steps, n_ev - 1))
+    for k in range(args.steps):
+        for j in range(n_ev - 1):
+            per_call[k, j] = events[k][j].elapsed_time(events[k][j + 1])   # ms
+    step_ms = per_call.sum(axis=1)
+    total_ms = float(step_ms.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    assert csa2.csa2_check_device_error(cache) == 0
+
+    # --- algorithmic work of one step (from the sets the step produced) ---
+    L = w.lengths[0]
+    B = w.batch
+    nb = (L + 7) // 8
+    full_sets = synthetic.DecodeStep(w, cache, layers=["F"])
+    full_sets.run(append=False)
+    torch.cuda.synchronize()
+    rows_full = sum(_attended_rows(r, L) for r in full_sets.iset.idx.cpu().numpy())
+    rows_ri = sum(_attended_rows(r, L) for r in step.iset.idx.cpu().numpy())
+    rows_per_layer = [rows_full if i < 4 else rows_ri for i in range(len(w.layers))]
+    bytes_attn = [r * 288 for r in rows_per_layer]
+    flops_attn = [4.0 * w.heads * 512 * r for r in rows_per_layer]
+    bytes_full_idx = B * (nb * 128 + 16384 * 128)
+    bytes_ri_idx = B * 16384 * 128
+    step_bytes = bytes_full_idx + bytes_ri_idx + sum(bytes_attn)
+    mean_call = per_call.mean(axis=0)        # ms per call type (append, L0..L7)
+
+    peaks = _peaks()
+    # per call type: attention calls (Reuse layers are attention only)
+    reuse_ms = float(np.mean([mean_call[1 + i] for i, m in enumerate(w.layers) if m == "R"]))
+    reuse_flops = float(np.mean([flops_attn[i] for i, m in enumerate(w.layers) if m == "R"]))
+    reuse_bytes = float(np.mean([bytes_attn[i] for i, m in enumerate(w.layers) if m == "R"]))
+    # the Full layer = indexer + attention; its indexer share is Full - Reuse-like attention
+    full_ms = float(mean_call[1])
+    ri_ms = float(mean_call[1 + w.layers.index("RI")])
+    attn_total_ms = reuse_ms * len(w.layers)
+    idx_total_ms = (full_ms - reuse_ms) + (ri_ms - reuse_ms)
+    if attn_total_ms >= idx_total_ms:
+        dom = {"kernel": "csa2_sparse_attn (attn_split_kernel + attn_combine_kernel), Reuse layer",
+               "bound": "tensor", "achieved": reuse_flops / (reuse_ms * 1e-3) / 1e12,
+               "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+               "hbm_achieved_gbs": reuse_bytes / (reuse_ms * 1e-3) / 1e9}
+    else:
+        b = bytes_full_idx
+        t = (full_ms - reuse_ms) * 1e-3
+        dom = {"kernel": "csa2_indexer_score_topk (Full: block + pool scoring, two top-k)",
+               "bound": "hbm", "achieved": b / t / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    dom["frac"] = dom["achieved"] / dom["peak"]
+    dom["peak_source"] = peaks["source"]
+    dom["traffic"] = None
+
+    units = len(w.layers) * args.steps * world
+    value = units / (total_ms * 1e-3)
+    ms_per_step = total_ms / args.steps
+    hbm_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
+
+    # --- end to end through the C ABI with host buffers ---
+    e2e = run_e2e(args, w, step, stream, flush)
+    if world > 1:
+        t = torch.tensor([e2e["ms"]], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e["ms"] = float(t.item())
+    e2e_value = len(w.layers) * args.steps * world / (e2e["ms"] * 1e-3)
+
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)",
+        "config": _config_json(w, world),
+        "tokens_per_s": B * world * args.steps / (total_ms * 1e-3),
+        "hbm_gbs_achieved": hbm_gbs, "hbm_frac": hbm_gbs / peaks["hbm_gbs"],
+        "step_algorithmic_bytes": step_bytes,
+        "ms_per_call": {c: float(m) for c, m in zip(calls, mean_call)},
+        "roofline": dom,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
+                "d2h_bytes_per_step": e2e["d2h"]},
+        "gpu_launches": args.steps * launches_per_step(w),
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(args, seqs=tuple(range(w.batch)))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def launches_per_step(w) -> int:
+    n = 2                                   # append: rows + block keys
+    for m in w.layers:
+        n += 2                              # attention: split + combine
+        if m == "F":
+            n += 4                          # block scores, block top-k, pool scores, pool top-k
+        elif m == "RI":
+            n += 2                          # pool scores, top-k
+    return n
+
+
+def run_e2e(args, w, step, stream, flush):
+    """Same step through the C ABI, inputs copied from pinned host memory and the
+    outputs read back every step, all inside the timed region."""
+    import torch
+    host_in = {"new_kv": step.new_kv, "new_k": step.new_k}
+    for i, q in enumerate(step.q):
+        host_in[f"q{i}"] = q
+    for i, q in step.idxq.items():
+        host_in[f"iq{i}"] = q
+    pinned = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in host_in.items()}
+    for k, v in host_in.items():
+        pinned[k].copy_(v)
+    outs = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in step.out]
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+
+    def one():
+        for k, v in host_in.items():
+            v.copy_(pinned[k], non_blocking=True)
+        step.run()
+        for o, h in zip(step.out, outs):
+            h.copy_(o, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        one()
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)
+        ev0[k].record(stream)
+        one()
+        ev1[k].record(stream)
+    torch.cuda.synchronize()
+    ms = sum(ev0[k].elapsed_time(ev1[k]) for k in range(args.steps))
+    return {"ms": ms, "h2d": h2d, "d2h": d2h}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle arm
+# ---------------------------------------------------------------------------
+
+def _oracle_sample(w, seqs):
+    """Host inputs of a bounded sample (whole sequences of the workload)."""
+    import workload as wl
+    from oracle import codec as ocodec
+    L = w.lengths[0]
+    data = []
+    for s in seqs:
+        keys = wl.idxk_rows(w.seed, s, 0, L)
+        kv_bits = wl.kv_rows(w.seed, s, 0, L)
+        iq = {l: wl.idxq_rows(w.seed, l, s) for l, m in enumerate(w.layers) if m in ("F", "RI")}
+        q = {l: wl.q_rows(w.seed, l, s, w.heads) for l in range(len(w.layers))}
+        data.append((keys, kv_bits, iq, q))
+    return data
+
+
+def _oracle_step(w, sample):
+    """The oracle's whole decode step for the sampled sequences: encode the cache
+    rows the step reads, then run the layer schedule."""
+    from oracle import codec as ocodec
+    from oracle import modes as omodes
+    L = w.lengths[0]
+    for keys, kv_bits, iq, q in sample:
+        rows_cache = {}
+
+        def rows(pos, kv_bits=kv_bits, rows_cache=rows_cache):
+            miss = [p for p in pos.tolist() if p not in rows_cache]
+            if miss:
+                enc = ocodec.encode_bf16_rows(kv_bits[np.asarray(miss)])
+                c, s = ocodec.unpack_rows(enc)
+                dec = ocodec.dequantize(c, s)
+                for p, r in zip(miss, dec):
+                    rows_cache[p] = r
+            return np.stack([rows_cache[p] for p in pos.tolist()])
+
+        omodes.run_layers(w.layers, L, keys, lambda l: iq[l], lambda l: q[l], rows)
+
+
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_baseline(args, seqs=(0,)):
+    import workload as wl
+    w = wl.workload(CONFIG_ID)
+    sample = _oracle_sample(w, list(seqs))
+    t0 = time.perf_counter()
+    _oracle_step(w, sample)
+    dt = time.perf_counter() - t0
+    # layer-steps over the whole batch: the sample covers len(seqs) of B sequences
+    per_batch_step = dt * w.batch / len(seqs)
+    scale = "" if len(seqs) == w.batch else f", scaled x{w.batch / len(seqs):g} to the batch"
+    return {"value": len(w.layers) / per_batch_step, "unit": UNIT, "cores": _blas_threads(),
+            "kind": "oracle",
+            "sample": f"{len(seqs)} of {w.batch} sequences, all {len(w.layers)} layers of one step "
+                      f"(indexer + fp64 attention){scale}; {dt:.1f} s of CPU work"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import workload as wl
+    w = wl.workload(CONFIG_ID)
+    seqs = list(range(8))
+    sample = _oracle_sample(w, seqs)
+    for _ in range(args.warmup):
+        _oracle_step(w, sample)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_step(w, sample)
+    dt = time.perf_counter() - t0
+    per_batch_step = dt / args.steps * w.batch / len(seqs)
+    value = len(w.layers) / per_batch_step
+    cores = _blas_threads()
+    result = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_batch_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)", "config": _config_json(w, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{len(seqs)} of {w.batch} sequences per step (all "
+                                   f"{len(w.layers)} layers), scaled x{w.batch // len(seqs)} to the batch"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(result), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,252 @@
+"""Thin Python binding of the CSA2 C ABI (``include/csa2.h``, ``lib/libcsa2.so``).
+
+Argument marshalling only: every function below checks tensor dtypes/devices,
+passes raw device pointers and the current torch CUDA stream to the C entry
+point of the same name, and raises :class:`Csa2Error` on a non-zero status.
+All computation happens in the library's CUDA kernels; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import _build
+
+FULL, REINDEX, REUSE = 0, 1, 2
+OP_INDEXER, OP_ATTENTION = 1, 2
+LATENT_DIM = 512
+ROW_BYTES = 288
+PAGE_TOKENS = 64
+PAGE_BYTES = ROW_BYTES * PAGE_TOKENS
+IDX_PAGE_BYTES = 64 * 128
+BK_PAGE_BYTES = 8 * 128
+TOP_K = 512
+POOL_BLOCKS = 2048
+WINDOW = 128
+
+DEVERR_PAGE, DEVERR_POS, DEVERR_SEQ = 1, 2, 4
+
+
+class Csa2Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class CacheStruct(ctypes.Structure):
+    _fields_ = [
+        ("kv_pool", ctypes.c_void_p),
+        ("idxk_pool", ctypes.c_void_p),
+        ("blockkey_pool", ctypes.c_void_p),
+        ("n_pages", ctypes.c_int64),
+        ("page_table", ctypes.c_void_p),
+        ("max_pages", ctypes.c_int32),
+        ("batch", ctypes.c_int32),
+        ("seq_lens", ctypes.c_void_p),
+        ("error_word", ctypes.c_void_p),
+        ("cache_id", ctypes.c_uint64),
+    ]
+
+
+class IndexSetStruct(ctypes.Structure):
+    _fields_ = [
+        ("idx", ctypes.c_void_p),
+        ("pool_blocks", ctypes.c_void_p),
+        ("rows", ctypes.c_int32),
+        ("layer", ctypes.c_int32),
+        ("mode", ctypes.c_int32),
+        ("pool_layer", ctypes.c_int32),
+        ("cache_id", ctypes.c_uint64),
+        ("nq", ctypes.c_int32),
+    ]
+
+
+# every entry point declared in include/csa2.h, with its ctypes signature
+_VP, _I32, _I64, _F32, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "csa2_indexset_init": (None, [_VP, _VP, _VP, _I32]),
+    "csa2_kv_quant_append": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _I32, _I32, _VP]),
+    "csa2_indexer_score_topk": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _I32, _I64, _I32, _I32, _I32,
+                                               _VP, _VP, _SZ, _VP]),
+    "csa2_sparse_attn": (ctypes.c_int, [_VP, _VP, _I32, _F32, _VP, _VP, _I32, _I32, _I32, _VP, _VP,
+                                        _VP, _SZ, _VP]),
+    "csa2_swa_replay": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP]),
+    "csa2_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I64, _I32]),
+    "csa2_check_device_error": (ctypes.c_int, [_VP, _VP, ctypes.POINTER(ctypes.c_uint32)]),
+    "csa2_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "csa2_version": (ctypes.c_int, []),
+}
+
+_lib = None
+
+
+def lib():
+    """The loaded library.  Raises if it has not been built (no fallback path)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_build.LIB):
+            raise RuntimeError(f"CSA2 CUDA library missing at {_build.LIB}: run "
+                               "__graft_entry__.build() (nvcc, sm_100a) first")
+        l = ctypes.CDLL(_build.LIB)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().csa2_status_string(status).decode()
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise Csa2Error(status, where)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: torch.Tensor | None, dtypes, name: str, numel: int | None = None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype} not in {dtypes}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if numel is not None and t.numel() < numel:
+        raise ValueError(f"{name}: {t.numel()} elements, need {numel}")
+    return t.data_ptr()
+
+
+_BF16 = (torch.bfloat16, torch.int16, torch.uint16)
+_I32T = (torch.int32,)
+
+
+class Cache:
+    """Paged FP4 cache: three page pools, page table, lengths, error word."""
+
+    def __init__(self, n_pages: int, batch: int, max_pages: int, device="cuda", cache_id: int = 1):
+        dev = torch.device(device)
+        self.n_pages, self.batch, self.max_pages = n_pages, batch, max_pages
+        self.kv_pool = torch.zeros(n_pages * PAGE_BYTES, dtype=torch.uint8, device=dev)
+        self.idxk_pool = torch.zeros(n_pages * IDX_PAGE_BYTES, dtype=torch.uint8, device=dev)
+        self.bk_pool = torch.zeros(n_pages * BK_PAGE_BYTES, dtype=torch.uint8, device=dev)
+        self.page_table = torch.full((batch, max_pages), -1, dtype=torch.int32, device=dev)
+        self.seq_lens = torch.zeros(batch, dtype=torch.int32, device=dev)
+        self.error_word = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.cache_id = cache_id
+        self.struct = CacheStruct()
+        self.refresh()
+
+    def refresh(self):
+        s = self.struct
+        s.kv_pool = self.kv_pool.data_ptr()
+        s.idxk_pool = self.idxk_pool.data_ptr()
+        s.blockkey_pool = self.bk_pool.data_ptr()
+        s.n_pages = self.n_pages
+        s.page_table = self.page_table.data_ptr()
+        s.max_pages = self.max_pages
+        s.batch = self.batch
+        s.seq_lens = self.seq_lens.data_ptr()
+        s.error_word = self.error_word.data_ptr()
+        s.cache_id = self.cache_id
+
+    def ref(self):
+        return ctypes.byref(self.struct)
+
+
+class IndexSet:
+    """Device index rows [rows, 512] + pool rows [rows, 2048] and their mode tags."""
+
+    def __init__(self, rows: int, device="cuda"):
+        dev = torch.device(device)
+        self.idx = torch.full((rows, TOP_K), -1, dtype=torch.int32, device=dev)
+        self.pool_blocks = torch.full((rows, POOL_BLOCKS), -1, dtype=torch.int32, device=dev)
+        self.struct = IndexSetStruct()
+        lib().csa2_indexset_init(ctypes.byref(self.struct), self.idx.data_ptr(),
+                                 self.pool_blocks.data_ptr(), rows)
+
+    def ref(self):
+        return ctypes.byref(self.struct)
+
+    @property
+    def layer(self):
+        return self.struct.layer
+
+    @property
+    def mode(self):
+        return self.struct.mode
+
+
+def csa2_workspace_bytes(op: int, nq: int, heads: int = 0, max_visible: int = 0,
+                         hierarchical: bool = True) -> int:
+    return int(lib().csa2_workspace_bytes(op, nq, heads, max_visible, int(bool(hierarchical))))
+
+
+def csa2_kv_quant_append(cache: Cache, kv: torch.Tensor, idxk: torch.Tensor, entry_seq: torch.Tensor,
+                         entry_pos: torch.Tensor, compress: int = 1, stream=None):
+    n = entry_seq.numel()
+    if entry_pos.numel() != n:
+        raise ValueError("entry_seq and entry_pos differ in length")
+    st = lib().csa2_kv_quant_append(
+        cache.ref(), _ptr(kv, _BF16, "kv", n * compress * LATENT_DIM),
+        _ptr(idxk, _BF16, "idxk", n * compress * 64), _ptr(entry_seq, _I32T, "entry_seq"),
+        _ptr(entry_pos, _I32T, "entry_pos"), n, compress, _stream(stream))
+    _check(st, "csa2_kv_quant_append")
+
+
+def csa2_indexer_score_topk(cache: Cache, idx_q: torch.Tensor, q_seq: torch.Tensor, mode: int,
+                            layer: int, indexset: IndexSet, workspace: torch.Tensor, max_visible: int,
+                            q_visible: torch.Tensor | None = None, head_w: torch.Tensor | None = None,
+                            hierarchical: bool = True, stream=None):
+    nq = q_seq.numel()
+    st = lib().csa2_indexer_score_topk(
+        cache.ref(), _ptr(idx_q, _BF16, "idx_q", nq * 256),
+        _ptr(head_w, (torch.float32,), "head_w", nq * 4), _ptr(q_seq, _I32T, "q_seq"),
+        _ptr(q_visible, _I32T, "q_visible", nq), nq, int(max_visible), mode, int(bool(hierarchical)),
+        layer, indexset.ref(), _ptr(workspace, (torch.uint8,), "workspace"),
+        workspace.numel(), _stream(stream))
+    _check(st, "csa2_indexer_score_topk")
+
+
+def csa2_sparse_attn(cache: Cache, q: torch.Tensor, q_seq: torch.Tensor, mode: int, layer: int,
+                     indexset: IndexSet, out: torch.Tensor, workspace: torch.Tensor,
+                     sm_scale: float = 1.0, q_visible: torch.Tensor | None = None, stream=None):
+    nq = q_seq.numel()
+    heads = q.shape[-2]
+    st = lib().csa2_sparse_attn(
+        cache.ref(), _ptr(q, _BF16, "q", nq * heads * LATENT_DIM), heads, float(sm_scale),
+        _ptr(q_seq, _I32T, "q_seq"), _ptr(q_visible, _I32T, "q_visible", nq), nq, mode, layer,
+        indexset.ref(), _ptr(out, _BF16, "out", nq * heads * LATENT_DIM),
+        _ptr(workspace, (torch.uint8,), "workspace"), workspace.numel(), _stream(stream))
+    _check(st, "csa2_sparse_attn")
+
+
+def csa2_swa_replay(cache: Cache, kv_last: torch.Tensor, idxk_last: torch.Tensor, miss: torch.Tensor,
+                    stream=None):
+    b = cache.batch
+    st = lib().csa2_swa_replay(
+        cache.ref(), _ptr(kv_last, _BF16, "kv_last", b * 128 * LATENT_DIM),
+        _ptr(idxk_last, _BF16, "idxk_last", b * 128 * 64),
+        _ptr(miss, (torch.uint8, torch.bool), "miss", b), _stream(stream))
+    _check(st, "csa2_swa_replay")
+
+
+def csa2_check_device_error(cache: Cache, stream=None) -> int:
+    """Synchronise, read and clear the cache's device error word; returns its bits."""
+    bits = ctypes.c_uint32(0)
+    st = lib().csa2_check_device_error(cache.ref(), _stream(stream), ctypes.byref(bits))
+    if st not in (0, 7):
+        raise Csa2Error(st, "csa2_check_device_error")
+    return int(bits.value)

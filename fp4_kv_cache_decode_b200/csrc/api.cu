@@ -1,0 +1,270 @@
+// C ABI of the CSA2 library: host-side validation, mode-order checks and
+// kernel launches.  No allocation, no host synchronisation (except in
+// csa2_check_device_error); every launch goes to the caller's stream.
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace csa2 {
+cudaError_t launch_append(const CacheView&, const uint16_t*, const uint16_t*, const int32_t*,
+                          const int32_t*, int, int, cudaStream_t);
+cudaError_t launch_replay(const CacheView&, const uint16_t*, const uint16_t*, const uint8_t*,
+                          cudaStream_t);
+cudaError_t launch_score(int, const CacheView&, const uint16_t*, const float*, const int32_t*,
+                         const int32_t*, const int32_t*, int, int64_t, int64_t, float*, cudaStream_t);
+cudaError_t launch_topk(int, const CacheView&, const float*, int64_t, const int32_t*, const int32_t*,
+                        const int32_t*, int, int, int32_t*, int64_t, cudaStream_t);
+cudaError_t indexer_set_attributes();
+cudaError_t attention_set_attributes();
+size_t attn_workspace_bytes(int nq, int H);
+cudaError_t launch_attention(const CacheView&, const uint16_t*, int, float, const int32_t*,
+                             const int32_t*, const int32_t*, int, uint16_t*, void*, cudaStream_t);
+}  // namespace csa2
+
+using namespace csa2;
+
+namespace {
+
+constexpr int kSrcFlat = 0, kSrcBlockKeys = 1, kSrcPool = 2;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Kernel attributes (dynamic shared-memory opt-in) are per device: set once.
+int ensure_device_setup() {
+  static std::mutex mu;
+  static bool done[128] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return CSA2_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done[dev]) {
+    if (indexer_set_attributes() != cudaSuccess) return CSA2_ERR_CUDA;
+    if (attention_set_attributes() != cudaSuccess) return CSA2_ERR_CUDA;
+    done[dev] = true;
+  }
+  return CSA2_OK;
+}
+
+int make_view(const csa2_cache* c, CacheView* v) {
+  if (c == nullptr) return CSA2_ERR_INVALID_ARG;
+  if (!c->kv_pool || !c->idxk_pool || !c->blockkey_pool || !c->page_table || !c->seq_lens ||
+      !c->error_word)
+    return CSA2_ERR_INVALID_ARG;
+  if (c->n_pages <= 0 || c->max_pages <= 0 || c->batch <= 0) return CSA2_ERR_SHAPE;
+  if (c->n_pages > ((int64_t)1 << 31)) return CSA2_ERR_SHAPE;
+  if (!aligned(c->kv_pool, 16) || !aligned(c->idxk_pool, 16) || !aligned(c->blockkey_pool, 16) ||
+      !aligned(c->page_table, 4) || !aligned(c->seq_lens, 4) || !aligned(c->error_word, 4))
+    return CSA2_ERR_ALIGNMENT;
+  v->kv = static_cast<uint8_t*>(c->kv_pool);
+  v->idxk = static_cast<uint8_t*>(c->idxk_pool);
+  v->bk = static_cast<uint8_t*>(c->blockkey_pool);
+  v->n_pages = c->n_pages;
+  v->pt = c->page_table;
+  v->max_pages = c->max_pages;
+  v->batch = c->batch;
+  v->seq_lens = c->seq_lens;
+  v->err = c->error_word;
+  return CSA2_OK;
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Score-buffer stride (floats per query) of an indexer call.
+int64_t indexer_stride(int64_t max_visible, int hierarchical) {
+  const int64_t nb = ceil_div(max_visible, kBlock);
+  if (hierarchical) {
+    const int64_t bk = ceil_div(nb, kBlocksPerPage) * kBlocksPerPage;
+    const int64_t pool = (int64_t)kPoolBlocks * kBlock;
+    return bk > pool ? bk : pool;
+  }
+  return nb * kBlock;
+}
+
+}  // namespace
+
+extern "C" {
+
+void csa2_indexset_init(csa2_indexset* set, int32_t* idx, int32_t* pool_blocks, int32_t rows) {
+  if (!set) return;
+  set->idx = idx;
+  set->pool_blocks = pool_blocks;
+  set->rows = rows;
+  set->layer = -1;
+  set->mode = -1;
+  set->pool_layer = -1;
+  set->cache_id = 0;
+  set->nq = 0;
+}
+
+int csa2_kv_quant_append(const csa2_cache* cache, const uint16_t* kv, const uint16_t* idxk,
+                         const int32_t* entry_seq, const int32_t* entry_pos, int32_t n,
+                         int32_t compress, csa2_stream_t stream) {
+  CacheView v;
+  int st = make_view(cache, &v);
+  if (st) return st;
+  if (n < 0) return CSA2_ERR_INVALID_ARG;
+  if (compress != 1 && compress != 2) return CSA2_ERR_SHAPE;
+  if (n == 0) return CSA2_OK;
+  if (!kv || !idxk || !entry_seq || !entry_pos) return CSA2_ERR_INVALID_ARG;
+  if (!aligned(kv, 16) || !aligned(idxk, 4) || !aligned(entry_seq, 4) || !aligned(entry_pos, 4))
+    return CSA2_ERR_ALIGNMENT;
+  return from_cuda(launch_append(v, kv, idxk, entry_seq, entry_pos, n, compress, (cudaStream_t)stream));
+}
+
+int csa2_indexer_score_topk(const csa2_cache* cache, const uint16_t* idx_q, const float* head_w,
+                            const int32_t* q_seq, const int32_t* q_visible, int32_t nq,
+                            int64_t max_visible, int32_t mode, int32_t hierarchical, int32_t layer,
+                            csa2_indexset* set, void* workspace, size_t workspace_bytes,
+                            csa2_stream_t stream) {
+  CacheView v;
+  int st = make_view(cache, &v);
+  if (st) return st;
+  if (mode != CSA2_FULL && mode != CSA2_REINDEX) return CSA2_ERR_INVALID_ARG;
+  if (nq < 0 || max_visible < 0 || max_visible > ((int64_t)1 << 31) - 1 || layer < 0)
+    return CSA2_ERR_INVALID_ARG;
+  if (!set || !set->idx) return CSA2_ERR_INVALID_ARG;
+  if (nq > set->rows) return CSA2_ERR_SHAPE;
+  const bool hier = hierarchical != 0 || mode == CSA2_REINDEX;
+  if (hier && !set->pool_blocks) return CSA2_ERR_INVALID_ARG;
+  if (mode == CSA2_REINDEX) {
+    // Reindex ranks the pool of the last hierarchical Full layer on this cache
+    if (set->pool_layer < 0 || set->pool_layer >= layer || set->cache_id != cache->cache_id ||
+        nq > set->nq)
+      return CSA2_ERR_MODE_STATE;
+  }
+  if (nq > 0 && (!idx_q || !q_seq)) return CSA2_ERR_INVALID_ARG;
+  if (!aligned(idx_q, 16) || !aligned(head_w, 4) || !aligned(q_seq, 4) || !aligned(q_visible, 4) ||
+      !aligned(set->idx, 4) || !aligned(set->pool_blocks, 4))
+    return CSA2_ERR_ALIGNMENT;
+  const size_t need = csa2_workspace_bytes(CSA2_OP_INDEXER, nq, 0, max_visible, hier ? 1 : 0);
+  if (nq > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16)))
+    return CSA2_ERR_WORKSPACE;
+  if (nq > 0) {
+    if ((st = ensure_device_setup())) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    float* scores = static_cast<float*>(workspace);
+    const int64_t stride = indexer_stride(max_visible, hier ? 1 : 0);
+    const int64_t nb = ceil_div(max_visible, kBlock);
+    cudaError_t e = cudaSuccess;
+    if (mode == CSA2_FULL && hier) {
+      const int64_t bk_units = ceil_div(nb, kBlocksPerPage);
+      e = launch_score(kSrcBlockKeys, v, idx_q, head_w, q_seq, q_visible, nullptr, nq, bk_units,
+                       stride, scores, s);
+      if (e == cudaSuccess)
+        e = launch_topk(kSrcBlockKeys, v, scores, stride, q_seq, q_visible, nullptr, nq,
+                        kPoolBlocks, set->pool_blocks, kPoolBlocks, s);
+    }
+    if (e == cudaSuccess && hier) {
+      e = launch_score(kSrcPool, v, idx_q, head_w, q_seq, q_visible, set->pool_blocks, nq,
+                       kPoolBlocks, stride, scores, s);
+      if (e == cudaSuccess)
+        e = launch_topk(kSrcPool, v, scores, stride, q_seq, q_visible, set->pool_blocks, nq, kTopK,
+                        set->idx, kTopK, s);
+    }
+    if (e == cudaSuccess && !hier) {
+      e = launch_score(kSrcFlat, v, idx_q, head_w, q_seq, q_visible, nullptr, nq, nb, stride,
+                       scores, s);
+      if (e == cudaSuccess)
+        e = launch_topk(kSrcFlat, v, scores, stride, q_seq, q_visible, nullptr, nq, kTopK, set->idx,
+                        kTopK, s);
+    }
+    if (e != cudaSuccess) return CSA2_ERR_CUDA;
+  }
+  set->layer = layer;
+  set->mode = mode;
+  set->cache_id = cache->cache_id;
+  if (mode == CSA2_FULL) {
+    set->nq = nq;
+    set->pool_layer = hier ? layer : -1;
+  }
+  return CSA2_OK;
+}
+
+int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int32_t heads, float sm_scale,
+                     const int32_t* q_seq, const int32_t* q_visible, int32_t nq, int32_t mode,
+                     int32_t layer, const csa2_indexset* set, uint16_t* out, void* workspace,
+                     size_t workspace_bytes, csa2_stream_t stream) {
+  CacheView v;
+  int st = make_view(cache, &v);
+  if (st) return st;
+  if (mode != CSA2_FULL && mode != CSA2_REINDEX && mode != CSA2_REUSE) return CSA2_ERR_INVALID_ARG;
+  if (heads != 16 && heads != 32 && heads != 48 && heads != 64) return CSA2_ERR_SHAPE;
+  if (nq < 0 || layer < 0 || !set || !set->idx) return CSA2_ERR_INVALID_ARG;
+  if (nq > set->rows) return CSA2_ERR_SHAPE;
+  if (set->cache_id != cache->cache_id || set->layer < 0 || nq > set->nq) return CSA2_ERR_MODE_STATE;
+  if (mode == CSA2_REUSE) {
+    // Reuse consumes the latest Full / Reindex indices of an earlier layer
+    if (set->layer >= layer || (set->mode != CSA2_FULL && set->mode != CSA2_REINDEX))
+      return CSA2_ERR_MODE_STATE;
+  } else if (set->layer != layer || set->mode != mode) {
+    return CSA2_ERR_MODE_STATE;   // Full / Reindex attend over their own fresh set
+  }
+  if (nq > 0 && (!q || !q_seq || !out)) return CSA2_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(q_seq, 4) || !aligned(q_visible, 4))
+    return CSA2_ERR_ALIGNMENT;
+  const size_t need = csa2_workspace_bytes(CSA2_OP_ATTENTION, nq, heads, 0, 0);
+  if (nq > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16)))
+    return CSA2_ERR_WORKSPACE;
+  if (nq == 0) return CSA2_OK;
+  if ((st = ensure_device_setup())) return st;
+  return from_cuda(launch_attention(v, q, heads, sm_scale, q_seq, q_visible, set->idx, nq, out,
+                                    workspace, (cudaStream_t)stream));
+}
+
+int csa2_swa_replay(const csa2_cache* cache, const uint16_t* kv_last, const uint16_t* idxk_last,
+                    const uint8_t* miss, csa2_stream_t stream) {
+  CacheView v;
+  int st = make_view(cache, &v);
+  if (st) return st;
+  if (!kv_last || !idxk_last || !miss) return CSA2_ERR_INVALID_ARG;
+  if (!aligned(kv_last, 16) || !aligned(idxk_last, 4)) return CSA2_ERR_ALIGNMENT;
+  return from_cuda(launch_replay(v, kv_last, idxk_last, miss, (cudaStream_t)stream));
+}
+
+size_t csa2_workspace_bytes(int32_t op, int32_t nq, int32_t heads, int64_t max_visible,
+                            int32_t hierarchical) {
+  if (nq < 0) return 0;
+  if (op == CSA2_OP_INDEXER) {
+    if (max_visible < 0) return 0;
+    return (size_t)nq * (size_t)indexer_stride(max_visible, hierarchical ? 1 : 0) * sizeof(float) + 256;
+  }
+  if (op == CSA2_OP_ATTENTION) {
+    if (heads != 16 && heads != 32 && heads != 48 && heads != 64) return 0;
+    return attn_workspace_bytes(nq, heads);
+  }
+  return 0;
+}
+
+int csa2_check_device_error(const csa2_cache* cache, csa2_stream_t stream, uint32_t* bits) {
+  if (!cache || !cache->error_word) return CSA2_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint32_t h = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return CSA2_ERR_CUDA;
+  if (cudaMemcpyAsync(&h, cache->error_word, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return CSA2_ERR_CUDA;
+  if (cudaMemsetAsync(cache->error_word, 0, sizeof(uint32_t), s) != cudaSuccess) return CSA2_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return CSA2_ERR_CUDA;
+  if (bits) *bits = h;
+  return h ? CSA2_ERR_DEVICE_BOUNDS : CSA2_OK;
+}
+
+const char* csa2_status_string(int status) {
+  switch (status) {
+    case CSA2_OK: return "ok";
+    case CSA2_ERR_INVALID_ARG: return "invalid argument";
+    case CSA2_ERR_SHAPE: return "unsupported shape";
+    case CSA2_ERR_ALIGNMENT: return "misaligned pointer";
+    case CSA2_ERR_MODE_STATE: return "layer mode called out of order";
+    case CSA2_ERR_WORKSPACE: return "workspace missing or too small";
+    case CSA2_ERR_CUDA: return "CUDA error";
+    case CSA2_ERR_DEVICE_BOUNDS: return "kernel found an out-of-range page, position or sequence";
+    default: return "unknown status";
+  }
+}
+
+int csa2_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,227 @@
+// FP4 main-KV encoder (csa2_kv_quant_append, csa2_swa_replay) and block keys.
+//
+// Codec: E2M1 codes with one E4M3 scale per 16 channels and no global scale
+// (agentnet.co.il, "דיפסיק משיקה את V4.1-פלאש ...", section "קוונטיזציה ופריסה:
+// FP4 ו-DRAM במקום SSD").  One warp encodes one 512-channel row: lane l owns
+// scale group l (channels 16l..16l+15), so the group maximum needs no
+// cross-lane traffic; the 32 lanes' 8-byte code words form the row's 256
+// code bytes in one coalesced 256-B store, their scale bytes the 32-B tail.
+//
+// Rounding is decided exactly:
+//  * scale: fp32 amax/6 (IEEE division) then the hardware's round-to-nearest-
+//    even, saturating E4M3 conversion.  For inputs with at most 24 significant
+//    bits the correctly rounded quotient can neither reach nor cross an E4M3
+//    midpoint that the exact quotient does not, so this equals rounding the
+//    exact amax/6;
+//  * code: |x| compared with midpoint x scale for the 7 E2M1 midpoints; each
+//    product has at most 7 significant bits and is exact in fp32, so this is
+//    the exact nearest-even rounding of |x|/scale, saturating at 6.
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+
+namespace csa2 {
+
+struct GroupCode {
+  uint2 codes;    // 16 nibbles, channel 2j of the group in the low nibble of byte j
+  uint32_t scale; // E4M3 byte
+};
+
+// Encode the 16 values of one scale group.
+__device__ __forceinline__ GroupCode encode_group(const float (&x)[16]) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(x[j]));
+  const float q = __fdiv_rn(amax, 6.0f);
+  const uint32_t sb = (uint32_t)__nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3) & 0x7Fu;
+  const float s = e4m3_pos_value(sb);
+  GroupCode g;
+  g.scale = sb;
+  uint32_t w[2] = {0u, 0u};
+  if (s != 0.0f) {
+    // midpoints of the E2M1 magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}, scaled (exact)
+    const float t0 = 0.25f * s, t1 = 0.75f * s, t2 = 1.25f * s, t3 = 1.75f * s;
+    const float t4 = 2.5f * s, t5 = 3.5f * s, t6 = 5.0f * s;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float a = fabsf(x[j]);
+      uint32_t below = (t0 < a) + (t1 < a) + (t2 < a) + (t3 < a) + (t4 < a) + (t5 < a) + (t6 < a);
+      const bool tie = (a == t0) | (a == t1) | (a == t2) | (a == t3) | (a == t4) | (a == t5) |
+                       (a == t6);
+      below += (tie && (below & 1u)) ? 1u : 0u;
+      const uint32_t code = below | ((__float_as_uint(x[j]) >> 31) << 3);
+      w[j >> 3] |= code << ((j & 7) * 4);
+    }
+  }
+  g.codes = make_uint2(w[0], w[1]);
+  return g;
+}
+
+// Unpack 8 bf16 values from a 16-B word.
+__device__ __forceinline__ void unpack8(const uint4& v, float* out) {
+  out[0] = bf16_lo(v.x); out[1] = bf16_hi(v.x);
+  out[2] = bf16_lo(v.y); out[3] = bf16_hi(v.y);
+  out[4] = bf16_lo(v.z); out[5] = bf16_hi(v.z);
+  out[6] = bf16_lo(v.w); out[7] = bf16_hi(v.w);
+}
+
+// One warp: encode input row(s) `src` (compress 1 or 2 consecutive bf16 rows of
+// 512) into the cache row at (seq, pos), and store the indexer key.
+__device__ __forceinline__ void encode_entry_warp(const CacheView& c, int lane,
+                                                 const uint16_t* __restrict__ kv_src,
+                                                 const uint16_t* __restrict__ idxk_src,
+                                                 int compress, int seq, int64_t pos) {
+  const int64_t page = page_of(c, seq, pos);
+  if (page < 0) return;
+  float x[16];
+  {
+    const uint4* r0 = reinterpret_cast<const uint4*>(kv_src) + lane * 2;
+    unpack8(__ldg(r0), x);
+    unpack8(__ldg(r0 + 1), x + 8);
+    if (compress == 2) {
+      float y[16];
+      const uint4* r1 = reinterpret_cast<const uint4*>(kv_src + kD) + lane * 2;
+      unpack8(__ldg(r1), y);
+      unpack8(__ldg(r1 + 1), y + 8);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) x[j] = __fmul_rn(__fadd_rn(x[j], y[j]), 0.5f);
+    }
+  }
+  const GroupCode g = encode_group(x);
+  uint8_t* row = c.kv + page * kPageBytes + (pos & (kPageTokens - 1)) * kRowBytes;
+  reinterpret_cast<uint2*>(row)[lane] = g.codes;
+  row[kCodeBytes + lane] = (uint8_t)g.scale;
+
+  // indexer key: lane owns dims 2*lane, 2*lane+1
+  uint32_t kw = __ldg(reinterpret_cast<const uint32_t*>(idxk_src) + lane);
+  if (compress == 2) {
+    const uint32_t kw2 = __ldg(reinterpret_cast<const uint32_t*>(idxk_src + kIdxDim) + lane);
+    const float a = __fmul_rn(__fadd_rn(bf16_lo(kw), bf16_lo(kw2)), 0.5f);
+    const float b = __fmul_rn(__fadd_rn(bf16_hi(kw), bf16_hi(kw2)), 0.5f);
+    kw = (uint32_t)f32_to_bf16_rne(a) | ((uint32_t)f32_to_bf16_rne(b) << 16);
+  }
+  uint8_t* krow = c.idxk + page * kIdxPageBytes + (pos & (kPageTokens - 1)) * kIdxRowBytes;
+  reinterpret_cast<uint32_t*>(krow)[lane] = kw;
+}
+
+// One warp: recompute the block key of block `blk` of sequence `seq` from the
+// stored keys of its present tokens [8*blk, min(8*blk+8, len)).
+__device__ __forceinline__ void block_key_warp(const CacheView& c, int lane, int seq, int64_t blk,
+                                               int64_t len) {
+  const int64_t t0 = blk * kBlock;
+  if (t0 >= len || t0 < 0) return;
+  const int64_t page = page_of(c, seq, t0);
+  if (page < 0) return;
+  const int64_t t1 = min(t0 + kBlock, len);
+  const uint8_t* kp = c.idxk + page * kIdxPageBytes;
+  float a = 0.0f, b = 0.0f;
+  for (int64_t t = t0; t < t1; ++t) {
+    const uint32_t w = reinterpret_cast<const uint32_t*>(kp + (t & (kPageTokens - 1)) * kIdxRowBytes)[lane];
+    a = __fadd_rn(a, bf16_lo(w));
+    b = __fadd_rn(b, bf16_hi(w));
+  }
+  const float n = (float)(t1 - t0);
+  const uint32_t out = (uint32_t)f32_to_bf16_rne(__fdiv_rn(a, n)) |
+                       ((uint32_t)f32_to_bf16_rne(__fdiv_rn(b, n)) << 16);
+  uint8_t* dst = c.bk + page * kBkPageBytes + (blk & (kBlocksPerPage - 1)) * kIdxRowBytes;
+  reinterpret_cast<uint32_t*>(dst)[lane] = out;
+}
+
+constexpr int kWarpsPerCta = 8;
+
+__global__ void __launch_bounds__(256) append_rows_kernel(CacheView c, const uint16_t* __restrict__ kv,
+                                                          const uint16_t* __restrict__ idxk,
+                                                          const int32_t* __restrict__ eseq,
+                                                          const int32_t* __restrict__ epos, int n,
+                                                          int compress) {
+  const int lane = threadIdx.x & 31;
+  const int i = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+  if (i >= n) return;
+  const int seq = eseq[i];
+  const int64_t pos = epos[i];
+  if (seq < 0 || seq >= c.batch) {
+    if (lane == 0) raise_error(c.err, CSA2_DEVERR_SEQ);
+    return;
+  }
+  if (pos < 0 || pos >= c.seq_lens[seq]) {
+    if (lane == 0) raise_error(c.err, CSA2_DEVERR_POS);
+    return;
+  }
+  encode_entry_warp(c, lane, kv + (int64_t)i * compress * kD, idxk + (int64_t)i * compress * kIdxDim,
+                    compress, seq, pos);
+}
+
+// Block keys of the blocks touched by an append.  Entry i recomputes its
+// block unless entry i-1 touched the same block (the usual contiguous case);
+// a block listed twice non-contiguously is recomputed twice to the same value.
+__global__ void __launch_bounds__(256) append_block_keys_kernel(CacheView c,
+                                                                const int32_t* __restrict__ eseq,
+                                                                const int32_t* __restrict__ epos,
+                                                                int n) {
+  const int lane = threadIdx.x & 31;
+  const int i = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+  if (i >= n) return;
+  const int seq = eseq[i];
+  const int64_t pos = epos[i];
+  if (seq < 0 || seq >= c.batch || pos < 0) return;
+  const int64_t len = c.seq_lens[seq];
+  if (pos >= len) return;
+  const int64_t blk = pos / kBlock;
+  if (i > 0 && eseq[i - 1] == seq && epos[i - 1] >= 0 && epos[i - 1] / kBlock == blk) return;
+  block_key_warp(c, lane, seq, blk, len);
+}
+
+// Replay: warp (b, r) handles row r of the supplied last-128 block of seq b.
+__global__ void __launch_bounds__(256) replay_rows_kernel(CacheView c, const uint16_t* __restrict__ kv_last,
+                                                          const uint16_t* __restrict__ idxk_last,
+                                                          const uint8_t* __restrict__ miss) {
+  const int lane = threadIdx.x & 31;
+  const int b = blockIdx.y;
+  const int r = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+  if (r >= kReplay) return;
+  const int64_t len = c.seq_lens[b];
+  const int64_t nrep = miss[b] ? (len < kReplay ? len : (int64_t)kReplay) : (len > 0 ? 1 : 0);
+  if (r < kReplay - nrep) return;
+  const int64_t pos = len - kReplay + r;
+  const int64_t row = (int64_t)b * kReplay + r;
+  encode_entry_warp(c, lane, kv_last + row * kD, idxk_last + row * kIdxDim, 1, b, pos);
+}
+
+// Replay block keys: warp (b, j) recomputes the j-th block touched in seq b.
+__global__ void __launch_bounds__(256) replay_block_keys_kernel(CacheView c, const uint8_t* __restrict__ miss) {
+  const int lane = threadIdx.x & 31;
+  const int b = blockIdx.y;
+  const int j = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+  const int64_t len = c.seq_lens[b];
+  const int64_t nrep = miss[b] ? (len < kReplay ? len : (int64_t)kReplay) : (len > 0 ? 1 : 0);
+  if (nrep == 0) return;
+  const int64_t first = (len - nrep) / kBlock, last = (len - 1) / kBlock;
+  if (first + j > last) return;
+  block_key_warp(c, lane, b, first + j, len);
+}
+
+}  // namespace csa2
+
+// ---- launchers used by api.cu ----
+namespace csa2 {
+
+cudaError_t launch_append(const CacheView& c, const uint16_t* kv, const uint16_t* idxk,
+                          const int32_t* eseq, const int32_t* epos, int n, int compress,
+                          cudaStream_t st) {
+  const int grid = (n + kWarpsPerCta - 1) / kWarpsPerCta;
+  append_rows_kernel<<<grid, 256, 0, st>>>(c, kv, idxk, eseq, epos, n, compress);
+  append_block_keys_kernel<<<grid, 256, 0, st>>>(c, eseq, epos, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_replay(const CacheView& c, const uint16_t* kv_last, const uint16_t* idxk_last,
+                          const uint8_t* miss, cudaStream_t st) {
+  dim3 g1(kReplay / kWarpsPerCta, c.batch);
+  replay_rows_kernel<<<g1, 256, 0, st>>>(c, kv_last, idxk_last, miss);
+  // a 128-token window touches at most 17 blocks of 8
+  dim3 g2((kReplay / kBlock + 1 + kWarpsPerCta - 1) / kWarpsPerCta, c.batch);
+  replay_block_keys_kernel<<<g2, 256, 0, st>>>(c, miss);
+  return cudaGetLastError();
+}
+
+}  // namespace csa2

@@ -1,0 +1,226 @@
+/*
+ * csa2.h -- C ABI of the CSA2 step over an FP4 KV cache (B200, sm_100a).
+ *
+ * CSA2 ("Compressed Sparse Attention 2") as described for DeepSeek-V4.1-Flash:
+ * every layer attends over 512 indices chosen by a lightweight indexer plus a
+ * 128-token sliding window; layers run in one of three static modes (Full,
+ * Reindex, Reuse) that share the main KV and the indexer keys across layers;
+ * the main KV is stored as E2M1 codes with one E4M3 scale per 16 channels
+ * (agentnet.co.il, "דיפסיק משיקה את V4.1-פלאש ...", sections "CSA2: דחיסה
+ * לאורך ציר השכבות" and "קוונטיזציה ופריסה: FP4 ו-DRAM במקום SSD"; ai-wave.ru,
+ * "DeepSeek V4.1-Flash: 1M контекст, FP4 KV-кэш ...", second to fourth
+ * paragraphs).
+ *
+ * Conventions for every call
+ * --------------------------
+ * - All tensor arguments are DEVICE pointers owned by the caller; the library
+ *   allocates no memory.  Scratch space comes from a caller workspace sized by
+ *   csa2_workspace_bytes().
+ * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *   default stream), performs no host synchronisation and no allocation, and
+ *   can be captured in a CUDA graph.  csa2_check_device_error() is the only
+ *   call that synchronises.
+ * - bf16 tensors are passed as uint16_t bit patterns.
+ * - Return value: CSA2_OK or a csa2_status error.  Argument, shape, alignment,
+ *   workspace and mode-order errors are detected on the host before anything is
+ *   launched (nothing is enqueued then).  Out-of-range page ids, positions or
+ *   sequence ids found by a kernel are not faults: the kernel skips that row,
+ *   ORs a CSA2_DEVERR_* bit into cache->error_word, and the host sees it through
+ *   csa2_check_device_error().
+ *
+ * Cache layout in HBM (all pools indexed by the same page id)
+ * ----------------------------------------------------------
+ * - kv_pool:       page p holds 64 token rows of 288 B at p*18432 + slot*288.
+ *                  Row = 256 B of E2M1 codes (channel 2j in the low nibble of
+ *                  byte j, channel 2j+1 in the high nibble) followed by 32 E4M3
+ *                  scale bytes (scale g covers channels 16g..16g+15).
+ * - idxk_pool:     page p holds 64 indexer keys, bf16 [64][64], 8192 B/page.
+ * - blockkey_pool: page p holds the 8 block keys of its 8-token blocks,
+ *                  bf16 [8][64], 1024 B/page.
+ * - page_table[b*max_pages + i] = page id of tokens 64i..64i+63 of sequence b.
+ * Positions are entry positions (after 2:1 compression, for ratio-2 caches).
+ */
+#ifndef CSA2_H
+#define CSA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* csa2_stream_t; /* == cudaStream_t */
+
+/* ---- constants of the method ---- */
+#define CSA2_LATENT_DIM 512       /* channels of the shared K = V latent            */
+#define CSA2_SCALE_GROUP 16       /* channels per E4M3 scale                        */
+#define CSA2_ROW_BYTES 288        /* 256 code bytes + 32 scale bytes per token      */
+#define CSA2_PAGE_TOKENS 64
+#define CSA2_IDX_HEADS 4          /* indexer query heads                            */
+#define CSA2_IDX_DIM 64           /* indexer head dim == shared indexer key dim     */
+#define CSA2_BLOCK_TOKENS 8       /* tokens per indexer block                       */
+#define CSA2_POOL_BLOCKS 2048     /* blocks in the hierarchical candidate pool      */
+#define CSA2_TOP_K 512            /* indices selected per query                     */
+#define CSA2_WINDOW 128           /* sliding-window length                          */
+#define CSA2_REPLAY 128           /* tokens recomputed by bounded replay            */
+
+typedef enum {
+  CSA2_OK = 0,
+  CSA2_ERR_INVALID_ARG = 1,   /* NULL pointer, bad enum, negative count       */
+  CSA2_ERR_SHAPE = 2,         /* unsupported size (heads, compress, ...)      */
+  CSA2_ERR_ALIGNMENT = 3,     /* pointer not 16-byte aligned where required   */
+  CSA2_ERR_MODE_STATE = 4,    /* layer modes called out of order              */
+  CSA2_ERR_WORKSPACE = 5,     /* workspace missing or too small               */
+  CSA2_ERR_CUDA = 6,          /* a CUDA launch or runtime call failed         */
+  CSA2_ERR_DEVICE_BOUNDS = 7  /* a kernel found an out-of-range id (see bits) */
+} csa2_status;
+
+typedef enum { CSA2_FULL = 0, CSA2_REINDEX = 1, CSA2_REUSE = 2 } csa2_mode;
+
+typedef enum { CSA2_OP_INDEXER = 1, CSA2_OP_ATTENTION = 2 } csa2_op;
+
+/* bits OR-ed into *error_word by kernels */
+#define CSA2_DEVERR_PAGE 1u  /* page id outside [0, n_pages) or page slot >= max_pages */
+#define CSA2_DEVERR_POS 2u   /* position/index outside the sequence's visible length   */
+#define CSA2_DEVERR_SEQ 4u   /* sequence id outside [0, batch)                         */
+
+/* Paged cache; every pointer is device memory owned by the caller. */
+typedef struct {
+  void* kv_pool;              /* n_pages * 18432 B, 16-B aligned               */
+  void* idxk_pool;            /* n_pages * 8192 B, 16-B aligned                */
+  void* blockkey_pool;        /* n_pages * 1024 B, 16-B aligned                */
+  int64_t n_pages;
+  const int32_t* page_table;  /* int32 [batch][max_pages]                      */
+  int32_t max_pages;
+  int32_t batch;
+  const int32_t* seq_lens;    /* int32 [batch]: entries present per sequence   */
+  uint32_t* error_word;       /* one uint32, zeroed by the caller              */
+  uint64_t cache_id;          /* caller-chosen identity used by mode checks    */
+} csa2_cache;
+
+/* Index sets produced by the indexer and consumed by attention.  Device
+ * buffers are caller-owned; the tags are host-side state kept by the library
+ * to enforce the Full -> Reindex -> Reuse order. */
+typedef struct {
+  int32_t* idx;          /* int32 [rows][512]: positions, ascending, -1 padded      */
+  int32_t* pool_blocks;  /* int32 [rows][2048]: candidate blocks, ascending, -1 pad */
+  int32_t rows;          /* capacity in queries                                     */
+  int32_t layer;         /* layer whose indexer call last wrote idx (-1: none)      */
+  int32_t mode;          /* CSA2_FULL or CSA2_REINDEX: mode of that call            */
+  int32_t pool_layer;    /* layer whose hierarchical Full call wrote pool_blocks    */
+  uint64_t cache_id;     /* cache the sets were computed on                         */
+  int32_t nq;            /* queries written by the last indexer call                */
+} csa2_indexset;
+
+/* Reset an index set's tags (no device work). */
+void csa2_indexset_init(csa2_indexset* set, int32_t* idx, int32_t* pool_blocks, int32_t rows);
+
+/*
+ * csa2_kv_quant_append -- write new entries into the FP4 cache.
+ *
+ * Defines the main-KV codec (agentnet.co.il, section "קוונטיזציה ופריסה: FP4
+ * ו-DRAM במקום SSD": E2M1 with one E4M3 scale per 16 channels, no global
+ * scale) and the encoder's compression ratio 2 (same page, section "CSA2:
+ * דחיסה לאורך ציר השכבות").  Entry i is built from input rows
+ * [compress*i, compress*i + compress) of kv (bf16 [compress*n][512]) and idxk
+ * (bf16 [compress*n][64]); with compress == 2 the pair is averaged in fp32.
+ * Per group of 16 channels: scale = E4M3 nearest to amax/6 (ties to even,
+ * saturating at 448); code = sign | E2M1 nearest to |x|/scale (ties to even,
+ * saturating at 6); a zero scale stores code 0.  The entry is written at
+ * position entry_pos[i] of sequence entry_seq[i] (both int32 [n]); the
+ * indexer key is stored as bf16; the block key of every touched 8-token block
+ * is recomputed as bf16(fp32 mean of the block's present keys, ascending
+ * order).  seq_lens must already count the new entries (entry_pos[i] <
+ * seq_lens[seq]).  kv and idxk must be 16-B aligned.
+ */
+int csa2_kv_quant_append(const csa2_cache* cache, const uint16_t* kv, const uint16_t* idxk,
+                         const int32_t* entry_seq, const int32_t* entry_pos, int32_t n,
+                         int32_t compress, csa2_stream_t stream);
+
+/*
+ * csa2_indexer_score_topk -- Full or Reindex indexer step.
+ *
+ * Defines the CSA2 indexer (agentnet.co.il, section "CSA2: דחיסה לאורך ציר
+ * השכבות": Full selects 512 fresh indices; Reindex ranks the last Full
+ * layer's indexer K with its own indexer Q; the decoder's hierarchical
+ * indexer builds a pool of up to 2,048 blocks x 8 = 16,384 positions).
+ * Query r (0 <= r < nq) has indexer query idx_q[r] (bf16 [4][64]), head
+ * weights head_w[r] (float [4], or head_w == NULL for all ones), sequence
+ * q_seq[r] and visible length q_visible[r] (or seq_lens[q_seq[r]] if
+ * q_visible == NULL); max_visible >= every visible length (host-known bound
+ * that sizes the grid and the workspace).
+ * score(q, k) = sum_h w_h * max(0, q_h . k) in fp32.
+ *  - CSA2_FULL, hierarchical != 0 (decoder): if ceil(v/8) > 2048 the 2,048
+ *    best block keys form the pool, else every block does; writes
+ *    set->pool_blocks[r] and the 512 best pool tokens to set->idx[r].
+ *  - CSA2_FULL, hierarchical == 0 (encoder): 512 best of positions [0, v).
+ *  - CSA2_REINDEX: 512 best tokens of the pool written by the last
+ *    hierarchical Full call on `set` (requires set->pool_layer < layer).
+ * Ranking: score descending, then position ascending; output ascending, -1
+ * padded.  Workspace: csa2_workspace_bytes(CSA2_OP_INDEXER, nq, 0,
+ * max_visible, hierarchical).  Sets set->layer = layer, set->mode = mode.
+ */
+int csa2_indexer_score_topk(const csa2_cache* cache, const uint16_t* idx_q, const float* head_w,
+                            const int32_t* q_seq, const int32_t* q_visible, int32_t nq,
+                            int64_t max_visible, int32_t mode, int32_t hierarchical,
+                            int32_t layer, csa2_indexset* set, void* workspace,
+                            size_t workspace_bytes, csa2_stream_t stream);
+
+/*
+ * csa2_sparse_attn -- CSA2 attention of one layer.
+ *
+ * Attended set of query r: the positions in set->idx[r] joined with the
+ * window [max(0, v-128), v), each position once (128-token sliding window:
+ * ai-wave.ru, second paragraph; agentnet.co.il, section "ארכיטקטורה שחותכת
+ * בחצי את הפריפיל").  K = V = the decoded FP4 rows (exact in bf16);
+ * s = sm_scale * q . k; p = softmax over the set; out[r] = sum p k, rounded
+ * to bf16.  q: bf16 [nq][heads][512]; out: bf16 [nq][heads][512]; heads in
+ * {16, 32, 48, 64}.  Mode checks (host): CSA2_FULL / CSA2_REINDEX need
+ * set->layer == layer and set->mode == mode (the set is this layer's own);
+ * CSA2_REUSE needs set->layer < layer (the latest Full or Reindex set).  An
+ * empty set gives a zero output.  Workspace: csa2_workspace_bytes(
+ * CSA2_OP_ATTENTION, nq, heads, 0, 0).
+ */
+int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int32_t heads, float sm_scale,
+                     const int32_t* q_seq, const int32_t* q_visible, int32_t nq, int32_t mode,
+                     int32_t layer, const csa2_indexset* set, uint16_t* out, void* workspace,
+                     size_t workspace_bytes, csa2_stream_t stream);
+
+/*
+ * csa2_swa_replay -- bounded replay of the sliding window.
+ *
+ * On a cache miss only the last 128 tokens are recomputed (ai-wave.ru, second
+ * paragraph; news.hamidun.com, section "Три механизма экономии памяти";
+ * agentnet.co.il, section "ארכיטקטורה שחותכת בחצי את הפריפיל").  For every
+ * sequence b with L = seq_lens[b]: if miss[b] != 0, positions
+ * [L - min(128, L), L) are re-encoded from the last min(128, L) rows of
+ * kv_last[b] (bf16 [batch][128][512]) and idxk_last[b] (bf16
+ * [batch][128][64]); otherwise only position L-1 is written, from row 127.
+ * Same codec and block-key rule as csa2_kv_quant_append (ratio 1).
+ */
+int csa2_swa_replay(const csa2_cache* cache, const uint16_t* kv_last, const uint16_t* idxk_last,
+                    const uint8_t* miss, csa2_stream_t stream);
+
+/* Workspace bytes for an indexer call (op = CSA2_OP_INDEXER: nq, max_visible,
+ * hierarchical) or an attention call (op = CSA2_OP_ATTENTION: nq, heads).
+ * Returns 0 for an invalid request. */
+size_t csa2_workspace_bytes(int32_t op, int32_t nq, int32_t heads, int64_t max_visible,
+                            int32_t hierarchical);
+
+/* Synchronise `stream`, read and clear cache->error_word; *bits (may be NULL)
+ * receives the CSA2_DEVERR_* bits.  Returns CSA2_ERR_DEVICE_BOUNDS if any bit
+ * was set, CSA2_ERR_CUDA if the stream reported an error, else CSA2_OK. */
+int csa2_check_device_error(const csa2_cache* cache, csa2_stream_t stream, uint32_t* bits);
+
+/* Static description of a status code. */
+const char* csa2_status_string(int status);
+
+/* Library version (major*10000 + minor*100 + patch). */
+int csa2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA2_H */

@@ -18,3 +18,11 @@ def host_gen():
     import workload
     workload.build_host()
     return workload
+
+
+@pytest.fixture(scope="session")
+def csa2_lib():
+    """The built CSA2 library (nvcc for sm_100a; a few seconds) and its binding."""
+    from fp4_kv_cache_decode_b200 import _build, csa2
+    _build.build()
+    return csa2
