@@ -72,6 +72,8 @@ SIGNATURES = {
                                                _VP, _VP, _SZ, _VP]),
     "csa2_sparse_attn": (ctypes.c_int, [_VP, _VP, _I32, _F32, _VP, _VP, _I32, _I32, _I32, _VP, _VP,
                                         _VP, _SZ, _VP]),
+    "csa2_indexer_score_topk_noalloc": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _I32, _I64, _I32, _I32,
+                                                       _I32, _VP, _VP]),
     "csa2_swa_replay": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP]),
     "csa2_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I64, _I32]),
     "csa2_check_device_error": (ctypes.c_int, [_VP, _VP, ctypes.POINTER(ctypes.c_uint32)]),
@@ -218,6 +220,26 @@ def csa2_indexer_score_topk(cache: Cache, idx_q: torch.Tensor, q_seq: torch.Tens
         layer, indexset.ref(), _ptr(workspace, (torch.uint8,), "workspace"),
         workspace.numel(), _stream(stream))
     _check(st, "csa2_indexer_score_topk")
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def csa2_indexer_score_topk_noalloc(cache: Cache, idx_q: torch.Tensor, q_seq: torch.Tensor, mode: int,
+                                    layer: int, indexset: IndexSet, max_visible: int,
+                                    q_visible: torch.Tensor | None = None,
+                                    head_w: torch.Tensor | None = None, hierarchical: bool = True,
+                                    stream=None):
+    """csa2_indexer_score_topk for callers that cannot allocate: the score buffer is
+    the library's own static device array (NOALLOC_SCRATCH_BYTES); calls that
+    overlap on the GPU share it and race."""
+    nq = q_seq.numel()
+    st = lib().csa2_indexer_score_topk_noalloc(
+        cache.ref(), _ptr(idx_q, _BF16, "idx_q", nq * 256),
+        _ptr(head_w, (torch.float32,), "head_w", nq * 4), _ptr(q_seq, _I32T, "q_seq"),
+        _ptr(q_visible, _I32T, "q_visible", nq), nq, int(max_visible), mode, int(bool(hierarchical)),
+        layer, indexset.ref(), _stream(stream))
+    _check(st, "csa2_indexer_score_topk_noalloc")
 
 
 def csa2_sparse_attn(cache: Cache, q: torch.Tensor, q_seq: torch.Tensor, mode: int, layer: int,

@@ -17,9 +17,10 @@
  *   allocates no memory.  Scratch space comes from a caller workspace sized by
  *   csa2_workspace_bytes().
  * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
- *   default stream), performs no host synchronisation and no allocation, and
- *   can be captured in a CUDA graph.  csa2_check_device_error() is the only
- *   call that synchronises.
+ *   default stream) and performs no host synchronisation and no allocation;
+ *   csa2_check_device_error() is the only call that synchronises.  The calls
+ *   that take their scratch from a caller workspace, and those that need no
+ *   scratch, can be captured in a CUDA graph.
  * - bf16 tensors are passed as uint16_t bit patterns.
  * - Return value: CSA2_OK or a csa2_status error.  Argument, shape, alignment,
  *   workspace and mode-order errors are detected on the host before anything is
@@ -201,6 +202,31 @@ int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int32_t heads, 
  */
 int csa2_swa_replay(const csa2_cache* cache, const uint16_t* kv_last, const uint16_t* idxk_last,
                     const uint8_t* miss, csa2_stream_t stream);
+
+/*
+ * csa2_indexer_score_topk_noalloc -- csa2_indexer_score_topk without a
+ * caller workspace, for callers that cannot allocate device memory (a host
+ * framework that owns all device memory and gives plugins no allocator, a
+ * serving loop that must never reach cudaMalloc, a fixed memory budget).
+ *
+ * The pages describe no such interface; it has no counterpart in the method.
+ * Same arguments and results as csa2_indexer_score_topk minus the workspace:
+ * the score buffer is a library-owned static device array of
+ * CSA2_NOALLOC_SCRATCH_BYTES, present on every GPU that loads the library
+ * until the process exits.  Requests whose workspace (csa2_workspace_bytes)
+ * exceeds that size return CSA2_ERR_WORKSPACE without launching anything.
+ * All calls share the one array: calls that overlap on the GPU race, so keep
+ * them on one stream.  The array keeps the last call's contents; nothing in
+ * it needs to start at zero.  The first call on a device looks up the
+ * array's device address (a one-time set-up); make it before any stream
+ * capture.  Allocates nothing.
+ */
+#define CSA2_NOALLOC_SCRATCH_BYTES (16u << 20)   /* 16 MiB */
+int csa2_indexer_score_topk_noalloc(const csa2_cache* cache, const uint16_t* idx_q,
+                                    const float* head_w, const int32_t* q_seq,
+                                    const int32_t* q_visible, int32_t nq, int64_t max_visible,
+                                    int32_t mode, int32_t hierarchical, int32_t layer,
+                                    csa2_indexset* set, csa2_stream_t stream);
 
 /* Workspace bytes for an indexer call (op = CSA2_OP_INDEXER: nq, max_visible,
  * hierarchical) or an attention call (op = CSA2_OP_ATTENTION: nq, heads).
