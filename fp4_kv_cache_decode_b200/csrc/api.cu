@@ -28,6 +28,7 @@ using namespace csa2;
 namespace {
 
 constexpr int kSrcFlat = 0, kSrcBlockKeys = 1, kSrcPool = 2;
+constexpr int32_t kMaxQueries = 65535;   // queries map to gridDim.y
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -126,7 +127,7 @@ int csa2_indexer_score_topk(const csa2_cache* cache, const uint16_t* idx_q, cons
   if (nq < 0 || max_visible < 0 || max_visible > ((int64_t)1 << 31) - 1 || layer < 0)
     return CSA2_ERR_INVALID_ARG;
   if (!set || !set->idx) return CSA2_ERR_INVALID_ARG;
-  if (nq > set->rows) return CSA2_ERR_SHAPE;
+  if (nq > set->rows || nq > kMaxQueries) return CSA2_ERR_SHAPE;
   const bool hier = hierarchical != 0 || mode == CSA2_REINDEX;
   if (hier && !set->pool_blocks) return CSA2_ERR_INVALID_ARG;
   if (mode == CSA2_REINDEX) {
@@ -193,7 +194,7 @@ int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int32_t heads, 
   if (mode != CSA2_FULL && mode != CSA2_REINDEX && mode != CSA2_REUSE) return CSA2_ERR_INVALID_ARG;
   if (heads != 16 && heads != 32 && heads != 48 && heads != 64) return CSA2_ERR_SHAPE;
   if (nq < 0 || layer < 0 || !set || !set->idx) return CSA2_ERR_INVALID_ARG;
-  if (nq > set->rows) return CSA2_ERR_SHAPE;
+  if (nq > set->rows || nq > kMaxQueries) return CSA2_ERR_SHAPE;
   if (set->cache_id != cache->cache_id || set->layer < 0 || nq > set->nq) return CSA2_ERR_MODE_STATE;
   if (mode == CSA2_REUSE) {
     // Reuse consumes the latest Full / Reindex indices of an earlier layer

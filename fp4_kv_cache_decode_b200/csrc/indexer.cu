@@ -29,9 +29,11 @@ namespace csa2 {
 
 enum UnitSource : int { SRC_FLAT = 0, SRC_BLOCKKEYS = 1, SRC_POOL = 2 };
 
-constexpr int kScoreWarps = 8;
-constexpr int kUnitsPerWarp = 4;
-constexpr int kUnitsPerCta = kScoreWarps * kUnitsPerWarp;  // 32
+constexpr int kScoreThreads = 256;
+constexpr int kScoreWarps = kScoreThreads / 32;
+constexpr int kUnitsPerCta = 64;                         // 64 KiB of keys per CTA
+constexpr int kUnitsPerWarp = kUnitsPerCta / kScoreWarps; // 8
+constexpr uint32_t kScoreSmem = kUnitsPerCta * 1024u;
 
 __device__ __forceinline__ int64_t visible_of(const CacheView& c, const int32_t* q_seq,
                                               const int32_t* q_vis, int r) {
@@ -46,29 +48,80 @@ __device__ __forceinline__ int64_t units_of(int src, int64_t v) {
   return kPoolBlocks;
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// One CTA scores 64 consecutive units of one query:
+//  1. threads 0..63 resolve their unit's HBM address (pool entry, page table)
+//     and how many of its 8 rows are candidates;
+//  2. every warp copies its 8 units (8 KiB) into shared memory with cp.async,
+//     all in flight at once (lane l copies bytes 32l..32l+31 of each unit);
+//  3. each lane reads back exactly the bytes it copied (row l/4, dims
+//     16(l%4)..+15), forms its 4 partial head dot products, and two shuffles
+//     finish each row's dot products.
 template <int SRC>
-__global__ void __launch_bounds__(256) score_units_kernel(CacheView c, const uint16_t* __restrict__ idx_q,
-                                                          const float* __restrict__ head_w,
-                                                          const int32_t* __restrict__ q_seq,
-                                                          const int32_t* __restrict__ q_vis,
-                                                          const int32_t* __restrict__ pool,
-                                                          int64_t max_units, int64_t stride,
-                                                          float* __restrict__ scores) {
+__global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView c, const uint16_t* __restrict__ idx_q,
+                                                                       const float* __restrict__ head_w,
+                                                                       const int32_t* __restrict__ q_seq,
+                                                                       const int32_t* __restrict__ q_vis,
+                                                                       const int32_t* __restrict__ pool,
+                                                                       int64_t max_units, int64_t stride,
+                                                                       float* __restrict__ scores) {
+  extern __shared__ __align__(16) uint8_t stage[];
+  __shared__ const uint8_t* ubase[kUnitsPerCta];
+  __shared__ int32_t urows[kUnitsPerCta];
   const int r = blockIdx.y;
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int seq = q_seq[r];
   const int64_t v = visible_of(c, q_seq, q_vis, r);
   int64_t nunits = units_of(SRC, v);
   if (nunits > max_units) {   // visible length beyond the bound the call was sized for
-    if (blockIdx.x == 0 && threadIdx.x == 0) raise_error(c.err, CSA2_DEVERR_POS);
+    if (blockIdx.x == 0 && tid == 0) raise_error(c.err, CSA2_DEVERR_POS);
     nunits = max_units;
   }
-  const int64_t u0 = (int64_t)blockIdx.x * kUnitsPerCta + warp * kUnitsPerWarp;
+  const int64_t u0 = (int64_t)blockIdx.x * kUnitsPerCta;
   if (u0 >= nunits) return;
   const int64_t nb = (v + kBlock - 1) / kBlock;
 
-  // this lane's 16 dims of each head's query
+  // 1. unit addresses and candidate rows
+  if (tid < kUnitsPerCta) {
+    const int64_t u = u0 + tid;
+    const uint8_t* base = nullptr;
+    int nrows = 0;
+    if (u < nunits) {
+      if (SRC == SRC_FLAT) {
+        const int64_t pg = page_of(c, seq, u * kBlock);
+        if (pg >= 0) {
+          base = c.idxk + pg * kIdxPageBytes + (u & (kBlocksPerPage - 1)) * (kBlock * kIdxRowBytes);
+          nrows = (int)(v - u * kBlock < kBlock ? v - u * kBlock : kBlock);
+        }
+      } else if (SRC == SRC_BLOCKKEYS) {
+        const int64_t pg = page_of(c, seq, u * kPageTokens);
+        if (pg >= 0) {
+          base = c.bk + pg * kBkPageBytes;
+          nrows = (int)(nb - u * kBlocksPerPage < kBlocksPerPage ? nb - u * kBlocksPerPage : kBlocksPerPage);
+        }
+      } else {
+        const int32_t blk = pool[(int64_t)r * kPoolBlocks + u];
+        if (blk >= 0) {
+          if ((int64_t)blk >= nb) {
+            raise_error(c.err, CSA2_DEVERR_POS);
+          } else {
+            const int64_t pg = page_of(c, seq, (int64_t)blk * kBlock);
+            if (pg >= 0) {
+              base = c.idxk + pg * kIdxPageBytes + (blk & (kBlocksPerPage - 1)) * (kBlock * kIdxRowBytes);
+              nrows = (int)(v - (int64_t)blk * kBlock < kBlock ? v - (int64_t)blk * kBlock : kBlock);
+            }
+          }
+        }
+      }
+    }
+    ubase[tid] = base;
+    urows[tid] = nrows;
+  }
+
+  // this lane's 16 dims of each head's query (loaded while the lookups run)
   const int row = lane >> 2;
   const int dq = (lane & 3) * 16;
   float q[kIdxHeads][16];
@@ -84,73 +137,50 @@ __global__ void __launch_bounds__(256) score_units_kernel(CacheView c, const uin
   float w[kIdxHeads];
 #pragma unroll
   for (int h = 0; h < kIdxHeads; ++h) w[h] = head_w ? __ldg(head_w + (int64_t)r * kIdxHeads + h) : 1.0f;
+  __syncthreads();
 
-  // issue every unit's loads first, then compute
-  uint4 ka[kUnitsPerWarp], kb[kUnitsPerWarp];
-  bool ok[kUnitsPerWarp];
+  // 2. all of this warp's units in flight at once
+  const uint32_t stage_s = (uint32_t)__cvta_generic_to_shared(stage);
 #pragma unroll
   for (int i = 0; i < kUnitsPerWarp; ++i) {
-    const int64_t u = u0 + i;
-    const uint8_t* base = nullptr;
-    ok[i] = false;
-    if (u < nunits) {
-      if (SRC == SRC_FLAT) {
-        const int64_t pg = page_of(c, seq, u * kBlock);
-        if (pg >= 0) {
-          base = c.idxk + pg * kIdxPageBytes + (u & (kBlocksPerPage - 1)) * (kBlock * kIdxRowBytes);
-          ok[i] = (u * kBlock + row) < v;
-        }
-      } else if (SRC == SRC_BLOCKKEYS) {
-        const int64_t pg = page_of(c, seq, u * kPageTokens);
-        if (pg >= 0) {
-          base = c.bk + pg * kBkPageBytes;
-          ok[i] = (u * kBlocksPerPage + row) < nb;
-        }
-      } else {
-        const int32_t blk = pool[(int64_t)r * kPoolBlocks + u];
-        if (blk >= 0) {
-          if ((int64_t)blk >= nb) {
-            raise_error(c.err, CSA2_DEVERR_POS);
-          } else {
-            const int64_t pg = page_of(c, seq, (int64_t)blk * kBlock);
-            if (pg >= 0) {
-              base = c.idxk + pg * kIdxPageBytes + (blk & (kBlocksPerPage - 1)) * (kBlock * kIdxRowBytes);
-              ok[i] = ((int64_t)blk * kBlock + row) < v;
-            }
-          }
-        }
-      }
-    }
+    const int j = warp * kUnitsPerWarp + i;
+    const uint8_t* base = ubase[j];
+    const uint32_t dst = stage_s + j * 1024u + lane * 32u;
     if (base != nullptr) {
-      const uint8_t* p = base + row * kIdxRowBytes + dq * 2;
-      ka[i] = ld_stream16(p);
-      kb[i] = ld_stream16(p + 16);
-    } else {
-      ka[i] = make_uint4(0, 0, 0, 0);
-      kb[i] = ka[i];
+      cp_async16(dst, base + lane * 32);
+      cp_async16(dst + 16, base + lane * 32 + 16);
     }
   }
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+
+  // 3. scores (each lane reads back its own bytes)
 #pragma unroll
   for (int i = 0; i < kUnitsPerWarp; ++i) {
-    const int64_t u = u0 + i;
+    const int j = warp * kUnitsPerWarp + i;
+    const int64_t u = u0 + j;
+    const bool have = ubase[j] != nullptr;
+    uint4 ka = make_uint4(0, 0, 0, 0), kb = ka;
+    if (have) {
+      ka = *reinterpret_cast<const uint4*>(stage + j * 1024 + lane * 32);
+      kb = *reinterpret_cast<const uint4*>(stage + j * 1024 + lane * 32 + 16);
+    }
     float k[16];
-    k[0] = bf16_lo(ka[i].x); k[1] = bf16_hi(ka[i].x); k[2] = bf16_lo(ka[i].y); k[3] = bf16_hi(ka[i].y);
-    k[4] = bf16_lo(ka[i].z); k[5] = bf16_hi(ka[i].z); k[6] = bf16_lo(ka[i].w); k[7] = bf16_hi(ka[i].w);
-    k[8] = bf16_lo(kb[i].x); k[9] = bf16_hi(kb[i].x); k[10] = bf16_lo(kb[i].y); k[11] = bf16_hi(kb[i].y);
-    k[12] = bf16_lo(kb[i].z); k[13] = bf16_hi(kb[i].z); k[14] = bf16_lo(kb[i].w); k[15] = bf16_hi(kb[i].w);
-    float s = 0.0f;
+    k[0] = bf16_lo(ka.x); k[1] = bf16_hi(ka.x); k[2] = bf16_lo(ka.y); k[3] = bf16_hi(ka.y);
+    k[4] = bf16_lo(ka.z); k[5] = bf16_hi(ka.z); k[6] = bf16_lo(ka.w); k[7] = bf16_hi(ka.w);
+    k[8] = bf16_lo(kb.x); k[9] = bf16_hi(kb.x); k[10] = bf16_lo(kb.y); k[11] = bf16_hi(kb.y);
+    k[12] = bf16_lo(kb.z); k[13] = bf16_hi(kb.z); k[14] = bf16_lo(kb.w); k[15] = bf16_hi(kb.w);
+    float sc = 0.0f;
 #pragma unroll
     for (int h = 0; h < kIdxHeads; ++h) {
       float p = 0.0f;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) p = fmaf(q[h][j], k[j], p);
+      for (int jj = 0; jj < 16; ++jj) p = fmaf(q[h][jj], k[jj], p);
       p += __shfl_xor_sync(0xffffffffu, p, 1);
       p += __shfl_xor_sync(0xffffffffu, p, 2);
-      s = fmaf(w[h], fmaxf(p, 0.0f), s);
+      sc = fmaf(w[h], fmaxf(p, 0.0f), sc);
     }
-    if (u < nunits && (lane & 3) == 0) {
-      scores[(int64_t)r * stride + u * kBlock + row] = ok[i] ? s : -INFINITY;
-    }
+    if (u < nunits && (lane & 3) == 0)
+      scores[(int64_t)r * stride + u * kBlock + row] = row < urows[j] ? sc : -INFINITY;
   }
 }
 
@@ -160,6 +190,7 @@ __global__ void __launch_bounds__(256) score_units_kernel(CacheView c, const uin
 
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkSmemKeys = 16384;   // keys cached in shared memory up to this count
+constexpr int kCandCap = 4096;         // boundary-bucket candidates kept for refinement
 
 // Exclusive scan of one value per thread across the CTA (1024 threads).
 // Returns the exclusive prefix; *total receives the CTA-wide sum.
@@ -191,22 +222,32 @@ __device__ __forceinline__ uint32_t cta_exclusive_scan(uint32_t v, uint32_t* war
   return res;
 }
 
-struct TopkSmem {
+struct __align__(16) TopkSmem {
   uint32_t hist[4096];
+  uint32_t cand[kCandCap];
   uint32_t warp_sums[33];
-  uint32_t bucket, above;   // result of a bucket search
-  uint32_t nvalid;
+  uint32_t bucket, above, nvalid, ncand;
 };
 
+// Histogram increment aggregated over the lanes of a warp that hit the same
+// bin (scores cluster in few top-digit bins; one atomic per distinct bin).
+// Every lane of the warp must call this.
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool pred) {
+  const uint32_t active = __ballot_sync(0xffffffffu, pred);
+  if (pred) {
+    const uint32_t peers = __match_any_sync(active, bin);
+    if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+  }
+}
+
 // Find the bucket holding the k_rem-th largest element of a histogram of
-// `nbins` bins (bins ordered by key; larger bin = larger key).  Sets
-// sm->bucket and sm->above (elements in higher bins).
+// `nbins` bins (larger bin = larger key).  Sets sm->bucket and sm->above
+// (elements in higher bins).
 __device__ __forceinline__ void find_bucket(TopkSmem* sm, int nbins, uint32_t k_rem) {
-  // thread t owns bins [nbins - 4(t+1), nbins - 4t) counted from the top
   const int per = 4;
   const int t = threadIdx.x;
   uint32_t local = 0;
-  const int hi = nbins - per * t;   // exclusive upper bin
+  const int hi = nbins - per * t;   // this thread's bins: [hi-4, hi), counted from the top
   if (hi > 0) {
 #pragma unroll
     for (int j = 1; j <= per; ++j)
@@ -237,7 +278,129 @@ __device__ __forceinline__ int32_t map_out(int64_t i, const int32_t* pool_row) {
   return (int32_t)i;
 }
 
+constexpr int kKeysPerThread = kTopkSmemKeys / kTopkThreads;   // 16
+
+// Top-k of up to 16,384 entries with every key held in registers: thread t
+// owns positions [16t, 16t+16).
+//  1. histogram of the keys' top 11 bits (2,048 bins, shared-memory atomics);
+//     the bucket holding the k-th key is found by a CTA scan over the bins;
+//  2. that bucket's keys are compacted into a candidate list (offsets from a
+//     CTA scan of per-thread match counts) and refined on bits 20..10 and
+//     9..0, giving the exact k-th largest key T and the number of keys equal
+//     to T to keep (the lowest-position ones);
+//  3. one CTA scan of per-thread (count > T, count == T) gives every thread
+//     its output offset; selected positions are written in position order.
+// If the boundary bucket holds more keys than the candidate list, the
+// refinement runs over all keys (same histograms, prefix-filtered).
+template <int SRC>
+__device__ __forceinline__ void topk_registers(const float* __restrict__ srow, int64_t n, int k,
+                                               const int32_t* pool_row, int32_t* __restrict__ orow,
+                                               TopkSmem* sm) {
+  const int tid = threadIdx.x;
+  const int64_t lo = (int64_t)tid * kKeysPerThread;
+  uint32_t key[kKeysPerThread];
+#pragma unroll
+  for (int j = 0; j < kKeysPerThread; j += 4) {
+    if (lo + j < n) {   // n is a multiple of 8, so a float4 never straddles the end
+      const float4 f = *reinterpret_cast<const float4*>(srow + lo + j);
+      key[j] = score_key(f.x); key[j + 1] = score_key(f.y);
+      key[j + 2] = score_key(f.z); key[j + 3] = score_key(f.w);
+    } else {
+      key[j] = key[j + 1] = key[j + 2] = key[j + 3] = 0u;
+    }
+  }
+  for (int i = tid; i < 2048; i += kTopkThreads) sm->hist[i] = 0;
+  __syncthreads();
+  uint32_t nv = 0;
+#pragma unroll
+  for (int j = 0; j < kKeysPerThread; ++j) {
+    if (key[j]) {
+      ++nv;
+      atomicAdd(&sm->hist[key[j] >> 21], 1u);
+    }
+  }
+  uint32_t nvalid;
+  cta_exclusive_scan(nv, sm->warp_sums, &nvalid);
+
+  uint32_t T = 1u, need_eq = 0xFFFFFFFFu;
+  if (nvalid > (uint32_t)k) {
+    uint32_t k_rem = (uint32_t)k;
+    find_bucket(sm, 2048, k_rem);
+    const uint32_t b1 = sm->bucket;
+    k_rem -= sm->above;
+    // compact the boundary bucket
+    uint32_t nm = 0;
+#pragma unroll
+    for (int j = 0; j < kKeysPerThread; ++j) nm += (key[j] && (key[j] >> 21) == b1) ? 1u : 0u;
+    uint32_t ncand;
+    uint32_t off = cta_exclusive_scan(nm, sm->warp_sums, &ncand);
+    const bool use_cand = ncand <= (uint32_t)kCandCap;
+    if (use_cand && nm) {
+#pragma unroll
+      for (int j = 0; j < kKeysPerThread; ++j)
+        if (key[j] && (key[j] >> 21) == b1) sm->cand[off++] = key[j];
+    }
+    uint32_t prefix = b1 << 21;
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+      const int shift = pass == 0 ? 10 : 0;
+      const uint32_t pmask = pass == 0 ? 0xFFE00000u : 0xFFFFFC00u;
+      const uint32_t dmask = pass == 0 ? 0x7FFu : 0x3FFu;
+      for (int i = tid; i < 2048; i += kTopkThreads) sm->hist[i] = 0;
+      __syncthreads();
+      if (use_cand) {
+        for (uint32_t i = tid; i < ncand; i += kTopkThreads) {
+          const uint32_t kk = sm->cand[i];
+          if ((kk & pmask) == prefix) atomicAdd(&sm->hist[(kk >> shift) & dmask], 1u);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < kKeysPerThread; ++j)
+          if (key[j] && (key[j] & pmask) == prefix) atomicAdd(&sm->hist[(key[j] >> shift) & dmask], 1u);
+      }
+      __syncthreads();
+      find_bucket(sm, pass == 0 ? 2048 : 1024, k_rem);
+      prefix |= sm->bucket << shift;
+      k_rem -= sm->above;
+    }
+    T = prefix;
+    need_eq = k_rem;
+  }
+  // output: one scan of packed (count > T, count == T); both fit 16 bits
+  uint32_t ngt = 0, neq = 0;
+#pragma unroll
+  for (int j = 0; j < kKeysPerThread; ++j) {
+    ngt += (key[j] != 0u && key[j] > T) ? 1u : 0u;
+    neq += (key[j] != 0u && key[j] == T) ? 1u : 0u;
+  }
+  uint32_t tot;
+  const uint32_t before = cta_exclusive_scan((ngt << 16) | neq, sm->warp_sums, &tot);
+  const uint32_t gt_before = before >> 16, eq_before = before & 0xFFFFu;
+  const uint32_t tot_gt = tot >> 16, tot_eq = tot & 0xFFFFu;
+  uint32_t slot = gt_before + min(eq_before, need_eq);
+  uint32_t eq_rank = eq_before;
+#pragma unroll
+  for (int j = 0; j < kKeysPerThread; ++j) {
+    const uint32_t kj = key[j];
+    bool sel = kj != 0u && kj > T;
+    if (kj != 0u && kj == T) sel = eq_rank++ < need_eq;
+    if (sel && slot < (uint32_t)k) orow[slot++] = map_out<SRC>(lo + j, pool_row);
+  }
+  const uint32_t total = tot_gt + min(tot_eq, need_eq);
+  for (int64_t s = (int64_t)total + tid; s < k; s += kTopkThreads) orow[s] = -1;
+}
+
 // One CTA per query: select the k best entries of scores[r][0 .. n_r).
+// Up to 16,384 entries: keys in registers (topk_registers).  Larger rows
+// (the block level of a 1M context, a long encoder prefix):
+//  1. histogram of the keys' top 12 bits (order-preserving uint32 of the
+//     scores, 0 = no candidate), read from the workspace;
+//  2. the bucket holding the k-th key is found; its keys are compacted into a
+//     candidate list and refined on bits 19..8 and 7..0, giving the exact
+//     k-th key T and how many keys equal to T are kept;
+//  3. each thread takes a contiguous segment of positions, counts its keys
+//     above T and equal to T, one CTA scan gives its output offset, and it
+//     writes its selected positions in order (ascending overall).
 template <int SRC>
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(CacheView c, const float* __restrict__ scores,
                                                             int64_t stride, const int32_t* __restrict__ q_seq,
@@ -246,86 +409,125 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(CacheView c, const f
                                                             int32_t* __restrict__ out, int64_t out_stride) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   TopkSmem* sm = reinterpret_cast<TopkSmem*>(smem_raw);
-  uint32_t* keys_sm = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkSmem));
 
   const int r = blockIdx.x;
   const int tid = threadIdx.x;
   const int64_t v = visible_of(c, q_seq, q_vis, r);
-  const int64_t n = min(units_of(SRC, v) * kBlock, stride);
+  const int64_t n = min(units_of(SRC, v) * kBlock, stride);   // a multiple of 8
   const float* srow = scores + (int64_t)r * stride;
   const int32_t* pool_row = pool ? pool + (int64_t)r * kPoolBlocks : nullptr;
   int32_t* orow = out + (int64_t)r * out_stride;
-  const bool cached = n <= kTopkSmemKeys;
+  if (n <= kTopkSmemKeys) {
+    topk_registers<SRC>(srow, n, k, pool_row, orow, sm);
+    return;
+  }
+  auto key_at = [&](int64_t i) -> uint32_t { return score_key(srow[i]); };
 
-  // pass 0: keys (cached), valid count, 12-bit histogram of the top digit
+  // pass 0: valid count, histogram of bits 31..20
   for (int i = tid; i < 4096; i += kTopkThreads) sm->hist[i] = 0;
-  if (tid == 0) sm->nvalid = 0;
+  if (tid == 0) {
+    sm->nvalid = 0;
+    sm->ncand = 0;
+  }
   __syncthreads();
   uint32_t myvalid = 0;
-  for (int64_t i = tid; i < n; i += kTopkThreads) {
-    const uint32_t key = score_key(srow[i]);
-    if (cached) keys_sm[i] = key;
-    if (key) {
-      ++myvalid;
-      atomicAdd(&sm->hist[key >> 20], 1u);
+  for (int64_t b0 = 0; b0 < n; b0 += 4 * kTopkThreads) {
+    const int64_t i4 = b0 + 4 * (int64_t)tid;
+    uint32_t kk[4] = {0u, 0u, 0u, 0u};
+    if (i4 < n) {
+      const float4 f = *reinterpret_cast<const float4*>(srow + i4);
+      kk[0] = score_key(f.x); kk[1] = score_key(f.y); kk[2] = score_key(f.z); kk[3] = score_key(f.w);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      myvalid += kk[j] ? 1u : 0u;
+      hist_add(sm->hist, kk[j] >> 20, kk[j] != 0u);
     }
   }
   atomicAdd(&sm->nvalid, myvalid);
   __syncthreads();
   const uint32_t nvalid = sm->nvalid;
-  auto key_at = [&](int64_t i) -> uint32_t { return cached ? keys_sm[i] : score_key(srow[i]); };
 
-  uint32_t T = 1u;           // select keys >= T ... refined below
-  uint32_t need_eq = 0xFFFFFFFFu;
+  uint32_t T = 1u;                  // keep every key > T ...
+  uint32_t need_eq = 0xFFFFFFFFu;   // ... and this many keys == T (lowest positions first)
   if (nvalid > (uint32_t)k) {
     uint32_t k_rem = (uint32_t)k;
     find_bucket(sm, 4096, k_rem);
-    uint32_t prefix = sm->bucket << 20;
+    const uint32_t b1 = sm->bucket;
     k_rem -= sm->above;
-    // pass 1: bits 19..8 among keys with the same top 12 bits
-    for (int i = tid; i < 4096; i += kTopkThreads) sm->hist[i] = 0;
-    __syncthreads();
-    for (int64_t i = tid; i < n; i += kTopkThreads) {
-      const uint32_t key = key_at(i);
-      if ((key & 0xFFF00000u) == prefix) atomicAdd(&sm->hist[(key >> 8) & 0xFFFu], 1u);
+    // compact the boundary bucket's keys
+    for (int64_t b0 = 0; b0 < n; b0 += kTopkThreads) {
+      const int64_t i = b0 + tid;
+      const uint32_t key = i < n ? key_at(i) : 0u;
+      const bool m = key != 0u && (key >> 20) == b1;
+      const uint32_t bal = __ballot_sync(0xffffffffu, m);
+      uint32_t base = 0;
+      if ((tid & 31) == 0 && bal) base = atomicAdd(&sm->ncand, (uint32_t)__popc(bal));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      const uint32_t slot = base + __popc(bal & ((1u << (tid & 31)) - 1u));
+      if (m && slot < (uint32_t)kCandCap) sm->cand[slot] = key;
     }
     __syncthreads();
-    find_bucket(sm, 4096, k_rem);
-    prefix |= sm->bucket << 8;
-    k_rem -= sm->above;
-    // pass 2: bits 7..0
-    for (int i = tid; i < 256; i += kTopkThreads) sm->hist[i] = 0;
-    __syncthreads();
-    for (int64_t i = tid; i < n; i += kTopkThreads) {
-      const uint32_t key = key_at(i);
-      if ((key & 0xFFFFFF00u) == prefix) atomicAdd(&sm->hist[key & 0xFFu], 1u);
+    const uint32_t ncand = sm->ncand;
+    const bool use_cand = ncand <= (uint32_t)kCandCap;
+    // refine on bits 19..8, then 7..0 (over the candidates, or over all keys
+    // with the bucket prefix when the bucket overflowed the candidate list)
+    uint32_t prefix = b1 << 20;
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+      const int shift = pass == 0 ? 8 : 0;
+      const uint32_t pmask = pass == 0 ? 0xFFF00000u : 0xFFFFFF00u;
+      const uint32_t dmask = pass == 0 ? 0xFFFu : 0xFFu;
+      for (int i = tid; i < 4096; i += kTopkThreads) sm->hist[i] = 0;
+      __syncthreads();
+      const int64_t m_n = use_cand ? (int64_t)ncand : n;
+      for (int64_t b0 = 0; b0 < m_n; b0 += kTopkThreads) {
+        const int64_t i = b0 + tid;
+        const uint32_t key = i < m_n ? (use_cand ? sm->cand[i] : key_at(i)) : 0u;
+        hist_add(sm->hist, (key >> shift) & dmask, key != 0u && (key & pmask) == prefix);
+      }
+      __syncthreads();
+      find_bucket(sm, pass == 0 ? 4096 : 256, k_rem);
+      prefix |= sm->bucket << shift;
+      k_rem -= sm->above;
     }
-    __syncthreads();
-    find_bucket(sm, 256, k_rem);
-    T = prefix | sm->bucket;
-    k_rem -= sm->above;
-    need_eq = k_rem;          // how many entries equal to T to keep (lowest positions)
+    T = prefix;
+    need_eq = k_rem;
   }
 
-  // final pass in position order: keep key > T, and key == T while need_eq lasts
-  uint32_t base_sel = 0, base_eq = 0;
-  for (int64_t c0 = 0; c0 < n; c0 += kTopkThreads) {
-    const int64_t i = c0 + tid;
-    uint32_t key = 0;
-    if (i < n) key = key_at(i);
-    const uint32_t gt = (key != 0 && key > T) ? 1u : 0u;
-    const uint32_t eq = (key != 0 && key == T) ? 1u : 0u;
-    uint32_t tot_eq;
-    const uint32_t eq_rank = cta_exclusive_scan(eq, sm->warp_sums, &tot_eq) + base_eq;
-    const uint32_t sel = gt | ((eq && eq_rank < need_eq) ? 1u : 0u);
-    uint32_t tot_sel;
-    const uint32_t slot = cta_exclusive_scan(sel, sm->warp_sums, &tot_sel) + base_sel;
-    if (sel && slot < (uint32_t)k) orow[slot] = map_out<SRC>(i, pool_row);
-    base_sel += tot_sel;
-    base_eq += tot_eq;
-    if (base_sel >= (uint32_t)k) break;
+  // output: contiguous segments in position order (read 4 keys at a time)
+  const int64_t seg = (((n + kTopkThreads - 1) / kTopkThreads) + 3) & ~(int64_t)3;
+  const int64_t lo = min((int64_t)tid * seg, n), hi = min(lo + seg, n);
+  uint32_t ngt = 0, neq = 0;
+  for (int64_t i = lo; i < hi; i += 4) {
+    const float4 f = *reinterpret_cast<const float4*>(srow + i);
+    const uint32_t kk[4] = {score_key(f.x), score_key(f.y), score_key(f.z), score_key(f.w)};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      ngt += (kk[j] != 0u && kk[j] > T) ? 1u : 0u;
+      neq += (kk[j] != 0u && kk[j] == T) ? 1u : 0u;
+    }
   }
-  for (int64_t s = (int64_t)base_sel + tid; s < k; s += kTopkThreads) orow[s] = -1;
+  uint32_t tot_gt, tot_eq;
+  const uint32_t gt_before = cta_exclusive_scan(ngt, sm->warp_sums, &tot_gt);
+  const uint32_t eq_before = cta_exclusive_scan(neq, sm->warp_sums, &tot_eq);
+  uint32_t slot = gt_before + min(eq_before, need_eq);
+  uint32_t eq_rank = eq_before;
+  if (ngt + neq > 0) {
+    for (int64_t i = lo; i < hi; i += 4) {
+      const float4 f = *reinterpret_cast<const float4*>(srow + i);
+      const uint32_t kk[4] = {score_key(f.x), score_key(f.y), score_key(f.z), score_key(f.w)};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (kk[j] == 0u || kk[j] < T) continue;
+        bool sel = kk[j] > T;
+        if (!sel) sel = eq_rank++ < need_eq;
+        if (sel && slot < (uint32_t)k) orow[slot++] = map_out<SRC>(i + j, pool_row);
+      }
+    }
+  }
+  const uint32_t total = tot_gt + min(tot_eq, need_eq);
+  for (int64_t s = (int64_t)total + tid; s < k; s += kTopkThreads) orow[s] = -1;
 }
 
 }  // namespace csa2
@@ -333,12 +535,18 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(CacheView c, const f
 // ---- launchers used by api.cu ----
 namespace csa2 {
 
-size_t topk_smem_bytes() { return sizeof(TopkSmem) + (size_t)kTopkSmemKeys * 4; }
+size_t topk_smem_bytes() { return sizeof(TopkSmem); }
 
 // Opt the top-k kernels in to their shared-memory size (once per device).
 cudaError_t indexer_set_attributes() {
   const int smem = (int)topk_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(topk_kernel<SRC_FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(score_units_kernel<SRC_FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(score_units_kernel<SRC_BLOCKKEYS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(score_units_kernel<SRC_POOL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmem);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(topk_kernel<SRC_BLOCKKEYS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess)
@@ -353,11 +561,11 @@ cudaError_t launch_score(int src, const CacheView& c, const uint16_t* idx_q, con
   dim3 grid((unsigned)((max_units + kUnitsPerCta - 1) / kUnitsPerCta), (unsigned)nq);
   if (grid.x == 0) return cudaSuccess;
   if (src == SRC_FLAT)
-    score_units_kernel<SRC_FLAT><<<grid, 256, 0, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, scores);
+    score_units_kernel<SRC_FLAT><<<grid, kScoreThreads, kScoreSmem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, scores);
   else if (src == SRC_BLOCKKEYS)
-    score_units_kernel<SRC_BLOCKKEYS><<<grid, 256, 0, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, scores);
+    score_units_kernel<SRC_BLOCKKEYS><<<grid, kScoreThreads, kScoreSmem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, scores);
   else
-    score_units_kernel<SRC_POOL><<<grid, 256, 0, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, scores);
+    score_units_kernel<SRC_POOL><<<grid, kScoreThreads, kScoreSmem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, scores);
   return cudaGetLastError();
 }
 

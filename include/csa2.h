@@ -85,6 +85,7 @@ typedef enum { CSA2_OP_INDEXER = 1, CSA2_OP_ATTENTION = 2 } csa2_op;
 #define CSA2_DEVERR_PAGE 1u  /* page id outside [0, n_pages) or page slot >= max_pages */
 #define CSA2_DEVERR_POS 2u   /* position/index outside the sequence's visible length   */
 #define CSA2_DEVERR_SEQ 4u   /* sequence id outside [0, batch)                         */
+#define CSA2_DEVERR_TIMEOUT 8u  /* a bounded wait for tensor-core completion ran out    */
 
 /* Paged cache; every pointer is device memory owned by the caller. */
 typedef struct {
@@ -150,7 +151,7 @@ int csa2_kv_quant_append(const csa2_cache* cache, const uint16_t* kv, const uint
  * weights head_w[r] (float [4], or head_w == NULL for all ones), sequence
  * q_seq[r] and visible length q_visible[r] (or seq_lens[q_seq[r]] if
  * q_visible == NULL); max_visible >= every visible length (host-known bound
- * that sizes the grid and the workspace).
+ * that sizes the grid and the workspace); nq <= 65535.
  * score(q, k) = sum_h w_h * max(0, q_h . k) in fp32.
  *  - CSA2_FULL, hierarchical != 0 (decoder): if ceil(v/8) > 2048 the 2,048
  *    best block keys form the pool, else every block does; writes
@@ -177,7 +178,7 @@ int csa2_indexer_score_topk(const csa2_cache* cache, const uint16_t* idx_q, cons
  * בחצי את הפריפיל").  K = V = the decoded FP4 rows (exact in bf16);
  * s = sm_scale * q . k; p = softmax over the set; out[r] = sum p k, rounded
  * to bf16.  q: bf16 [nq][heads][512]; out: bf16 [nq][heads][512]; heads in
- * {16, 32, 48, 64}.  Mode checks (host): CSA2_FULL / CSA2_REINDEX need
+ * {16, 32, 48, 64}; nq <= 65535.  Mode checks (host): CSA2_FULL / CSA2_REINDEX need
  * set->layer == layer and set->mode == mode (the set is this layer's own);
  * CSA2_REUSE needs set->layer < layer (the latest Full or Reindex set).  An
  * empty set gives a zero output.  Workspace: csa2_workspace_bytes(
