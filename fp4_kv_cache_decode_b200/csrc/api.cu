@@ -207,7 +207,7 @@ int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int32_t heads, 
   if (!aligned(q, 16) || !aligned(out, 16) || !aligned(q_seq, 4) || !aligned(q_visible, 4))
     return CSA2_ERR_ALIGNMENT;
   const size_t need = csa2_workspace_bytes(CSA2_OP_ATTENTION, nq, heads, 0, 0);
-  if (nq > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16)))
+  if (nq > 0 && need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16)))
     return CSA2_ERR_WORKSPACE;
   if (nq == 0) return CSA2_OK;
   if ((st = ensure_device_setup())) return st;

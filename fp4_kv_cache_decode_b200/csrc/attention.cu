@@ -141,12 +141,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // the unscaled values.  The 8 magnitudes' bf16 bytes are byte-permute tables:
 // low bytes {00,00,80,C0,00,40,80,C0}, high bytes {00,3F,3F,3F,40,40,40,40}
 // for 0, .5, 1, 1.5, 2, 3, 4, 6; the code's bit 3 becomes the bf16 sign.
+// The four sign bits (code bits 3, 7, 11, 15) are moved to bit 7 of the
+// matching high byte via the byte pattern [b0, b0, b1, b1] of the codes.
 __device__ __forceinline__ void e2m1x4_to_bf16(uint32_t c16, uint32_t& w0, uint32_t& w1) {
   const uint32_t sel = c16 & 0x7777u;
   const uint32_t lo = __byte_perm(0xC0800000u, 0xC0804000u, sel);
-  const uint32_t hi = __byte_perm(0x3F3F3F00u, 0x40404040u, sel);
-  w0 = __byte_perm(lo, hi, 0x5140) | ((c16 << 12) & 0x8000u) | ((c16 << 24) & 0x80000000u);
-  w1 = __byte_perm(lo, hi, 0x7362) | ((c16 << 4) & 0x8000u) | ((c16 << 16) & 0x80000000u);
+  const uint32_t dup = __byte_perm(c16, 0u, 0x1100);
+  const uint32_t hi = __byte_perm(0x3F3F3F00u, 0x40404040u, sel) | (dup & 0x80008000u) |
+                      ((dup << 4) & 0x00800080u);
+  w0 = __byte_perm(lo, hi, 0x5140);
+  w1 = __byte_perm(lo, hi, 0x7362);
 }
 
 // 8 decoded channels (one 16-B chunk): codes word (4 bytes) x scale (bf16x2).

@@ -31,9 +31,11 @@ enum UnitSource : int { SRC_FLAT = 0, SRC_BLOCKKEYS = 1, SRC_POOL = 2 };
 
 constexpr int kScoreThreads = 256;
 constexpr int kScoreWarps = kScoreThreads / 32;
-constexpr int kUnitsPerCta = 64;                         // 64 KiB of keys per CTA
-constexpr int kUnitsPerWarp = kUnitsPerCta / kScoreWarps; // 8
-constexpr uint32_t kScoreSmem = kUnitsPerCta * 1024u;
+constexpr int kUnitsPerCta = 256;                         // 256 KiB of keys per CTA
+constexpr int kStageUnits = 32;                           // 32 KiB per pipeline stage
+constexpr int kStages = 3;
+constexpr int kWarpStageUnits = kStageUnits / kScoreWarps;   // 4 units per warp per stage
+constexpr uint32_t kScoreSmem = kStages * kStageUnits * 1024u;
 
 __device__ __forceinline__ int64_t visible_of(const CacheView& c, const int32_t* q_seq,
                                               const int32_t* q_vis, int r) {
@@ -52,14 +54,15 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 
-// One CTA scores 64 consecutive units of one query:
-//  1. threads 0..63 resolve their unit's HBM address (pool entry, page table)
-//     and how many of its 8 rows are candidates;
-//  2. every warp copies its 8 units (8 KiB) into shared memory with cp.async,
-//     all in flight at once (lane l copies bytes 32l..32l+31 of each unit);
+// One CTA scores up to 256 consecutive units of one query:
+//  1. thread t resolves unit t's HBM address (pool entry, page table) and how
+//     many of its 8 rows are candidates -- all 256 lookups in flight at once;
+//  2. the units stream through a 3-stage ring of 32-KiB shared-memory stages
+//     with cp.async (lane l of a warp copies bytes 32l..32l+31 of each of the
+//     warp's 4 units per stage), two stages ahead of the compute;
 //  3. each lane reads back exactly the bytes it copied (row l/4, dims
 //     16(l%4)..+15), forms its 4 partial head dot products, and two shuffles
-//     finish each row's dot products.
+//     finish each row's dot products.  No CTA-wide barrier inside the stream.
 template <int SRC>
 __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView c, const uint16_t* __restrict__ idx_q,
                                                                        const float* __restrict__ head_w,
@@ -83,13 +86,14 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView
   const int64_t u0 = (int64_t)blockIdx.x * kUnitsPerCta;
   if (u0 >= nunits) return;
   const int64_t nb = (v + kBlock - 1) / kBlock;
+  const int nu = (int)(nunits - u0 < kUnitsPerCta ? nunits - u0 : kUnitsPerCta);
 
   // 1. unit addresses and candidate rows
-  if (tid < kUnitsPerCta) {
+  {
     const int64_t u = u0 + tid;
     const uint8_t* base = nullptr;
     int nrows = 0;
-    if (u < nunits) {
+    if (tid < nu) {
       if (SRC == SRC_FLAT) {
         const int64_t pg = page_of(c, seq, u * kBlock);
         if (pg >= 0) {
@@ -139,49 +143,61 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView
   for (int h = 0; h < kIdxHeads; ++h) w[h] = head_w ? __ldg(head_w + (int64_t)r * kIdxHeads + h) : 1.0f;
   __syncthreads();
 
-  // 2. all of this warp's units in flight at once
   const uint32_t stage_s = (uint32_t)__cvta_generic_to_shared(stage);
+  const int nstage = (nu + kStageUnits - 1) / kStageUnits;
+  // issue the copies of stage s (this warp's 4 units) into ring slot s % kStages
+  auto issue = [&](int st) {
+    if (st < nstage) {
 #pragma unroll
-  for (int i = 0; i < kUnitsPerWarp; ++i) {
-    const int j = warp * kUnitsPerWarp + i;
-    const uint8_t* base = ubase[j];
-    const uint32_t dst = stage_s + j * 1024u + lane * 32u;
-    if (base != nullptr) {
-      cp_async16(dst, base + lane * 32);
-      cp_async16(dst + 16, base + lane * 32 + 16);
+      for (int i = 0; i < kWarpStageUnits; ++i) {
+        const int j = st * kStageUnits + warp * kWarpStageUnits + i;
+        const uint8_t* base = ubase[j];
+        const uint32_t dst = stage_s + ((st % kStages) * kStageUnits + warp * kWarpStageUnits + i) * 1024u + lane * 32u;
+        if (j < nu && base != nullptr) {
+          cp_async16(dst, base + lane * 32);
+          cp_async16(dst + 16, base + lane * 32 + 16);
+        }
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  issue(0);
+  issue(1);
+#pragma unroll 1
+  for (int st = 0; st < nstage; ++st) {
+    issue(st + 2);
+    asm volatile("cp.async.wait_group 2;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < kWarpStageUnits; ++i) {
+      const int j = st * kStageUnits + warp * kWarpStageUnits + i;
+      const int64_t u = u0 + j;
+      const bool have = j < nu && ubase[j] != nullptr;
+      const uint8_t* sl = stage + ((st % kStages) * kStageUnits + warp * kWarpStageUnits + i) * 1024 + lane * 32;
+      uint4 ka = make_uint4(0, 0, 0, 0), kb = ka;
+      if (have) {
+        ka = *reinterpret_cast<const uint4*>(sl);
+        kb = *reinterpret_cast<const uint4*>(sl + 16);
+      }
+      float k[16];
+      k[0] = bf16_lo(ka.x); k[1] = bf16_hi(ka.x); k[2] = bf16_lo(ka.y); k[3] = bf16_hi(ka.y);
+      k[4] = bf16_lo(ka.z); k[5] = bf16_hi(ka.z); k[6] = bf16_lo(ka.w); k[7] = bf16_hi(ka.w);
+      k[8] = bf16_lo(kb.x); k[9] = bf16_hi(kb.x); k[10] = bf16_lo(kb.y); k[11] = bf16_hi(kb.y);
+      k[12] = bf16_lo(kb.z); k[13] = bf16_hi(kb.z); k[14] = bf16_lo(kb.w); k[15] = bf16_hi(kb.w);
+      float sc = 0.0f;
+#pragma unroll
+      for (int h = 0; h < kIdxHeads; ++h) {
+        float p = 0.0f;
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) p = fmaf(q[h][jj], k[jj], p);
+        p += __shfl_xor_sync(0xffffffffu, p, 1);
+        p += __shfl_xor_sync(0xffffffffu, p, 2);
+        sc = fmaf(w[h], fmaxf(p, 0.0f), sc);
+      }
+      if (j < nu && (lane & 3) == 0)
+        scores[(int64_t)r * stride + u * kBlock + row] = row < urows[j] ? sc : -INFINITY;
     }
   }
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-
-  // 3. scores (each lane reads back its own bytes)
-#pragma unroll
-  for (int i = 0; i < kUnitsPerWarp; ++i) {
-    const int j = warp * kUnitsPerWarp + i;
-    const int64_t u = u0 + j;
-    const bool have = ubase[j] != nullptr;
-    uint4 ka = make_uint4(0, 0, 0, 0), kb = ka;
-    if (have) {
-      ka = *reinterpret_cast<const uint4*>(stage + j * 1024 + lane * 32);
-      kb = *reinterpret_cast<const uint4*>(stage + j * 1024 + lane * 32 + 16);
-    }
-    float k[16];
-    k[0] = bf16_lo(ka.x); k[1] = bf16_hi(ka.x); k[2] = bf16_lo(ka.y); k[3] = bf16_hi(ka.y);
-    k[4] = bf16_lo(ka.z); k[5] = bf16_hi(ka.z); k[6] = bf16_lo(ka.w); k[7] = bf16_hi(ka.w);
-    k[8] = bf16_lo(kb.x); k[9] = bf16_hi(kb.x); k[10] = bf16_lo(kb.y); k[11] = bf16_hi(kb.y);
-    k[12] = bf16_lo(kb.z); k[13] = bf16_hi(kb.z); k[14] = bf16_lo(kb.w); k[15] = bf16_hi(kb.w);
-    float sc = 0.0f;
-#pragma unroll
-    for (int h = 0; h < kIdxHeads; ++h) {
-      float p = 0.0f;
-#pragma unroll
-      for (int jj = 0; jj < 16; ++jj) p = fmaf(q[h][jj], k[jj], p);
-      p += __shfl_xor_sync(0xffffffffu, p, 1);
-      p += __shfl_xor_sync(0xffffffffu, p, 2);
-      sc = fmaf(w[h], fmaxf(p, 0.0f), sc);
-    }
-    if (u < nunits && (lane & 3) == 0)
-      scores[(int64_t)r * stride + u * kBlock + row] = row < urows[j] ? sc : -INFINITY;
-  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -229,15 +245,10 @@ struct __align__(16) TopkSmem {
   uint32_t bucket, above, nvalid, ncand;
 };
 
-// Histogram increment aggregated over the lanes of a warp that hit the same
-// bin (scores cluster in few top-digit bins; one atomic per distinct bin).
-// Every lane of the warp must call this.
+// Histogram increment (plain shared-memory atomics measured faster here than
+// aggregating equal bins across a warp with match_any).
 __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool pred) {
-  const uint32_t active = __ballot_sync(0xffffffffu, pred);
-  if (pred) {
-    const uint32_t peers = __match_any_sync(active, bin);
-    if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
-  }
+  if (pred) atomicAdd(&hist[bin], 1u);
 }
 
 // Find the bucket holding the k_rem-th largest element of a histogram of
