@@ -3,36 +3,41 @@
 // A query attends over its selected positions joined with the 128-token
 // sliding window (agentnet.co.il, "דיפסיק משיקה את V4.1-פלאש ...", sections
 // "CSA2: דחיסה לאורך ציר השכבות" and "ארכיטקטורה שחותכת בחצי את הפריפיל").
-// The selection is ascending, so the selected positions below the window
-// start form a prefix of the index row and the attended list is
-//   rows [0, n_sel)           = idx[0 .. n_sel)      (positions < w0)
-//   rows [n_sel, n_sel + W')  = w0 .. v-1            (the window)
-// with every position listed once (at most 640 rows).
+// Every query has 640 candidate slots: slot j < 512 holds idx[j] (used when
+// 0 <= idx[j] < w0, the window start), slot 512 + i holds position w0 + i
+// (used when it is below the visible length v).  The used slots list every
+// attended position exactly once.
 //
-// Work split: a query's row list is cut into S contiguous ranges, one CTA
-// each (S chosen so that the grid fills the GPU; S = 1 for large batches).
-// A CTA walks its range in 64-row tiles through a warp-specialised pipeline:
-//   * producer warps (8) gather the tile's 288-B FP4 rows (16 lanes per row,
-//     coalesced) and decode them to bf16 straight into one of two shared-
-//     memory buffers in the UMMA 128-byte-swizzle K-major layout; every
-//     E2M1 x E4M3 product is exact in bf16 (byte-permute lookup of the E2M1
-//     magnitude, one bf16x2 multiply by the group scale);
+// Work split: the 640 slots of a query are cut into S contiguous ranges, one
+// CTA each (S chosen so that the grid fills the GPU; S = 1 for large
+// batches).  A CTA compacts the used slots of its range into a row list and
+// walks it in 64-row tiles through a warp-specialised pipeline:
+//   * producer warps (8) keep the FP4 bytes of the next two tiles in flight
+//     in registers while they decode the current tile to bf16 (16 lanes per
+//     288-B row, coalesced) into one of two shared-memory buffers in the UMMA
+//     128-byte-swizzle K-major layout; every E2M1 x E4M3 product is exact in
+//     bf16 (byte-permute lookup of the E2M1 magnitude, one bf16x2 multiply by
+//     the group scale);
 //   * one MMA thread issues S^T = K^ . Q^T (tcgen05.mma, M = 64 rows, N = 64
 //     heads, K = 512) into one of two TMEM score buffers -- the next tile's
 //     QK runs while the current tile's softmax does -- and, once P^T is
 //     ready, O^T += V^T . P^T (M = 128 channels x 4, N = 64, K = 64) into a
 //     TMEM accumulator that persists across the CTA's tiles (V = K^, read
-//     MN-major from the same bytes);
-//   * softmax warps (4, one per TMEM sub-partition) keep a running max m and
-//     sum l per head (online softmax).  The max used for the exponentials is
-//     only moved when a tile exceeds it by more than 8 (natural log), and
-//     then O^T and l are rescaled in place, so exponentials stay <= e^8 and
-//     the final O / l is exact up to rounding.
+//     MN-major from the same bytes), plus l += 1^T . P^T (a ones row) so that
+//     the softmax denominator comes from the same bf16 weights as O;
+//   * softmax warps (4, one per TMEM sub-partition, all 32 lanes busy) keep
+//     a running max m per head in base-2 units.  It is moved only when a
+//     score exceeds it by more than kSlack2 (then O^T and l are rescaled in
+//     place), so the weights 2^(s - m) stay below 2^kSlack2 and the final
+//     O / l is exact up to rounding.
 // With S = 1 the CTA writes the normalised bf16 output; otherwise it writes
-// (m, l, O) and a combine kernel merges the S ranges (log-sum-exp).
-// Hand-offs use mbarriers (tcgen05.commit for tensor-core completion); every
-// wait is bounded and reports CSA2_DEVERR_TIMEOUT instead of hanging.
+// (m, l, O) and a combine kernel merges the S ranges (log-sum-exp).  Results
+// leave through shared memory with one bulk copy.  Hand-offs use mbarriers
+// (tcgen05.commit for tensor-core completion); every wait is bounded and
+// reports CSA2_DEVERR_TIMEOUT instead of hanging.
 #include "common.cuh"
+
+#include <cuda_fp16.h>
 
 namespace csa2 {
 
@@ -49,30 +54,36 @@ constexpr int kSmxThreads = 32 * kSoftmaxWarps;        // 128
 constexpr uint32_t kQsBytes = 8u * kHeadsMma * 128u;   // 64 KiB: Q [64 heads x 512], 8 channel blocks
 constexpr uint32_t kKtBytes = 8u * kRowTile * 128u;    // 64 KiB: K^ tile [64 rows x 512]
 constexpr uint32_t kPtBytes = kRowTile * 128u;         // 8 KiB: P^T tile [64 rows x 64 heads]
+constexpr uint32_t kOnesBytes = 64u * 128u;            // 8 KiB: [64 x 64] bf16, row 0 ones, K-major
 constexpr uint32_t kOffQs = 0;
-constexpr uint32_t kOffK = kOffQs + kQsBytes;          // two K^ buffers
+constexpr uint32_t kOffK = kOffQs + kQsBytes;          // two K^ buffers (result staging at the end)
 constexpr uint32_t kOffP = kOffK + 2 * kKtBytes;       // two P^T buffers
-constexpr uint32_t kOffRedM = kOffP + 2 * kPtBytes;    // float [4][64] tile max per warp
-constexpr uint32_t kOffRedL = kOffRedM + 1024;         // float [4][64] tile sum per warp
-constexpr uint32_t kOffRun = kOffRedL + 1024;          // float m_run[64], l_run[64], fac[64], m_tile[64]
+constexpr uint32_t kOffOnes = kOffP + 2 * kPtBytes;
+constexpr uint32_t kOffRedM = kOffOnes + kOnesBytes;   // float [4][64] tile max per warp
+constexpr uint32_t kOffRun = kOffRedM + 1024;          // float m_run[64], fac[64], l[64], f[64]
 constexpr uint32_t kOffRows = kOffRun + 1024;          // uint32 physical row ids [640]
-constexpr uint32_t kOffBar = kOffRows + 4u * kMaxRows; // 8 mbarriers, TMEM base, counters
-constexpr uint32_t kPipeSmem = kOffBar + 128 + 1024;   // + slack for 1024-B alignment
-constexpr uint32_t kTmemCols = 512;                    // S^T 2 x 64 + O^T 4 x 64 = 384, rounded up
+constexpr uint32_t kOffMl = kOffRows + 4u * kMaxRows;  // float2 [8 ranks][64 heads]: the cluster's (m, l)
+constexpr uint32_t kOffBar = kOffMl + 8u * 64u * 8u;   // 9 mbarriers
+constexpr uint32_t kOffMisc = kOffBar + 80;            // 44 words: TMEM base, counters
+constexpr uint32_t kPipeSmem = kOffBar + 256 + 1024;   // + slack for 1024-B alignment
+constexpr uint32_t kTmemCols = 512;                    // S^T 2x64 + O^T 4x64 + l 64 = 448, rounded up
 constexpr uint32_t kColO = 128;                        // first O^T column
+constexpr uint32_t kColL = 384;                        // l row (TMEM lane 0)
 constexpr uint32_t kNoRow = 0xFFFFFFFFu;
-constexpr float kRescaleSlack = 8.0f;                  // natural-log headroom before the max moves
+constexpr float kSlack2 = 12.0f;                       // base-2 headroom before the max moves
+static_assert(kPipeSmem <= 232448, "shared memory budget");
 
 // Instruction descriptors for tcgen05.mma kind::f16: D fp32 (bits 4-5 = 1),
-// A and B bf16 (bits 7-9 = 1, 10-12 = 1), N>>3 at bit 17, M>>4 at bit 24;
-// bit 15 / 16 = A / B are MN-major.
-constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) |
-                              ((uint32_t)(kHeadsMma >> 3) << 17) | ((uint32_t)(kRowTile >> 4) << 24);
-constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
-                              ((uint32_t)(kHeadsMma >> 3) << 17) | (8u << 24);
+// A and B f16 (type fields at bits 7-9 and 10-12 = 0), N>>3 at bit 17,
+// M>>4 at bit 24; bit 15 / 16 = A / B are MN-major.
+constexpr uint32_t kIdescQK = (1u << 4) | ((uint32_t)(kHeadsMma >> 3) << 17) | ((uint32_t)(kRowTile >> 4) << 24);
+constexpr uint32_t kIdescPV = (1u << 4) | (1u << 15) | (1u << 16) | ((uint32_t)(kHeadsMma >> 3) << 17) | (8u << 24);
+// l: A = ones row (K-major, M = 64), B = P^T (MN-major), N = 64.
+constexpr uint32_t kIdescL = (1u << 4) | (1u << 16) | ((uint32_t)(kHeadsMma >> 3) << 17) | ((uint32_t)(64 >> 4) << 24);
 
 
-constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr uint32_t kWaitLimit = 1u << 22;    // try_wait rounds before a wait gives up
+constexpr uint32_t kPollLimit = 1u << 26;    // idle polls of the MMA thread before it gives up
 
 // Shared-memory matrix descriptor: start address, leading and stride byte
 // offsets (16-B units), descriptor version 1, 128-byte swizzle.
@@ -81,7 +92,7 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
                                          uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
@@ -92,6 +103,18 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b
 __device__ __forceinline__ void mma_commit(uint32_t mbar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
                : "memory");
+}
+
+// Non-blocking check of an mbarrier phase.
+__device__ __forceinline__ bool mbar_test(uint32_t mbar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(mbar), "r"(parity)
+      : "memory");
+  return ok != 0;
 }
 
 __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
@@ -130,71 +153,35 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
-
-__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t d;
   asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(d) : "f"(lo), "f"(hi));
   return d;
 }
 
-// Four E2M1 codes (16 bits, channel i in bits 4i..4i+3) -> two bf16x2 words of
-// the unscaled values.  The 8 magnitudes' bf16 bytes are byte-permute tables:
-// low bytes {00,00,80,C0,00,40,80,C0}, high bytes {00,3F,3F,3F,40,40,40,40}
-// for 0, .5, 1, 1.5, 2, 3, 4, 6; the code's bit 3 becomes the bf16 sign.
-// The four sign bits (code bits 3, 7, 11, 15) are moved to bit 7 of the
-// matching high byte via the byte pattern [b0, b0, b1, b1] of the codes.
-__device__ __forceinline__ void e2m1x4_to_bf16(uint32_t c16, uint32_t& w0, uint32_t& w1) {
-  const uint32_t sel = c16 & 0x7777u;
-  const uint32_t lo = __byte_perm(0xC0800000u, 0xC0804000u, sel);
-  const uint32_t dup = __byte_perm(c16, 0u, 0x1100);
-  const uint32_t hi = __byte_perm(0x3F3F3F00u, 0x40404040u, sel) | (dup & 0x80008000u) |
-                      ((dup << 4) & 0x00800080u);
-  w0 = __byte_perm(lo, hi, 0x5140);
-  w1 = __byte_perm(lo, hi, 0x7362);
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %2, %1;" : "=r"(d) : "f"(lo), "f"(hi));
+  return d;
 }
 
-// 8 decoded channels (one 16-B chunk): codes word (4 bytes) x scale (bf16x2).
-__device__ __forceinline__ uint4 decode8(uint32_t codes, uint32_t scale2) {
-  uint4 o;
-  uint32_t a, b;
-  e2m1x4_to_bf16(codes & 0xFFFFu, a, b);
-  o.x = mul_bf16x2(a, scale2);
-  o.y = mul_bf16x2(b, scale2);
-  e2m1x4_to_bf16(codes >> 16, a, b);
-  o.z = mul_bf16x2(a, scale2);
-  o.w = mul_bf16x2(b, scale2);
-  return o;
+// One code word (8 E2M1 values, channel 2j in the low nibble of byte j) times
+// its group scale (f16x2, both halves equal) -> 8 f16 values.  E2M1 -> f16 and
+// E4M3 -> f16 are exact hardware conversions, and every product (at most 6
+// significant bits, magnitude in [2^-10, 2688]) is exact in f16.
+__device__ __forceinline__ uint4 decode8_f16(uint32_t codes, uint32_t scale2) {
+  uint32_t d0, d1, d2, d3;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}\n"
+      : "=r"(d0), "=r"(d1), "=r"(d2), "=r"(d3)
+      : "r"(codes));
+  asm("mul.rn.f16x2 %0, %0, %1;" : "+r"(d0) : "r"(scale2));
+  asm("mul.rn.f16x2 %0, %0, %1;" : "+r"(d1) : "r"(scale2));
+  asm("mul.rn.f16x2 %0, %0, %1;" : "+r"(d2) : "r"(scale2));
+  asm("mul.rn.f16x2 %0, %0, %1;" : "+r"(d3) : "r"(scale2));
+  return make_uint4(d0, d1, d2, d3);
 }
-
-// Lane l ends up with op over the 32 lanes of element l of v (31 shuffles).
-template <bool kMax>
-__device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
-#pragma unroll
-  for (int w = 16; w >= 1; w >>= 1) {
-    const bool up = (lane & w) != 0;
-#pragma unroll
-    for (int i = 0; i < w; ++i) {
-      const float send = up ? v[i] : v[i + w];
-      const float keep = up ? v[i + w] : v[i];
-      const float recv = __shfl_xor_sync(0xffffffffu, send, w);
-      v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
-    }
-  }
-  return v[0];
-}
-
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
@@ -232,118 +219,264 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       : "memory");
 }
 
-// Over lanes 0..15 (and separately 16..31): lane l ends with op over the 16
-// lanes of elements 4(l%16) .. 4(l%16)+3 of v[64] (60 shuffles).
-template <bool kMax>
-__device__ __forceinline__ void reduce_scatter16x64(float (&v)[64], int lane, float (&res)[4]) {
+// 32 fp32 TMEM columns from one 16-lane half of a sub-partition (the rows of
+// an M = 64 accumulator): thread t < 16 reads lane base + t, columns
+// col .. col + 31; thread t >= 16 reads lane base + t - 16, columns
+// col + 32 .. col + 63.
+__device__ __forceinline__ void tmem_ld16x2(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], 32;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 2^x (hardware approximation, relative error ~2^-22; 2^-inf = 0).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Max over the 16 lanes of each half-warp, scattered: lane l ends with the
+// maxima of elements 2(l%16) and 2(l%16)+1 in v[0], v[1] (30 shuffles).
+__device__ __forceinline__ void max_scatter32x16(float (&v)[32], int lane) {
 #pragma unroll
   for (int w = 8; w >= 1; w >>= 1) {
     const bool up = (lane & w) != 0;
 #pragma unroll
-    for (int i = 0; i < 4 * w; ++i) {
-      const float send = up ? v[i] : v[i + 4 * w];
-      const float keep = up ? v[i + 4 * w] : v[i];
-      const float recv = __shfl_xor_sync(0xffffffffu, send, w);
-      v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+    for (int i = 0; i < 2 * w; ++i) {
+      const float send = up ? v[i] : v[i + 2 * w];
+      const float keep = up ? v[i + 2 * w] : v[i];
+      v[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, w));
     }
   }
+}
+
+// Bulk prefetch of a 16-B aligned range (size a multiple of 16) into L2.
+__device__ __forceinline__ void l2_prefetch_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Thread-block cluster: barrier over all threads of the cluster, address of
+// the same shared-memory offset in CTA `rank`, and accesses through it.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_v2(uint32_t addr, float a, float b) {
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
+}
+
+// Shared -> global bulk copy through the async proxy; returns once the
+// shared-memory source has been read (the writes complete with the grid).
+__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "r"(bytes)
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+__device__ __forceinline__ uint4 ld_nc16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+// 16-B load through L2 only (data written by other CTAs of this grid).
+__device__ __forceinline__ uint4 ld_cg16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t ld_nc_u32(const void* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
+// Producer thread layout for one 64-row tile: 16 lanes per row, lane
+// `piece` (0..15) takes the 16-B code chunk `piece` (32 channels) and the two
+// scale bytes of those channels; thread rsub (0..15) of a piece takes rows
+// rsub + 16 it, it = 0..3.  A warp load then covers two rows' 256 contiguous
+// code bytes (few cache lines per instruction).
+struct RawTile {
+  uint4 c[4];       // code chunk of rows rsub + 16 it
+  uint32_t s[4];    // the 4-B scale word holding its two scale bytes
+};
+
+__device__ __forceinline__ void raw_load(RawTile& R, const uint8_t* __restrict__ kv, const uint32_t* rows_s,
+                                         int t, int nrow, int rsub, int piece) {
 #pragma unroll
-  for (int e = 0; e < 4; ++e) res[e] = v[e];
+  for (int it = 0; it < 4; ++it) {
+    const int li = t * kRowTile + rsub + 16 * it;
+    const uint32_t id = li < nrow ? rows_s[li] : kNoRow;
+    if (id != kNoRow) {
+      const uint8_t* rp = kv + (int64_t)id * kRowBytes;
+      R.c[it] = ld_nc16(rp + piece * 16);
+      R.s[it] = ld_nc_u32(rp + kCodeBytes + (piece >> 1) * 4);
+    } else {   // zero codes and zero scales decode to zeros
+      R.c[it] = make_uint4(0, 0, 0, 0);
+      R.s[it] = 0;
+    }
+  }
+}
+
+// Decode into the swizzled K^ buffer at kbuf (channel block kb = piece >> 1,
+// 16-B columns 4 (piece & 1) + j).  The four output words are produced in
+// the order j = (jj + kb) & 3 so that the 8 lanes of a quarter-warp (same
+// row, 4 channel blocks) store to 8 different bank groups.  soff[jj] is the
+// byte offset of column 4 (piece & 1) + ((jj + kb) & 3) within the swizzled row.
+__device__ __forceinline__ void raw_decode(const RawTile& R, uint8_t* sp, uint32_t kbuf, int rsub, int piece,
+                                           const uint32_t (&soff)[4]) {
+  const int kb = piece >> 1, rot = kb & 3;
+  const uint32_t base = kbuf + (uint32_t)kb * (kRowTile * 128u) + (uint32_t)rsub * 128u;
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    // rotate the code words by rot; words 0, 1 use scale byte 0, words 2, 3 byte 1
+    uint32_t w0 = R.c[it].x, w1 = R.c[it].y, w2 = R.c[it].z, w3 = R.c[it].w;
+    if (rot & 1) { const uint32_t t = w0; w0 = w1; w1 = w2; w2 = w3; w3 = t; }
+    if (rot & 2) { uint32_t t = w0; w0 = w2; w2 = t; t = w1; w1 = w3; w3 = t; }
+    const uint32_t sc16 = (piece & 1) ? (R.s[it] >> 16) : (R.s[it] & 0xFFFFu);
+    uint32_t sc, s0, s1;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(sc) : "h"((unsigned short)sc16));
+    s0 = __byte_perm(sc, 0u, 0x1010);
+    s1 = __byte_perm(sc, 0u, 0x3232);
+    const uint32_t cw[4] = {w0, w1, w2, w3};
+    const uint32_t rowb = base + (uint32_t)(16 * it) * 128u;
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const uint32_t sj = ((jj + rot) & 2) ? s1 : s0;
+      *reinterpret_cast<uint4*>(sp + rowb + soff[jj]) = decode8_f16(cw[jj], sj);
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kPipeThreads, 1)
 attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_scale,
                  const int32_t* __restrict__ q_seq, const int32_t* __restrict__ q_vis,
-                 const int32_t* __restrict__ idx, int nsplit, int range_rows,
-                 uint16_t* __restrict__ out, float* __restrict__ part_o, float2* __restrict__ part_ml) {
+                 const int32_t* __restrict__ idx, int nsplit, int range_slots, uint16_t* __restrict__ out,
+                 uint16_t* __restrict__ part) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw_s = (uint32_t)__cvta_generic_to_shared(smem_raw);
   const uint32_t sb = (raw_s + 1023u) & ~1023u;            // 1024-B aligned base (swizzle atoms)
   uint8_t* const sp = smem_raw + (sb - raw_s);
   float* const red_m = reinterpret_cast<float*>(sp + kOffRedM);
-  float* const red_l = reinterpret_cast<float*>(sp + kOffRedL);
-  float* const m_run = reinterpret_cast<float*>(sp + kOffRun);
-  float* const l_run = m_run + 64;
-  float* const fac = m_run + 128;
-  float* const m_tile = m_run + 192;
+  float* const m_run = reinterpret_cast<float*>(sp + kOffRun);   // base-2 running max per head
+  float* const fac = m_run + 64;
+  float* const l_s = m_run + 128;
+  float* const f_s = m_run + 192;                                 // output factor per head
   uint32_t* const rows_s = reinterpret_cast<uint32_t*>(sp + kOffRows);
-  uint32_t* const misc = reinterpret_cast<uint32_t*>(sp + kOffBar + 64);   // [0] tmem, [1] n_sel, [2] flags
+  // [0] TMEM base, [1] last barrier the MMA thread committed to (0: none), [2] its parity,
+  // [4 + w] used-slot count of warp w, [20 + w] largest |q| bits seen by warp w
+  uint32_t* const misc = reinterpret_cast<uint32_t*>(sp + kOffMisc);
   const uint32_t bar0 = sb + kOffBar;
   auto kfull = [&](int b) { return bar0 + 8u * b; };
   auto kempty = [&](int b) { return bar0 + 16u + 8u * b; };
   auto sfull = [&](int b) { return bar0 + 32u + 8u * b; };
   auto pfull = [&](int b) { return bar0 + 48u + 8u * b; };
+  const uint32_t qready = bar0 + 64u;
 
-  const int split = blockIdx.x;
+  const int split = blockIdx.x;                            // rank in the query's cluster
   const int r = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int32_t* idx_row = idx + (int64_t)r * kTopK;
+  // the cluster's CTAs all run before any touches another's shared memory:
+  // arrive now, wait just before the first remote access
+  if (nsplit > 1) cluster_arrive_relaxed();
+
+  // the query's bf16 rows, 16-B chunk e = tid + kPipeThreads * i (heads >= H read as zero);
+  // they are scaled by 2^qexp and stored as f16 once the largest magnitude is known
+  constexpr int kQChunks = kHeadsMma * (kD / 8);                     // 4096
+  constexpr int kQPerThread = (kQChunks + kPipeThreads - 1) / kPipeThreads;   // 10
+  uint4 qv[kQPerThread];
+  {
+    const uint4* qsrc = reinterpret_cast<const uint4*>(q + (int64_t)r * H * kD);
+#pragma unroll
+    for (int i = 0; i < kQPerThread; ++i) {
+      const int e = tid + kPipeThreads * i;
+      qv[i] = (e < kQChunks && (e >> 6) < H) ? ld_nc16(qsrc + e) : make_uint4(0, 0, 0, 0);
+    }
+  }
+  // ones row for the softmax denominator: row 0 of a K-major [64 x 64] f16 tile
+  for (int e = tid; e < (int)(kOnesBytes / 16); e += kPipeThreads)
+    *reinterpret_cast<uint4*>(sp + kOffOnes + 16 * e) =
+        e < 8 ? make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u) : make_uint4(0, 0, 0, 0);
+
+  // this CTA's candidate slots; thread tid takes slots lo + 2 tid and lo + 2 tid + 1
+  const int lo = split * range_slots;
+  const int hi = min(lo + range_slots, kMaxRows);
+  const int s0 = lo + 2 * tid;
+  int32_t e0 = -1, e1 = -1;
+  if (s0 < hi && s0 < kTopK) e0 = idx_row[s0];
+  if (s0 + 1 < hi && s0 + 1 < kTopK) e1 = idx_row[s0 + 1];
   const int seq = q_seq[r];
   const int64_t v = q_vis ? (int64_t)q_vis[r] : (int64_t)seq_len_of(c, seq);
   const int64_t w0 = v > kWindow ? v - kWindow : 0;
-  const int32_t* idx_row = idx + (int64_t)r * kTopK;
-
-  // query -> Q (K-major, 128-B swizzle), asynchronous; heads >= H are zero
-  {
-    const uint4* qsrc = reinterpret_cast<const uint4*>(q + (int64_t)r * H * kD);
-    for (int e = tid; e < kHeadsMma * (kD / 8); e += kPipeThreads) {
-      const int h = e >> 6, c16 = e & 63, kb = c16 >> 3, j = c16 & 7;
-      const uint32_t off = kOffQs + kb * (kHeadsMma * 128u) + (h >> 3) * 1024u + (h & 7) * 128u +
-                           ((j ^ (h & 7)) << 4);
-      if (h < H) cp_async16(sb + off, qsrc + (h * (kD / 8) + c16));
-      else *reinterpret_cast<uint4*>(sp + off) = make_uint4(0, 0, 0, 0);
-    }
-  }
-  // selected positions below the window (a prefix of the ascending row)
-  if (tid == 0) {
-    misc[1] = 0;
-    misc[2] = 0;
-    misc[3] = 0;   // last barrier the MMA thread committed to (0: none)
-    misc[4] = 0;
-  }
-  __syncthreads();
-  {
-    int cnt = 0;
-    for (int j = tid; j < kTopK; j += kPipeThreads) {
-      const int32_t e = idx_row[j];
+  auto slot_pos = [&](int sl, int32_t e) -> int64_t {   // attended position of a slot, -1 if unused
+    if (sl >= hi) return -1;
+    if (sl < kTopK) {
       if (e >= v) raise_error(c.err, CSA2_DEVERR_POS);
-      cnt += (e >= 0 && e < w0) ? 1 : 0;
+      return (e >= 0 && e < w0) ? (int64_t)e : -1;
     }
+    const int64_t p = w0 + (sl - kTopK);
+    return p < v ? p : -1;
+  };
+  const int64_t p0 = slot_pos(s0, e0), p1 = slot_pos(s0 + 1, e1);
+  uint32_t id0 = kNoRow, id1 = kNoRow;
+  if (p0 >= 0) {
+    const int64_t pg = page_of(c, seq, p0);
+    if (pg >= 0) id0 = (uint32_t)(pg * kPageTokens + (p0 & (kPageTokens - 1)));
+  }
+  if (p1 >= 0) {
+    const int64_t pg = page_of(c, seq, p1);
+    if (pg >= 0) id1 = (uint32_t)(pg * kPageTokens + (p1 & (kPageTokens - 1)));
+  }
+  // largest |q| of the warp (the loads above were in flight meanwhile)
+  uint32_t qmax = 0;   // as bf16 bits: magnitudes order like their bit patterns
+  {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-    if (lane == 0 && cnt) atomicAdd(&misc[1], (uint32_t)cnt);
-  }
-  __syncthreads();
-  const int n_sel = (int)misc[1];
-  const int64_t n_rows = n_sel + (v - w0);
-  const int64_t rb = (int64_t)split * range_rows;
-  const int64_t re = min(rb + (int64_t)range_rows, n_rows);
-  if (rb >= re) {   // nothing to attend in this range: no TMEM is touched
-    if (nsplit > 1) {
-      float2* ml = part_ml + ((int64_t)r * nsplit + split) * H;
-      for (int h = tid; h < H; h += kPipeThreads) ml[h] = make_float2(-INFINITY, 0.0f);
-    } else {
-      for (int e = tid; e < H * (kD / 8); e += kPipeThreads)
-        reinterpret_cast<uint4*>(out + (int64_t)r * H * kD)[e] = make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < kQPerThread; ++i) {
+      qmax = __vmaxu2(qmax, qv[i].x & 0x7FFF7FFFu);
+      qmax = __vmaxu2(qmax, qv[i].y & 0x7FFF7FFFu);
+      qmax = __vmaxu2(qmax, qv[i].z & 0x7FFF7FFFu);
+      qmax = __vmaxu2(qmax, qv[i].w & 0x7FFF7FFFu);
     }
-    cp_async_wait_all();
-    return;
+    qmax = max(qmax & 0xFFFFu, qmax >> 16);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) qmax = max(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
   }
-  const int nrow = (int)(re - rb);
-  const int nt = (nrow + kRowTile - 1) / kRowTile;
-
-  // physical row ids of the range
-  for (int i = tid; i < nrow; i += kPipeThreads) {
-    const int64_t li = rb + i;
-    const int32_t p = li < n_sel ? idx_row[li] : (int32_t)(w0 + (li - n_sel));
-    uint32_t id = kNoRow;
-    if (p >= 0) {
-      const int64_t pg = page_of(c, seq, p);
-      if (pg >= 0) id = (uint32_t)(pg * kPageTokens + (p & (kPageTokens - 1)));
-    }
-    rows_s[i] = id;
+  // compact the used slots (in slot order) into rows_s
+  const uint32_t cnt = (p0 >= 0 ? 1u : 0u) + (p1 >= 0 ? 1u : 0u);
+  uint32_t incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
   }
+  if (lane == 31) misc[4 + warp] = incl;
+  if (lane == 0) misc[20 + warp] = qmax;
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sb + kOffBar + 64),
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sb + kOffMisc),
                  "r"(kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
@@ -354,255 +487,388 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
       mbar_init(sfull(b), 1);
       mbar_init(pfull(b), kSmxThreads);
     }
+    mbar_init(qready, kPipeThreads);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    misc[1] = 0;
+    misc[2] = 0;
   }
-  cp_async_wait_all();
-  fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  uint32_t before = 0, total = 0;
+#pragma unroll 1
+  for (int w = 0; w <= kMmaWarp; ++w) {
+    const uint32_t x = misc[4 + w];
+    before += w < warp ? x : 0u;
+    total += x;
+    qmax = max(qmax, misc[20 + w]);
+  }
+  {
+    const uint32_t at = before + incl - cnt;
+    if (p0 >= 0) rows_s[at] = id0;
+    if (p1 >= 0) rows_s[at + (p0 >= 0 ? 1u : 0u)] = id1;
+    // start the rows on their way into L2 while the pipeline sets up
+    if (id0 != kNoRow) l2_prefetch_bulk(c.kv + (int64_t)id0 * kRowBytes, kRowBytes);
+    if (id1 != kNoRow) l2_prefetch_bulk(c.kv + (int64_t)id1 * kRowBytes, kRowBytes);
+  }
+  // Q in f16 scaled by 2^qexp so that the largest |q| lies in [2^14, 2^15):
+  // exact for every element of magnitude >= 2^-28 of the largest; the scores
+  // are scaled back in the softmax.
+  const int qexp = qmax == 0 ? 0 : max(-100, min(100, 141 - (int)(qmax >> 7)));
+  auto store_q = [&]() {   // this thread's Q chunks -> f16, swizzled K-major; then signal
+    const float qs = __uint_as_float((uint32_t)(127 + qexp) << 23);
+#pragma unroll
+    for (int i = 0; i < kQPerThread; ++i) {
+      const int e = tid + kPipeThreads * i;
+      if (e < kQChunks) {
+        const int h = e >> 6, c16 = e & 63, kb = c16 >> 3, j = c16 & 7;
+        const uint32_t off = kOffQs + kb * (kHeadsMma * 128u) + (h >> 3) * 1024u + (h & 7) * 128u +
+                             ((j ^ (h & 7)) << 4);
+        uint4 o;
+        o.x = pack_f16x2(bf16_lo(qv[i].x) * qs, bf16_hi(qv[i].x) * qs);
+        o.y = pack_f16x2(bf16_lo(qv[i].y) * qs, bf16_hi(qv[i].y) * qs);
+        o.z = pack_f16x2(bf16_lo(qv[i].z) * qs, bf16_hi(qv[i].z) * qs);
+        o.w = pack_f16x2(bf16_lo(qv[i].w) * qs, bf16_hi(qv[i].w) * qs);
+        *reinterpret_cast<uint4*>(sp + off) = o;
+      }
+    }
+    fence_async_smem();
+    mbar_arrive(qready);
+  };
+  const int nrow = (int)total;
+  const int nt = (nrow + kRowTile - 1) / kRowTile;
   const uint32_t tmem = misc[0];
+  fence_async_smem();
+  __syncthreads();
   bool ok = true;
 
   if (warp >= kSoftmaxWarps && warp < kMmaWarp) {
     // ---------------- producers: gather + decode ----------------
     const int ptid = tid - kSmxThreads;
-    const int piece = ptid & 15, rsub = ptid >> 4;       // 16 lanes per row, 16 rows per round
-    const int kb = piece >> 1, half = piece & 1;
-    for (int t = 0; t < nt && ok; ++t) {
+    const int piece = ptid & 15, rsub = ptid >> 4;
+    uint32_t soff[4];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj)
+      soff[jj] = (uint32_t)((((piece & 1) * 4 + ((jj + (piece >> 1)) & 3)) ^ (rsub & 7)) << 4);
+    // tile t's bytes sit in A, B, C for t % 3 = 0, 1, 2; tile t + 2 is loaded
+    // before tile t is decoded
+    RawTile A, B, C;
+    if (nt > 0) raw_load(A, c.kv, rows_s, 0, nrow, rsub, piece);
+    if (nt > 1) raw_load(B, c.kv, rows_s, 1, nrow, rsub, piece);
+    store_q();
+    auto step = [&](int t, RawTile& D, RawTile& L) -> bool {
+      if (t + 2 < nt) raw_load(L, c.kv, rows_s, t + 2, nrow, rsub, piece);
       const int b = t & 1;
-      if (t >= 2 && !mbar_wait(kempty(b), ((t - 2) >> 1) & 1)) { ok = false; break; }
-      uint4 cw[4];
-      uint32_t sw[4];
-      bool have[4];
-#pragma unroll
-      for (int it = 0; it < 4; ++it) {
-        const int row = rsub + 16 * it;
-        const int li = t * kRowTile + row;
-        const uint32_t id = li < nrow ? rows_s[li] : kNoRow;
-        have[it] = id != kNoRow;
-        if (have[it]) {
-          const uint8_t* rp = c.kv + (int64_t)id * kRowBytes;
-          cw[it] = __ldg(reinterpret_cast<const uint4*>(rp + piece * 16));
-          sw[it] = __ldg(reinterpret_cast<const unsigned short*>(rp + kCodeBytes + piece * 2));
-        } else {
-          cw[it] = make_uint4(0, 0, 0, 0);
-          sw[it] = 0;
-        }
-      }
-      const uint32_t kbase = kOffK + b * kKtBytes + kb * (kRowTile * 128u);
-#pragma unroll
-      for (int it = 0; it < 4; ++it) {
-        const int row = rsub + 16 * it;
-        const uint32_t base = kbase + (row >> 3) * 1024u + (row & 7) * 128u;
-        const uint32_t sb0 = __float_as_uint(e4m3_pos_value(sw[it] & 0x7Fu)) >> 16;
-        const uint32_t sb1 = __float_as_uint(e4m3_pos_value((sw[it] >> 8) & 0x7Fu)) >> 16;
-        const uint32_t s20 = sb0 | (sb0 << 16), s21 = sb1 | (sb1 << 16);
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const int j = (jj + kb) & 3;                   // rotate the store order (bank spread)
-          const uint32_t cj = j == 0 ? cw[it].x : j == 1 ? cw[it].y : j == 2 ? cw[it].z : cw[it].w;
-          const uint4 val = have[it] ? decode8(cj, j < 2 ? s20 : s21) : make_uint4(0, 0, 0, 0);
-          const int chunk = half * 4 + j;
-          *reinterpret_cast<uint4*>(sp + base + ((chunk ^ (row & 7)) << 4)) = val;
-        }
-      }
+      if (t >= 2 && !mbar_wait(kempty(b), ((t - 2) >> 1) & 1)) return false;
+      raw_decode(D, sp, kOffK + b * kKtBytes, rsub, piece, soff);
       fence_async_smem();
       mbar_arrive(kfull(b));
+      return true;
+    };
+#pragma unroll 1
+    for (int t = 0; t < nt; t += 3) {
+      if (!(ok = step(t, A, C)) || t + 1 >= nt) break;
+      if (!(ok = step(t + 1, B, A)) || t + 2 >= nt) break;
+      if (!(ok = step(t + 2, C, B))) break;
     }
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issue (one thread) ----------------
+    // QK(t) and PV(t) are issued as soon as their inputs are ready, in
+    // whichever order they become ready: QK(t) needs tile t decoded and the
+    // S buffer free (PV(t-2) issued); PV(t) needs P(t).
+    store_q();
     if (lane == 0) {
-      auto issue_qk = [&](int t) -> bool {
-        const int b = t & 1;
-        if (!mbar_wait(kfull(b), (t >> 1) & 1)) return false;
-        tc_fence_after();
-#pragma unroll 1
-        for (int kb = 0; kb < 8; ++kb) {
+      ok = mbar_wait(qready, 0);
+      int nqk = 0, npv = 0;
+      uint32_t idle = 0;
+      while (ok && npv < nt) {
+        bool progressed = false;
+        if (npv < nqk && mbar_test(pfull(npv & 1), (npv >> 1) & 1)) {
+          const int t = npv, b = t & 1;
+          tc_fence_after();
+          // descriptors advance by plain adds of (byte offset >> 4) to the start field
+          const uint64_t a0 = smem_desc(sb + kOffK + b * kKtBytes, kRowTile * 128u, 1024u);
+          const uint64_t p0 = smem_desc(sb + kOffP + b * kPtBytes, 8192u, 1024u);
+          const uint64_t o0 = smem_desc(sb + kOffOnes, 16u, 1024u);
+          const uint32_t acc = t > 0 ? 1u : 0u;
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t a = smem_desc(sb + kOffK + b * kKtBytes + kb * (kRowTile * 128u) + ks * 32u, 16u, 1024u);
-            const uint64_t bq = smem_desc(sb + kOffQs + kb * (kHeadsMma * 128u) + ks * 32u, 16u, 1024u);
-            mma_bf16(tmem + 64u * b, a, bq, kIdescQK, (kb | ks) ? 1u : 0u);
-          }
-        }
-        mma_commit(sfull(b));
-        misc[3] = sfull(b);
-        misc[4] = (t >> 1) & 1;
-        return true;
-      };
-      ok = issue_qk(0);
-      for (int t = 0; t < nt && ok; ++t) {
-        if (t + 1 < nt && !issue_qk(t + 1)) { ok = false; break; }
-        const int b = t & 1;
-        if (!mbar_wait(pfull(b), (t >> 1) & 1)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll 1
-        for (int mt = 0; mt < 4; ++mt) {
+          for (int mt = 0; mt < 4; ++mt) {
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t a = smem_desc(sb + kOffK + b * kKtBytes + (2 * mt) * (kRowTile * 128u) + ks * 2048u,
-                                         kRowTile * 128u, 1024u);
-            const uint64_t bp = smem_desc(sb + kOffP + b * kPtBytes + ks * 2048u, 8192u, 1024u);
-            mma_bf16(tmem + kColO + 64u * mt, a, bp, kIdescPV, (t > 0 || ks > 0) ? 1u : 0u);
+            for (int ks = 0; ks < 4; ++ks)
+              mma_f16(tmem + kColO + 64u * mt, a0 + (((2 * mt) * (kRowTile * 128u) + ks * 2048u) >> 4),
+                      p0 + ((ks * 2048u) >> 4), kIdescPV, (acc | ks) ? 1u : 0u);
           }
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_f16(tmem + kColL, o0 + ((ks * 32u) >> 4), p0 + ((ks * 2048u) >> 4), kIdescL, (acc | ks) ? 1u : 0u);
+          mma_commit(kempty(b));
+          misc[1] = kempty(b);
+          misc[2] = (t >> 1) & 1;
+          ++npv;
+          progressed = true;
         }
-        mma_commit(kempty(b));
-        misc[3] = kempty(b);
-        misc[4] = (t >> 1) & 1;
+        if (nqk < nt && nqk <= npv + 1 && mbar_test(kfull(nqk & 1), (nqk >> 1) & 1)) {
+          const int t = nqk, b = t & 1;
+          tc_fence_after();
+          const uint64_t a0 = smem_desc(sb + kOffK + b * kKtBytes, 16u, 1024u);
+          const uint64_t q0 = smem_desc(sb + kOffQs, 16u, 1024u);
+#pragma unroll
+          for (int kb = 0; kb < 8; ++kb) {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+              mma_f16(tmem + 64u * b, a0 + ((kb * (kRowTile * 128u) + ks * 32u) >> 4),
+                      q0 + ((kb * (kHeadsMma * 128u) + ks * 32u) >> 4), kIdescQK, (kb | ks) ? 1u : 0u);
+          }
+          mma_commit(sfull(b));
+          misc[1] = sfull(b);
+          misc[2] = (t >> 1) & 1;
+          ++nqk;
+          progressed = true;
+        }
+        if (progressed) idle = 0;
+        else if (++idle > kPollLimit) ok = false;
       }
     }
     __syncwarp();
   } else {
     // ---------------- softmax warps 0..3 ----------------
-    const int sw_ = warp;                             // TMEM sub-partition == warp
-    const int hl = lane & 15;
-    const bool lo_half = lane < 16;
+    store_q();
+    const int w = warp;                                // TMEM sub-partition == warp
+    const int rl = lane & 15, hh = lane >> 4;          // tile row 16 w + rl, heads 32 hh .. 32 hh + 31
+    const int row = 16 * w + rl;
     constexpr float kLog2e = 1.4426950408889634f;
+    const float scale2 = sm_scale * kLog2e * __uint_as_float((uint32_t)(127 - qexp) << 23);
+    const float* mr = m_run + 32 * hh;
+    const uint32_t lane_base = (uint32_t)(32 * w) << 16;
     for (int t = 0; t < nt && ok; ++t) {
       const int b = t & 1;
       if (!smx_all(mbar_wait(sfull(b), (t >> 1) & 1))) { ok = false; break; }
       tc_fence_after();
-      const int row = 16 * sw_ + hl;                  // tile row held by lanes 0..15
-      const bool valid = lo_half && (t * kRowTile + row) < nrow;
-      float s[64], w[64];
-      {
-        float a[32];
-        tmem_ld32(tmem + ((uint32_t)(32 * sw_) << 16) + 64u * b, a);
+      float s[32];
+      tmem_ld16x2(tmem + lane_base + 64u * b, s);
+      const bool valid = t * kRowTile + row < nrow;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[i] = a[i];
-        tmem_ld32(tmem + ((uint32_t)(32 * sw_) << 16) + 64u * b + 32u, a);
+      for (int i = 0; i < 32; ++i) s[i] = valid ? s[i] * scale2 : -INFINITY;
+      bool slow = t == 0;
+      if (!slow) {
+        bool exceed = false;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[32 + i] = a[i];
+        for (int i = 0; i < 32; ++i) exceed |= s[i] > mr[i] + kSlack2;
+        slow = !smx_all(!exceed);
       }
+      if (slow) {   // move the running max (uniform over the softmax warps)
+        float x[32];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        s[i] = valid ? s[i] * sm_scale : -INFINITY;
-        w[i] = s[i];
-      }
-      float rr[4];
-      reduce_scatter16x64<true>(w, lane, rr);
-      if (lo_half) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) red_m[sw_ * 64 + 4 * hl + e] = rr[e];
-      }
-      smx_bar();
-      if (tid < 64) {
-        const float mt = fmaxf(fmaxf(red_m[tid], red_m[64 + tid]), fmaxf(red_m[128 + tid], red_m[192 + tid]));
-        m_tile[tid] = mt;
-        if (t > 0 && mt > m_run[tid] + kRescaleSlack) atomicOr(&misc[2], 1u);
-      }
-      smx_bar();
-      const bool rescale = t > 0 && (misc[2] & 1u);
-      if (tid < 64) {
-        const float mt = m_tile[tid];
-        if (t == 0) {
-          m_run[tid] = mt;
-          l_run[tid] = 0.0f;
-          fac[tid] = 1.0f;
-        } else if (rescale) {
-          const float mn = fmaxf(m_run[tid], mt);
-          fac[tid] = (m_run[tid] == -INFINITY) ? 0.0f : exp2f((m_run[tid] - mn) * kLog2e);
-          m_run[tid] = mn;
-          l_run[tid] *= fac[tid];
-        }
-      }
-      smx_bar();
-      if (rescale) {
-        if (tid == 0) misc[2] = 0;
-        // O^T must be complete before it is rescaled: PV of tile t-1
-        if (!smx_all(mbar_wait(kempty((t - 1) & 1), ((t - 1) >> 1) & 1))) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll 1
-        for (int mt = 0; mt < 4; ++mt) {
-#pragma unroll 1
-          for (int hh = 0; hh < 2; ++hh) {
-            float o[32];
-            const uint32_t ta = tmem + ((uint32_t)(32 * sw_) << 16) + kColO + 64u * mt + 32u * hh;
-            tmem_ld32(ta, o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= fac[32 * hh + i];
-            tmem_st32(ta, o);
+        for (int i = 0; i < 32; ++i) x[i] = s[i];
+        max_scatter32x16(x, lane);
+        red_m[w * 64 + 32 * hh + 2 * rl] = x[0];
+        red_m[w * 64 + 32 * hh + 2 * rl + 1] = x[1];
+        smx_bar();
+        if (tid < 64) {
+          const float mt = fmaxf(fmaxf(red_m[tid], red_m[64 + tid]), fmaxf(red_m[128 + tid], red_m[192 + tid]));
+          if (t == 0) {
+            m_run[tid] = mt;
+            fac[tid] = 1.0f;
+          } else {
+            const float mn = fmaxf(m_run[tid], mt);
+            fac[tid] = ex2(m_run[tid] - mn);
+            m_run[tid] = mn;
           }
         }
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-      }
-      // probabilities with the running max (<= e^8 between rescales)
-      float ps[4];
+        smx_bar();
+        if (t > 0) {
+          // O^T and l must be complete before they are rescaled: PV of tile t-1
+          if (!smx_all(mbar_wait(kempty((t - 1) & 1), ((t - 1) >> 1) & 1))) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll 1
+          for (int ct = 0; ct < 5; ++ct) {
+#pragma unroll 1
+            for (int h2 = 0; h2 < 2; ++h2) {
+              float o[32];
+              const uint32_t ta = tmem + lane_base + (ct < 4 ? kColO + 64u * ct : kColL) + 32u * h2;
+              tmem_ld32(ta, o);
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        s[i] = valid ? exp2f((s[i] - m_run[i]) * kLog2e) : 0.0f;
-        w[i] = s[i];
+              for (int i = 0; i < 32; ++i) o[i] *= fac[32 * h2 + i];
+              tmem_st32(ta, o);
+            }
+          }
+          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        }
       }
-      reduce_scatter16x64<false>(w, lane, ps);
-      if (lo_half) {
+      // weights 2^(s - m) <= 2^kSlack2 (0 for unused rows)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) red_l[sw_ * 64 + 4 * hl + e] = ps[e];
-      }
+      for (int i = 0; i < 32; ++i) s[i] = ex2(s[i] - mr[i]);
       // P^T buffer b is free once PV of tile t-2 is done
       if (t >= 2 && !smx_all(mbar_wait(kempty(b), ((t - 2) >> 1) & 1))) { ok = false; break; }
-      if (lo_half) {
+      {
         const uint32_t pbase = kOffP + b * kPtBytes + (row >> 3) * 1024u + (row & 7) * 128u;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 4; ++j) {
           uint4 pk;
-          pk.x = pack_bf16x2(s[8 * j + 0], s[8 * j + 1]);
-          pk.y = pack_bf16x2(s[8 * j + 2], s[8 * j + 3]);
-          pk.z = pack_bf16x2(s[8 * j + 4], s[8 * j + 5]);
-          pk.w = pack_bf16x2(s[8 * j + 6], s[8 * j + 7]);
-          *reinterpret_cast<uint4*>(sp + pbase + ((j ^ (row & 7)) << 4)) = pk;
+          pk.x = pack_f16x2(s[8 * j + 0], s[8 * j + 1]);
+          pk.y = pack_f16x2(s[8 * j + 2], s[8 * j + 3]);
+          pk.z = pack_f16x2(s[8 * j + 4], s[8 * j + 5]);
+          pk.w = pack_f16x2(s[8 * j + 6], s[8 * j + 7]);
+          *reinterpret_cast<uint4*>(sp + pbase + (((4 * hh + j) ^ (row & 7)) << 4)) = pk;
         }
       }
       fence_async_smem();
       tc_fence_before();
       mbar_arrive(pfull(b));
-      smx_bar();
-      if (tid < 64) l_run[tid] += (red_l[tid] + red_l[64 + tid]) + (red_l[128 + tid] + red_l[192 + tid]);
     }
-    // epilogue: the last PV completes O^T
-    ok = smx_all(ok) && smx_all(mbar_wait(kempty((nt - 1) & 1), ((nt - 1) >> 1) & 1));
+    // epilogue: the last PV completes O^T and l
+    ok = smx_all(ok) && (nt == 0 || smx_all(mbar_wait(kempty((nt - 1) & 1), ((nt - 1) >> 1) & 1)));
     tc_fence_after();
-    if (__all_sync(0xffffffffu, ok)) {
-      const int chl = 32 * sw_ + lane;                 // channel within a 128-channel tile
-#pragma unroll 1
-      for (int mt = 0; mt < 4; ++mt) {
-#pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {
-          if (32 * hh >= H) continue;
-          float o[32];
-          tmem_ld32(tmem + ((uint32_t)(32 * sw_) << 16) + kColO + 64u * mt + 32u * hh, o);
-          const int ch = 128 * mt + chl;
-          if (nsplit == 1) {
+    if (ok) {
+      if (nt > 0) {
+        if (w == 0) {   // l sits in TMEM lane 0
+          float a[32];
+          tmem_ld32(tmem + kColL, a);
+          if (lane == 0) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int h = 32 * hh + i;
-              if (h < H) {
-                const float l = l_run[h];
-                out[((int64_t)r * H + h) * kD + ch] = f32_to_bf16_rne(l > 0.0f ? o[i] / l : 0.0f);
-              }
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(l_s + i) = make_float4(a[i], a[i + 1], a[i + 2], a[i + 3]);
+          }
+          tmem_ld32(tmem + kColL + 32u, a);
+          if (lane == 0) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(l_s + 32 + i) = make_float4(a[i], a[i + 1], a[i + 2], a[i + 3]);
+          }
+        }
+      } else if (tid < 64) {   // nothing attended in this range
+        l_s[tid] = 0.0f;
+        m_run[tid] = -INFINITY;
+      }
+      smx_bar();
+      if (nsplit == 1) {
+        if (tid < 64) f_s[tid] = l_s[tid] > 0.0f ? 1.0f / l_s[tid] : 0.0f;
+        smx_bar();
+        // stage bf16 [H][512] in the K^ buffers (free now), then one bulk copy out
+        uint16_t* st = reinterpret_cast<uint16_t*>(sp + kOffK);
+        const int chl = 32 * w + lane;                 // channel within a 128-channel tile
+#pragma unroll 1
+        for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll 1
+          for (int h2 = 0; h2 < 2; ++h2) {
+            if (32 * h2 >= H) continue;
+            float o[32];
+            if (nt > 0) {
+              tmem_ld32(tmem + lane_base + kColO + 64u * mt + 32u * h2, o);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = 0.0f;
             }
-          } else {
-            float* po = part_o + (((int64_t)r * nsplit + split) * H) * kD;
+            const int ch = 128 * mt + chl;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              const int h = 32 * hh + i;
-              if (h < H) po[(int64_t)h * kD + ch] = o[i];
+              const int h = 32 * h2 + i;
+              if (h < H) st[h * kD + ch] = f32_to_bf16_rne(o[i] * f_s[h]);
             }
           }
         }
+        fence_async_smem();
+        smx_bar();
+        if (tid == 0) bulk_store(out + (int64_t)r * H * kD, sb + kOffK, (uint32_t)(H * kD * 2));
       }
-      if (nsplit > 1 && tid < H)
-        part_ml[((int64_t)r * nsplit + split) * H + tid] = make_float2(m_run[tid], l_run[tid]);
+    }
+  }
+
+  const bool all_ok = __syncthreads_and(ok) != 0;
+  if (!all_ok) {
+    if (tid == 0) raise_error(c.err, CSA2_DEVERR_TIMEOUT);
+    // bounded: let the MMAs issued so far drain before TMEM is read or released
+    if (misc[1] != 0) mbar_wait(misc[1], misc[2]);
+  }
+
+  if (nsplit > 1) {
+    // ---- merge the cluster's ranges ----
+    // Every rank scales its O^T by 2^(m_j - M) / L (M, L over the cluster),
+    // writes it as f16 [H][512] to its slice of `part` (the CTA's shared
+    // memory is too slow a path between SMs for 100+ KiB), and after a
+    // cluster barrier rank j sums channels [j C, (j + 1) C), C = 512 / nsplit,
+    // over the nsplit slices.  f16 keeps each term to 2^-11 relative, below
+    // the final bf16 rounding.
+    const int nch = kD / nsplit;
+    cluster_wait();
+    // publish this rank's (m, l) per head in every rank's table (l = 0: nothing to add)
+    if (tid < 64) {
+      const float mj = all_ok ? m_run[tid] : -INFINITY, lj = all_ok ? l_s[tid] : 0.0f;
+      const uint32_t slot = sb + kOffMl + 8u * (uint32_t)(split * 64 + tid);
+      for (int j = 0; j < nsplit; ++j) st_cluster_v2(map_shared(slot, (uint32_t)j), mj, lj);
+    }
+    cluster_sync_all();   // every rank's tiles are done and its (m, l) have arrived
+    if (tid < 64) {
+      const float2* ml = reinterpret_cast<const float2*>(sp + kOffMl);
+      float M = -INFINITY;
+      for (int j = 0; j < nsplit; ++j) {
+        const float2 x = ml[j * 64 + tid];
+        if (x.y > 0.0f) M = fmaxf(M, x.x);
+      }
+      float L = 0.0f;
+      for (int j = 0; j < nsplit; ++j) {
+        const float2 x = ml[j * 64 + tid];
+        if (x.y > 0.0f) L += ex2(x.x - M) * x.y;
+      }
+      const float2 self = ml[split * 64 + tid];
+      f_s[tid] = (self.y > 0.0f && L > 0.0f) ? ex2(self.x - M) / L : 0.0f;
+    }
+    __syncthreads();
+    // stage f . O^T as f16 [H][512] in the K^ buffers
+    if (warp < kSoftmaxWarps) {   // TMEM sub-partition == warp: channels 128 mt + 32 warp + lane
+      uint16_t* st = reinterpret_cast<uint16_t*>(sp + kOffK);
+#pragma unroll 1
+      for (int mt = 0; mt < 4; ++mt) {
+        const int ch = 128 * mt + 32 * warp + lane;
+#pragma unroll 1
+        for (int h2 = 0; h2 < 2; ++h2) {
+          if (32 * h2 >= H) continue;
+          float o[32];
+          if (all_ok && nt > 0) {
+            tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + kColO + 64u * mt + 32u * h2, o);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = 0.0f;
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int h = 32 * h2 + i;
+            if (h < H) st[h * kD + ch] = __half_as_ushort(__float2half_rn(o[i] * f_s[h]));
+          }
+        }
+      }
+    }
+    __syncthreads();
+    {
+      const uint4* st4 = reinterpret_cast<const uint4*>(sp + kOffK);
+      uint4* dst = reinterpret_cast<uint4*>(part + ((int64_t)r * nsplit + split) * H * kD);
+      for (int e = tid; e < H * (kD / 8); e += kPipeThreads) dst[e] = st4[e];
+    }
+    cluster_sync_all();   // every rank's slice is in global memory
+    const int c8n = nch / 8;
+    for (int task = tid; task < H * c8n; task += kPipeThreads) {
+      const int h = task / c8n, ch0 = split * nch + 8 * (task % c8n);
+      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int j = 0; j < nsplit; ++j) {
+        const uint4 x = ld_cg16(part + (((int64_t)r * nsplit + j) * H + h) * kD + ch0);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+          acc[2 * k] += f2.x;
+          acc[2 * k + 1] += f2.y;
+        }
+      }
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      *reinterpret_cast<uint4*>(out + ((int64_t)r * H + h) * kD + ch0) = o;
     }
   }
 
   // teardown
-  const bool all_ok = __syncthreads_and(ok) != 0;
-  if (!all_ok) {
-    if (tid == 0) raise_error(c.err, CSA2_DEVERR_TIMEOUT);
-    // bounded: let the MMAs issued so far drain before TMEM is released
-    if (misc[3] != 0) mbar_wait(misc[3], misc[4]);
-  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -610,72 +876,64 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
   }
 }
 
-// Merge the S ranges of each (query, head): out = sum_j e^(m_j-M) O_j / sum_j e^(m_j-M) l_j.
-// CTA = (query, 4 heads); thread = 8 channels of one head.
-__global__ void __launch_bounds__(256) attn_combine_kernel(int H, int nsplit, const float* __restrict__ part_o,
-                                                           const float2* __restrict__ part_ml,
-                                                           uint16_t* __restrict__ out) {
-  const int r = blockIdx.y;
-  const int h = blockIdx.x * 4 + (threadIdx.x >> 6);
-  const int c8 = (threadIdx.x & 63) * 8;
-  if (h >= H) return;
-  float M = -INFINITY;
-  for (int j = 0; j < nsplit; ++j) {
-    const float2 ml = part_ml[((int64_t)r * nsplit + j) * H + h];
-    if (ml.y > 0.0f) M = fmaxf(M, ml.x);
-  }
-  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  float den = 0.0f;
-  if (M != -INFINITY) {
-    for (int j = 0; j < nsplit; ++j) {
-      const float2 ml = part_ml[((int64_t)r * nsplit + j) * H + h];
-      if (!(ml.y > 0.0f)) continue;
-      const float wgt = exp2f((ml.x - M) * 1.4426950408889634f);
-      den = fmaf(wgt, ml.y, den);
-      const float4* src = reinterpret_cast<const float4*>(part_o + (((int64_t)r * nsplit + j) * H + h) * kD + c8);
-      const float4 a = src[0], b = src[1];
-      acc[0] = fmaf(wgt, a.x, acc[0]); acc[1] = fmaf(wgt, a.y, acc[1]);
-      acc[2] = fmaf(wgt, a.z, acc[2]); acc[3] = fmaf(wgt, a.w, acc[3]);
-      acc[4] = fmaf(wgt, b.x, acc[4]); acc[5] = fmaf(wgt, b.y, acc[5]);
-      acc[6] = fmaf(wgt, b.z, acc[6]); acc[7] = fmaf(wgt, b.w, acc[7]);
-    }
-  }
-  const float inv = den > 0.0f ? 1.0f / den : 0.0f;
-  uint4 o;
-  o.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-  o.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-  o.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
-  o.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
-  *reinterpret_cast<uint4*>(out + ((int64_t)r * H + h) * kD + c8) = o;
-}
-
 }  // namespace csa2
 
 // ---- launchers used by api.cu ----
 namespace csa2 {
 
-// Ranges per query: enough CTAs to cover the SMs, at most one per 64-row tile.
-static int attn_splits(int nq) {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int s = nq > 0 ? sms / nq : 1;
-  if (s < 1) s = 1;
-  if (s > kMaxSplits) s = kMaxSplits;
+// Cluster sizes that fit one query per cluster in a single wave, per device.
+static int g_max_clusters[8][4];   // [device][log2 cluster size] (entries 1..3 used)
+
+// Largest range count any launch may use for nq queries: a power of two
+// <= 8 with ranges x nq <= 148 (the SM count the workspace is sized for).
+static int attn_split_bound(int nq) {
+  int s = 8;
+  while (s > 1 && (int64_t)s * nq > 148) s >>= 1;
   return s;
 }
 
+// Ranges per query: the largest cluster size whose clusters all fit at once.
+static int attn_splits(int nq) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 8) return 1;
+  const int bound = attn_split_bound(nq);
+  for (int lg = 3; lg >= 1; --lg)
+    if ((1 << lg) <= bound && nq <= g_max_clusters[dev][lg]) return 1 << lg;
+  return 1;
+}
+
 size_t attn_workspace_bytes(int nq, int H) {
-  const int s = attn_splits(nq);
-  if (s == 1) return 0;
-  const size_t o = (size_t)nq * s * H * kD * sizeof(float);
-  const size_t ml = (size_t)nq * s * H * sizeof(float2);
-  return o + ml + 256;
+  const int s = attn_split_bound(nq);
+  return s > 1 ? (size_t)nq * s * H * kD * sizeof(uint16_t) + 256 : 0;
 }
 
 cudaError_t attention_set_attributes() {
-  return cudaFuncSetAttribute(attn_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)kPipeSmem);
+  cudaError_t e = cudaFuncSetAttribute(attn_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kPipeSmem);
+  if (e != cudaSuccess) return e;
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if (dev < 0 || dev >= 8) return cudaSuccess;
+  for (int lg = 1; lg <= 3; ++lg) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1 << lg, 1);
+    cfg.blockDim = dim3(kPipeThreads);
+    cfg.dynamicSmemBytes = kPipeSmem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 1u << lg;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, attn_pipe_kernel, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    g_max_clusters[dev][lg] = n;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_attention(const CacheView& c, const uint16_t* q, int H, float sm_scale,
@@ -685,14 +943,20 @@ cudaError_t launch_attention(const CacheView& c, const uint16_t* q, int H, float
   if (H % 16 != 0 || H < 16 || H > kHeadsMma) return cudaErrorInvalidValue;
   const int s = attn_splits(nq);
   const int range = (kMaxRows + s - 1) / s;
-  float* part_o = reinterpret_cast<float*>(ws);
-  float2* part_ml = s > 1 ? reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(ws) +
-                                                      (size_t)nq * s * H * kD * sizeof(float))
-                          : nullptr;
-  attn_pipe_kernel<<<dim3(s, nq), kPipeThreads, kPipeSmem, st>>>(c, q, H, sm_scale, q_seq, q_vis, idx, s,
-                                                                 range, out, part_o, part_ml);
-  if (s > 1) attn_combine_kernel<<<dim3((H + 3) / 4, nq), 256, 0, st>>>(H, s, part_o, part_ml, out);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(s, nq);
+  cfg.blockDim = dim3(kPipeThreads);
+  cfg.dynamicSmemBytes = kPipeSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = (unsigned)s;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = s > 1 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, attn_pipe_kernel, c, q, H, sm_scale, q_seq, q_vis, idx, s, range, out,
+                            reinterpret_cast<uint16_t*>(ws));
 }
 
 }  // namespace csa2

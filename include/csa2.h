@@ -175,14 +175,18 @@ int csa2_indexer_score_topk(const csa2_cache* cache, const uint16_t* idx_q, cons
  * Attended set of query r: the positions in set->idx[r] joined with the
  * window [max(0, v-128), v), each position once (128-token sliding window:
  * ai-wave.ru, second paragraph; agentnet.co.il, section "ארכיטקטורה שחותכת
- * בחצי את הפריפיל").  K = V = the decoded FP4 rows (exact in bf16);
- * s = sm_scale * q . k; p = softmax over the set; out[r] = sum p k, rounded
- * to bf16.  q: bf16 [nq][heads][512]; out: bf16 [nq][heads][512]; heads in
+ * בחצי את הפריפיל").  K = V = the decoded FP4 rows (every E2M1 x E4M3
+ * product is exact in f16 and bf16); s = sm_scale * q . k; p = softmax over
+ * the set; out[r] = sum p k, rounded to bf16.  The products run on the tensor
+ * cores in f16 with fp32 accumulation: q is scaled by a power of two per
+ * query so that it is exact in f16 down to 2^-28 of its largest element, and
+ * the weights p are rounded to f16.  q: bf16 [nq][heads][512]; out: bf16 [nq][heads][512]; heads in
  * {16, 32, 48, 64}; nq <= 65535.  Mode checks (host): CSA2_FULL / CSA2_REINDEX need
  * set->layer == layer and set->mode == mode (the set is this layer's own);
  * CSA2_REUSE needs set->layer < layer (the latest Full or Reindex set).  An
  * empty set gives a zero output.  Workspace: csa2_workspace_bytes(
- * CSA2_OP_ATTENTION, nq, heads, 0, 0).
+ * CSA2_OP_ATTENTION, nq, heads, 0, 0) (0 when a query's rows are not split
+ * across CTAs; workspace may then be NULL).
  */
 int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int32_t heads, float sm_scale,
                      const int32_t* q_seq, const int32_t* q_visible, int32_t nq, int32_t mode,
@@ -231,7 +235,7 @@ int csa2_indexer_score_topk_noalloc(const csa2_cache* cache, const uint16_t* idx
 
 /* Workspace bytes for an indexer call (op = CSA2_OP_INDEXER: nq, max_visible,
  * hierarchical) or an attention call (op = CSA2_OP_ATTENTION: nq, heads).
- * Returns 0 for an invalid request. */
+ * Returns 0 for an invalid request or when none is needed. */
 size_t csa2_workspace_bytes(int32_t op, int32_t nq, int32_t heads, int64_t max_visible,
                             int32_t hierarchical);
 

@@ -49,9 +49,10 @@ def test_workspace_sizes(csa2_lib):
     assert ws(1, 4, 0, 1048576, True) == 4 * 131072 * 4 + 256
     # flat encoder chunk: 8192 queries x 65536 entries
     assert ws(1, 8192, 0, 65536, False) == 8192 * 65536 * 4 + 256
-    # attention: per-split fp32 partial O and (m, l); with no device visible the split
-    # count uses 148 SMs, so 32 queries take 4 splits each and 148 queries take 1
-    assert ws(2, 32, 64, 0, False) == 32 * 4 * 64 * (512 * 4 + 8) + 256
+    # attention: 32 queries split 4 ways (4 x 32 <= 148 SMs) exchange f16 partials
+    # [4][64][512]; 148 queries are not split
+    assert ws(2, 32, 64, 0, False) == 32 * 4 * 64 * 512 * 2 + 256
+    assert ws(2, 16, 32, 0, False) == 16 * 8 * 32 * 512 * 2 + 256
     assert ws(2, 148, 64, 0, False) == 0
     assert ws(2, 32, 20, 0, False) == 0          # unsupported head count
     assert ws(7, 1, 64, 0, False) == 0
