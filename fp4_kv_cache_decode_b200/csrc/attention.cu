@@ -285,14 +285,6 @@ __device__ __forceinline__ void st_cluster_v2(uint32_t addr, float a, float b) {
   asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
 }
 
-// Shared -> global bulk copy through the async proxy; returns once the
-// shared-memory source has been read (the writes complete with the grid).
-__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(ssrc), "r"(bytes)
-               : "memory");
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
 
 __device__ __forceinline__ uint4 ld_nc16(const void* p) {
   uint4 v;
@@ -301,13 +293,6 @@ __device__ __forceinline__ uint4 ld_nc16(const void* p) {
                : "l"(p));
   return v;
 }
-// 16-B load through L2 only (data written by other CTAs of this grid).
-__device__ __forceinline__ uint4 ld_cg16(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-  return v;
-}
-
 __device__ __forceinline__ uint32_t ld_nc_u32(const void* p) {
   uint32_t v;
   asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
@@ -740,37 +725,6 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
         l_s[tid] = 0.0f;
         m_run[tid] = -INFINITY;
       }
-      smx_bar();
-      if (nsplit == 1) {
-        if (tid < 64) f_s[tid] = l_s[tid] > 0.0f ? 1.0f / l_s[tid] : 0.0f;
-        smx_bar();
-        // stage bf16 [H][512] in the K^ buffers (free now), then one bulk copy out
-        uint16_t* st = reinterpret_cast<uint16_t*>(sp + kOffK);
-        const int chl = 32 * w + lane;                 // channel within a 128-channel tile
-#pragma unroll 1
-        for (int mt = 0; mt < 4; ++mt) {
-#pragma unroll 1
-          for (int h2 = 0; h2 < 2; ++h2) {
-            if (32 * h2 >= H) continue;
-            float o[32];
-            if (nt > 0) {
-              tmem_ld32(tmem + lane_base + kColO + 64u * mt + 32u * h2, o);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = 0.0f;
-            }
-            const int ch = 128 * mt + chl;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int h = 32 * h2 + i;
-              if (h < H) st[h * kD + ch] = f32_to_bf16_rne(o[i] * f_s[h]);
-            }
-          }
-        }
-        fence_async_smem();
-        smx_bar();
-        if (tid == 0) bulk_store(out + (int64_t)r * H * kD, sb + kOffK, (uint32_t)(H * kD * 2));
-      }
     }
   }
 
@@ -781,15 +735,15 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
     if (misc[1] != 0) mbar_wait(misc[1], misc[2]);
   }
 
+  // ---- output ----
+  // One range per query (nsplit == 1): out = O / l in bf16.  Otherwise every
+  // rank of the query's cluster scales its O^T by 2^(m_j - M) / L (M, L over
+  // the cluster), writes it as f16 [H][512] to its slice of `part` (shared
+  // memory is too slow a path between SMs for 100+ KiB), and after a cluster
+  // barrier rank j sums channels [j C, (j + 1) C), C = 512 / nsplit, over
+  // the nsplit slices.  f16 keeps each term to 2^-11 relative, below the
+  // final bf16 rounding.
   if (nsplit > 1) {
-    // ---- merge the cluster's ranges ----
-    // Every rank scales its O^T by 2^(m_j - M) / L (M, L over the cluster),
-    // writes it as f16 [H][512] to its slice of `part` (the CTA's shared
-    // memory is too slow a path between SMs for 100+ KiB), and after a
-    // cluster barrier rank j sums channels [j C, (j + 1) C), C = 512 / nsplit,
-    // over the nsplit slices.  f16 keeps each term to 2^-11 relative, below
-    // the final bf16 rounding.
-    const int nch = kD / nsplit;
     cluster_wait();
     // publish this rank's (m, l) per head in every rank's table (l = 0: nothing to add)
     if (tid < 64) {
@@ -813,58 +767,79 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
       const float2 self = ml[split * 64 + tid];
       f_s[tid] = (self.y > 0.0f && L > 0.0f) ? ex2(self.x - M) / L : 0.0f;
     }
-    __syncthreads();
-    // stage f . O^T as f16 [H][512] in the K^ buffers
-    if (warp < kSoftmaxWarps) {   // TMEM sub-partition == warp: channels 128 mt + 32 warp + lane
-      uint16_t* st = reinterpret_cast<uint16_t*>(sp + kOffK);
+  } else if (tid < 64) {
+    f_s[tid] = (all_ok && l_s[tid] > 0.0f) ? 1.0f / l_s[tid] : 0.0f;
+  }
+  __syncthreads();
+  // f . O^T straight from TMEM to global [H][512]: the lanes of a warp hold 32
+  // consecutive channels, so each 2-B store instruction writes one 64-B run.
+  // Warps 0..11 share the work, three per TMEM sub-partition (warp % 4).
+  tc_fence_after();   // the last PV's completion was observed before the barriers above
+  if (warp < kMmaWarp) {
+    uint16_t* dst = nsplit == 1 ? out + (int64_t)r * H * kD : part + ((int64_t)r * nsplit + split) * H * kD;
+    const int sub = warp & 3;
 #pragma unroll 1
-      for (int mt = 0; mt < 4; ++mt) {
-        const int ch = 128 * mt + 32 * warp + lane;
-#pragma unroll 1
-        for (int h2 = 0; h2 < 2; ++h2) {
-          if (32 * h2 >= H) continue;
-          float o[32];
-          if (all_ok && nt > 0) {
-            tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + kColO + 64u * mt + 32u * h2, o);
-          } else {
+    for (int pr = warp >> 2; pr < 8; pr += 3) {   // (channel tile mt, head half h2)
+      const int mt = pr >> 1, h2 = pr & 1;
+      if (32 * h2 >= H) continue;
+      const int ch = 128 * mt + 32 * sub + lane;
+      float o[32];
+      if (all_ok && nt > 0) {
+        tmem_ld32(tmem + ((uint32_t)(32 * sub) << 16) + kColO + 64u * mt + 32u * h2, o);
+      } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = 0.0f;
-          }
+        for (int i = 0; i < 32; ++i) o[i] = 0.0f;
+      }
+      float fv[32];   // factors in registers: the stores below may not delay their loads
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int h = 32 * h2 + i;
-            if (h < H) st[h * kD + ch] = __half_as_ushort(__float2half_rn(o[i] * f_s[h]));
-          }
-        }
+      for (int i = 0; i < 32; i += 4)
+        *reinterpret_cast<float4*>(&fv[i]) = *reinterpret_cast<const float4*>(f_s + 32 * h2 + i);
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {   // two heads per packed conversion
+        const uint32_t pk = nsplit == 1 ? pack_bf16x2(o[i] * fv[i], o[i + 1] * fv[i + 1])
+                                        : pack_f16x2(o[i] * fv[i], o[i + 1] * fv[i + 1]);
+        const int h = 32 * h2 + i;
+        if (h < H) dst[h * kD + ch] = (uint16_t)(pk & 0xFFFFu);
+        if (h + 1 < H) dst[(h + 1) * kD + ch] = (uint16_t)(pk >> 16);
       }
     }
-    __syncthreads();
-    {
-      const uint4* st4 = reinterpret_cast<const uint4*>(sp + kOffK);
-      uint4* dst = reinterpret_cast<uint4*>(part + ((int64_t)r * nsplit + split) * H * kD);
-      for (int e = tid; e < H * (kD / 8); e += kPipeThreads) dst[e] = st4[e];
-    }
+  }
+  if (nsplit > 1) {
+    const int nch = kD / nsplit, c8n = nch / 8, ntask = H * c8n;
     cluster_sync_all();   // every rank's slice is in global memory
-    const int c8n = nch / 8;
-    for (int task = tid; task < H * c8n; task += kPipeThreads) {
+    // task = (head, 8 channels); the next task's loads are issued before this one is summed
+    auto load_task = [&](int task, uint4 (&xs)[8]) {
       const int h = task / c8n, ch0 = split * nch + 8 * (task % c8n);
-      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      for (int j = 0; j < nsplit; ++j) {
-        const uint4 x = ld_cg16(part + (((int64_t)r * nsplit + j) * H + h) * kD + ch0);
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
-          acc[2 * k] += f2.x;
-          acc[2 * k + 1] += f2.y;
+      for (int j = 0; j < 8; ++j)   // L2 only: written by this grid
+        if (j < nsplit) xs[j] = __ldcg(reinterpret_cast<const uint4*>(part + (((int64_t)r * nsplit + j) * H + h) * kD + ch0));
+    };
+    uint4 xa[8], xb[8];
+    if (tid < ntask) load_task(tid, xa);
+    for (int task = tid; task < ntask; task += kPipeThreads) {
+      if (task + kPipeThreads < ntask) load_task(task + kPipeThreads, xb);
+      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < nsplit) {
+          const uint32_t w[4] = {xa[j].x, xa[j].y, xa[j].z, xa[j].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+            acc[2 * k] += f2.x;
+            acc[2 * k + 1] += f2.y;
+          }
         }
       }
+      const int h = task / c8n, ch0 = split * nch + 8 * (task % c8n);
       uint4 o;
       o.x = pack_bf16x2(acc[0], acc[1]);
       o.y = pack_bf16x2(acc[2], acc[3]);
       o.z = pack_bf16x2(acc[4], acc[5]);
       o.w = pack_bf16x2(acc[6], acc[7]);
       *reinterpret_cast<uint4*>(out + ((int64_t)r * H + h) * kD + ch0) = o;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) xa[j] = xb[j];
     }
   }
 
