@@ -535,26 +535,26 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj)
       soff[jj] = (uint32_t)((((piece & 1) * 4 + ((jj + (piece >> 1)) & 3)) ^ (rsub & 7)) << 4);
-    // tile t's bytes sit in A, B, C for t % 3 = 0, 1, 2; tile t + 2 is loaded
-    // before tile t is decoded
-    RawTile A, B, C;
+    // tile t's bytes sit in A (t even) or B (t odd); once tile t is decoded its
+    // registers take tile t + 2, about one pipeline step ahead of its decode
+    // (two buffers keep the loop body small: three would triple the code)
+    RawTile A, B;
     if (nt > 0) raw_load(A, c.kv, rows_s, 0, nrow, rsub, piece);
     if (nt > 1) raw_load(B, c.kv, rows_s, 1, nrow, rsub, piece);
     store_q();
-    auto step = [&](int t, RawTile& D, RawTile& L) -> bool {
-      if (t + 2 < nt) raw_load(L, c.kv, rows_s, t + 2, nrow, rsub, piece);
+    auto step = [&](int t, RawTile& D) -> bool {
       const int b = t & 1;
       if (t >= 2 && !mbar_wait(kempty(b), ((t - 2) >> 1) & 1)) return false;
       raw_decode(D, sp, kOffK + b * kKtBytes, rsub, piece, soff);
       fence_async_smem();
       mbar_arrive(kfull(b));
+      if (t + 2 < nt) raw_load(D, c.kv, rows_s, t + 2, nrow, rsub, piece);
       return true;
     };
 #pragma unroll 1
-    for (int t = 0; t < nt; t += 3) {
-      if (!(ok = step(t, A, C)) || t + 1 >= nt) break;
-      if (!(ok = step(t + 1, B, A)) || t + 2 >= nt) break;
-      if (!(ok = step(t + 2, C, B))) break;
+    for (int t = 0; t < nt; t += 2) {
+      if (!(ok = step(t, A)) || t + 1 >= nt) break;
+      if (!(ok = step(t + 1, B))) break;
     }
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issue (one thread) ----------------

@@ -31,7 +31,7 @@ enum UnitSource : int { SRC_FLAT = 0, SRC_BLOCKKEYS = 1, SRC_POOL = 2 };
 
 constexpr int kScoreThreads = 256;
 constexpr int kScoreWarps = kScoreThreads / 32;
-constexpr int kUnitsPerCta = 256;                         // 256 KiB of keys per CTA
+constexpr int kUnitsPerCta = 256;                         // at most 256 KiB of keys per CTA
 constexpr int kStageUnits = 32;                           // 32 KiB per pipeline stage
 constexpr int kStages = 3;
 constexpr int kWarpStageUnits = kStageUnits / kScoreWarps;   // 4 units per warp per stage
@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView
                                                                        const int32_t* __restrict__ q_vis,
                                                                        const int32_t* __restrict__ pool,
                                                                        int64_t max_units, int64_t stride,
-                                                                       float* __restrict__ scores) {
+                                                                       int upc, float* __restrict__ scores) {
   extern __shared__ __align__(16) uint8_t stage[];
   __shared__ const uint8_t* ubase[kUnitsPerCta];
   __shared__ int32_t urows[kUnitsPerCta];
@@ -83,10 +83,10 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView
     if (blockIdx.x == 0 && tid == 0) raise_error(c.err, CSA2_DEVERR_POS);
     nunits = max_units;
   }
-  const int64_t u0 = (int64_t)blockIdx.x * kUnitsPerCta;
+  const int64_t u0 = (int64_t)blockIdx.x * upc;   // upc <= kUnitsPerCta, a multiple of kStageUnits
   if (u0 >= nunits) return;
   const int64_t nb = (v + kBlock - 1) / kBlock;
-  const int nu = (int)(nunits - u0 < kUnitsPerCta ? nunits - u0 : kUnitsPerCta);
+  const int nu = (int)(nunits - u0 < upc ? nunits - u0 : upc);
 
   // 1. unit addresses and candidate rows
   {
@@ -125,22 +125,21 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView
     urows[tid] = nrows;
   }
 
-  // this lane's 16 dims of each head's query (loaded while the lookups run)
+  // this lane's 16 dims of each head's query as 8 (even, odd) pairs (loaded while
+  // the lookups run); the lane's head after the reduce-scatter below is hsel
   const int row = lane >> 2;
   const int dq = (lane & 3) * 16;
-  float q[kIdxHeads][16];
+  float2 q[kIdxHeads][8];
 #pragma unroll
   for (int h = 0; h < kIdxHeads; ++h) {
     const uint4* qp = reinterpret_cast<const uint4*>(idx_q + ((int64_t)r * kIdxHeads + h) * kIdxDim + dq);
     const uint4 a = __ldg(qp), b = __ldg(qp + 1);
-    q[h][0] = bf16_lo(a.x); q[h][1] = bf16_hi(a.x); q[h][2] = bf16_lo(a.y); q[h][3] = bf16_hi(a.y);
-    q[h][4] = bf16_lo(a.z); q[h][5] = bf16_hi(a.z); q[h][6] = bf16_lo(a.w); q[h][7] = bf16_hi(a.w);
-    q[h][8] = bf16_lo(b.x); q[h][9] = bf16_hi(b.x); q[h][10] = bf16_lo(b.y); q[h][11] = bf16_hi(b.y);
-    q[h][12] = bf16_lo(b.z); q[h][13] = bf16_hi(b.z); q[h][14] = bf16_lo(b.w); q[h][15] = bf16_hi(b.w);
-  }
-  float w[kIdxHeads];
+    const uint32_t wq[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-  for (int h = 0; h < kIdxHeads; ++h) w[h] = head_w ? __ldg(head_w + (int64_t)r * kIdxHeads + h) : 1.0f;
+    for (int j = 0; j < 8; ++j) q[h][j] = make_float2(bf16_lo(wq[j]), bf16_hi(wq[j]));
+  }
+  const int hsel = ((lane & 1) << 1) | ((lane >> 1) & 1);
+  const float wsel = head_w ? __ldg(head_w + (int64_t)r * kIdxHeads + hsel) : 1.0f;
   __syncthreads();
 
   const uint32_t stage_s = (uint32_t)__cvta_generic_to_shared(stage);
@@ -178,21 +177,33 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView
         ka = *reinterpret_cast<const uint4*>(sl);
         kb = *reinterpret_cast<const uint4*>(sl + 16);
       }
-      float k[16];
-      k[0] = bf16_lo(ka.x); k[1] = bf16_hi(ka.x); k[2] = bf16_lo(ka.y); k[3] = bf16_hi(ka.y);
-      k[4] = bf16_lo(ka.z); k[5] = bf16_hi(ka.z); k[6] = bf16_lo(ka.w); k[7] = bf16_hi(ka.w);
-      k[8] = bf16_lo(kb.x); k[9] = bf16_hi(kb.x); k[10] = bf16_lo(kb.y); k[11] = bf16_hi(kb.y);
-      k[12] = bf16_lo(kb.z); k[13] = bf16_hi(kb.z); k[14] = bf16_lo(kb.w); k[15] = bf16_hi(kb.w);
-      float sc = 0.0f;
+      const uint32_t wk[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+      float2 k[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) k[j] = make_float2(bf16_lo(wk[j]), bf16_hi(wk[j]));
+      // partial dot products of the lane's 16 dims, even and odd dims in the two halves
+      float p[kIdxHeads];
 #pragma unroll
       for (int h = 0; h < kIdxHeads; ++h) {
-        float p = 0.0f;
+        float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) p = fmaf(q[h][jj], k[jj], p);
-        p += __shfl_xor_sync(0xffffffffu, p, 1);
-        p += __shfl_xor_sync(0xffffffffu, p, 2);
-        sc = fmaf(w[h], fmaxf(p, 0.0f), sc);
+        for (int j = 0; j < 8; ++j) acc = __ffma2_rn(q[h][j], k[j], acc);
+        p[h] = acc.x + acc.y;
       }
+      // the row's 4 lanes reduce-scatter the 4 heads: lane bit 0 keeps heads
+      // {0,1} or {2,3}, lane bit 1 then keeps one of the pair (head hsel)
+      {
+        const bool b0 = (lane & 1) != 0;
+        const float s0 = __shfl_xor_sync(0xffffffffu, b0 ? p[0] : p[2], 1);
+        const float s1 = __shfl_xor_sync(0xffffffffu, b0 ? p[1] : p[3], 1);
+        const float k0 = (b0 ? p[2] : p[0]) + s0, k1 = (b0 ? p[3] : p[1]) + s1;
+        const bool b1 = (lane & 2) != 0;
+        const float t0 = __shfl_xor_sync(0xffffffffu, b1 ? k0 : k1, 2);
+        p[0] = (b1 ? k1 : k0) + t0;
+      }
+      float sc = wsel * fmaxf(p[0], 0.0f);
+      sc += __shfl_xor_sync(0xffffffffu, sc, 1);
+      sc += __shfl_xor_sync(0xffffffffu, sc, 2);
       if (j < nu && (lane & 3) == 0)
         scores[(int64_t)r * stride + u * kBlock + row] = row < urows[j] ? sc : -INFINITY;
     }
@@ -569,14 +580,23 @@ cudaError_t indexer_set_attributes() {
 cudaError_t launch_score(int src, const CacheView& c, const uint16_t* idx_q, const float* head_w,
                          const int32_t* q_seq, const int32_t* q_vis, const int32_t* pool, int nq,
                          int64_t max_units, int64_t stride, float* scores, cudaStream_t st) {
-  dim3 grid((unsigned)((max_units + kUnitsPerCta - 1) / kUnitsPerCta), (unsigned)nq);
+  // units per CTA: enough CTAs for two per SM over the whole batch, in whole
+  // 32-unit stages, at most 256
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t per_query = nq > 0 ? ((int64_t)2 * sms + nq - 1) / nq : 1;   // CTAs per query wanted
+  int64_t upc = (max_units + per_query - 1) / per_query;
+  upc = (upc + kStageUnits - 1) / kStageUnits * kStageUnits;
+  if (upc > kUnitsPerCta) upc = kUnitsPerCta;
+  if (upc < kStageUnits) upc = kStageUnits;
+  dim3 grid((unsigned)((max_units + upc - 1) / upc), (unsigned)nq);
   if (grid.x == 0) return cudaSuccess;
   if (src == SRC_FLAT)
-    score_units_kernel<SRC_FLAT><<<grid, kScoreThreads, kScoreSmem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, scores);
+    score_units_kernel<SRC_FLAT><<<grid, kScoreThreads, kScoreSmem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores);
   else if (src == SRC_BLOCKKEYS)
-    score_units_kernel<SRC_BLOCKKEYS><<<grid, kScoreThreads, kScoreSmem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, scores);
+    score_units_kernel<SRC_BLOCKKEYS><<<grid, kScoreThreads, kScoreSmem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores);
   else
-    score_units_kernel<SRC_POOL><<<grid, kScoreThreads, kScoreSmem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, scores);
+    score_units_kernel<SRC_POOL><<<grid, kScoreThreads, kScoreSmem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores);
   return cudaGetLastError();
 }
 
