@@ -218,6 +218,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkSmemKeys = 16384;   // keys cached in shared memory up to this count
 constexpr int kCandCap = 4096;         // boundary-bucket candidates kept for refinement
+constexpr int kRankCand = 1024;        // up to this many are ranked by pairwise counting
 
 // Exclusive scan of one value per thread across the CTA (1024 threads).
 // Returns the exclusive prefix; *total receives the CTA-wide sum.
@@ -304,21 +305,27 @@ constexpr int kKeysPerThread = kTopkSmemKeys / kTopkThreads;   // 16
 
 // Top-k of up to 16,384 entries with every key held in registers: thread t
 // owns positions [16t, 16t+16).
-//  1. histogram of the keys' top 11 bits (2,048 bins, shared-memory atomics);
-//     the bucket holding the k-th key is found by a CTA scan over the bins;
-//  2. that bucket's keys are compacted into a candidate list (offsets from a
-//     CTA scan of per-thread match counts) and refined on bits 20..10 and
-//     9..0, giving the exact k-th largest key T and the number of keys equal
-//     to T to keep (the lowest-position ones);
+//  1. a CTA reduction gives the number of valid keys and their largest and
+//     smallest key; all valid keys share the bits above the highest bit where
+//     those two differ, so the radix passes start below that common prefix
+//     (scores of similar size then spread over the bins instead of piling
+//     into a few);
+//  2. pass 1 histograms the next up-to-12 bits of every key (shared-memory
+//     atomics) and a CTA scan over the bins finds the bucket holding the k-th
+//     key; the bucket's keys are gathered into a candidate list (atomic
+//     append) and each candidate counts the candidates above and equal to it
+//     (or, for a bucket of more than 1,024, further CTA histogram passes
+//     refine it), giving the exact k-th largest key T and the number of keys
+//     equal to T to keep (the lowest-position ones);
 //  3. one CTA scan of per-thread (count > T, count == T) gives every thread
 //     its output offset; selected positions are written in position order.
-// If the boundary bucket holds more keys than the candidate list, the
-// refinement runs over all keys (same histograms, prefix-filtered).
+// If the boundary bucket holds more keys than the candidate list, the further
+// passes run over all keys (prefix-filtered).
 template <int SRC>
 __device__ __forceinline__ void topk_registers(const float* __restrict__ srow, int64_t n, int k,
                                                const int32_t* pool_row, int32_t* __restrict__ orow,
                                                TopkSmem* sm) {
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t lo = (int64_t)tid * kKeysPerThread;
   uint32_t key[kKeysPerThread];
 #pragma unroll
@@ -331,62 +338,133 @@ __device__ __forceinline__ void topk_registers(const float* __restrict__ srow, i
       key[j] = key[j + 1] = key[j + 2] = key[j + 3] = 0u;
     }
   }
-  for (int i = tid; i < 2048; i += kTopkThreads) sm->hist[i] = 0;
-  __syncthreads();
-  uint32_t nv = 0;
+  // pool blocks of this thread's positions (16 positions = 2 blocks), fetched early
+  int32_t pb0 = 0, pb1 = 0;
+  if (SRC == SRC_POOL && lo < n) {
+    pb0 = pool_row[lo >> 3];
+    pb1 = pool_row[(lo >> 3) + 1];
+  }
+  // valid count, largest and smallest valid key
+  uint32_t nv = 0, kmax = 0u, kmin = 0xFFFFFFFFu;
 #pragma unroll
   for (int j = 0; j < kKeysPerThread; ++j) {
     if (key[j]) {
       ++nv;
-      atomicAdd(&sm->hist[key[j] >> 21], 1u);
+      kmax = max(kmax, key[j]);
+      kmin = min(kmin, key[j]);
     }
   }
-  uint32_t nvalid;
-  cta_exclusive_scan(nv, sm->warp_sums, &nvalid);
+  nv = __reduce_add_sync(0xffffffffu, nv);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  uint32_t* red = sm->cand;   // scratch: [0,32) counts, [32,64) maxima, [64,96) minima
+  if (lane == 0) {
+    red[warp] = nv;
+    red[32 + warp] = kmax;
+    red[64 + warp] = kmin;
+  }
+  for (int i = tid; i < 4096; i += kTopkThreads) sm->hist[i] = 0;
+  __syncthreads();
+  {
+    const uint32_t a = red[lane], bmax = red[32 + lane], bmin = red[64 + lane];
+    nv = __reduce_add_sync(0xffffffffu, a);
+    kmax = __reduce_max_sync(0xffffffffu, bmax);
+    kmin = __reduce_min_sync(0xffffffffu, bmin);
+  }
+  const uint32_t nvalid = nv;
 
   uint32_t T = 1u, need_eq = 0xFFFFFFFFu;
   if (nvalid > (uint32_t)k) {
     uint32_t k_rem = (uint32_t)k;
-    find_bucket(sm, 2048, k_rem);
-    const uint32_t b1 = sm->bucket;
-    k_rem -= sm->above;
-    // compact the boundary bucket
-    uint32_t nm = 0;
-#pragma unroll
-    for (int j = 0; j < kKeysPerThread; ++j) nm += (key[j] && (key[j] >> 21) == b1) ? 1u : 0u;
-    uint32_t ncand;
-    uint32_t off = cta_exclusive_scan(nm, sm->warp_sums, &ncand);
-    const bool use_cand = ncand <= (uint32_t)kCandCap;
-    if (use_cand && nm) {
+    // bits [0, top) are still open; the bits above are the valid keys' common prefix
+    int top = 32 - __clz((int)(kmax ^ kmin));
+    uint32_t prefix = kmax & ~((top >= 32) ? 0xFFFFFFFFu : ((1u << top) - 1u));
+    if (top == 0) {   // every valid key is equal
+      T = kmax;
+      need_eq = k_rem;
+    } else {
+      int width = top < 12 ? top : 12;
+      int shift = top - width;
+      // pass 1 over every valid key
 #pragma unroll
       for (int j = 0; j < kKeysPerThread; ++j)
-        if (key[j] && (key[j] >> 21) == b1) sm->cand[off++] = key[j];
-    }
-    uint32_t prefix = b1 << 21;
-#pragma unroll 1
-    for (int pass = 0; pass < 2; ++pass) {
-      const int shift = pass == 0 ? 10 : 0;
-      const uint32_t pmask = pass == 0 ? 0xFFE00000u : 0xFFFFFC00u;
-      const uint32_t dmask = pass == 0 ? 0x7FFu : 0x3FFu;
-      for (int i = tid; i < 2048; i += kTopkThreads) sm->hist[i] = 0;
+        if (key[j]) atomicAdd(&sm->hist[(key[j] >> shift) & ((1u << width) - 1u)], 1u);
       __syncthreads();
-      if (use_cand) {
-        for (uint32_t i = tid; i < ncand; i += kTopkThreads) {
-          const uint32_t kk = sm->cand[i];
-          if ((kk & pmask) == prefix) atomicAdd(&sm->hist[(kk >> shift) & dmask], 1u);
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < kKeysPerThread; ++j)
-          if (key[j] && (key[j] & pmask) == prefix) atomicAdd(&sm->hist[(key[j] >> shift) & dmask], 1u);
-      }
-      __syncthreads();
-      find_bucket(sm, pass == 0 ? 2048 : 1024, k_rem);
+      find_bucket(sm, 1 << width, k_rem);
       prefix |= sm->bucket << shift;
       k_rem -= sm->above;
+      if (shift > 0) {
+        // gather the boundary bucket (order does not matter for the selection)
+        const uint32_t pmask = ~((1u << shift) - 1u);
+        uint32_t nm = 0;
+#pragma unroll
+        for (int j = 0; j < kKeysPerThread; ++j) nm += (key[j] && (key[j] & pmask) == prefix) ? 1u : 0u;
+        if (tid == 0) sm->ncand = 0;
+        __syncthreads();
+        uint32_t off = nm ? atomicAdd(&sm->ncand, nm) : 0u;
+        if (nm) {
+#pragma unroll
+          for (int j = 0; j < kKeysPerThread; ++j)
+            if (key[j] && (key[j] & pmask) == prefix && off < (uint32_t)kCandCap) sm->cand[off++] = key[j];
+        }
+        __syncthreads();
+        const uint32_t ncand = sm->ncand;
+        if (ncand <= (uint32_t)kRankCand) {
+          // every candidate counts the candidates above and equal to it; the one
+          // whose rank brackets k_rem is the k-th largest key T
+          if (tid < (int)ncand) {
+            const uint32_t c = sm->cand[tid];
+            uint32_t gt = 0, eq = 0;
+            const uint4* c4 = reinterpret_cast<const uint4*>(sm->cand);
+            const uint32_t n4 = ncand >> 2;
+            for (uint32_t i = 0; i < n4; ++i) {
+              const uint4 x = c4[i];
+              gt += (x.x > c) + (x.y > c) + (x.z > c) + (x.w > c);
+              eq += (x.x == c) + (x.y == c) + (x.z == c) + (x.w == c);
+            }
+            for (uint32_t i = n4 << 2; i < ncand; ++i) {
+              const uint32_t x = sm->cand[i];
+              gt += x > c;
+              eq += x == c;
+            }
+            if (gt < k_rem && gt + eq >= k_rem) {   // equal candidates write the same values
+              sm->bucket = c;
+              sm->above = k_rem - gt;
+            }
+          }
+          __syncthreads();
+          prefix = sm->bucket;
+          k_rem = sm->above;
+        } else {
+          const bool use_cand = ncand <= (uint32_t)kCandCap;
+#pragma unroll 1
+          while (shift > 0) {
+            const uint32_t pm = ~((1u << shift) - 1u);
+            width = shift < 12 ? shift : 12;
+            shift -= width;
+            const uint32_t dmask = (1u << width) - 1u;
+            for (int i = tid; i < (1 << width); i += kTopkThreads) sm->hist[i] = 0;
+            __syncthreads();
+            if (use_cand) {
+              for (uint32_t i = tid; i < ncand; i += kTopkThreads) {
+                const uint32_t kk = sm->cand[i];
+                if ((kk & pm) == prefix) atomicAdd(&sm->hist[(kk >> shift) & dmask], 1u);
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < kKeysPerThread; ++j)
+                if (key[j] && (key[j] & pm) == prefix) atomicAdd(&sm->hist[(key[j] >> shift) & dmask], 1u);
+            }
+            __syncthreads();
+            find_bucket(sm, 1 << width, k_rem);
+            prefix |= sm->bucket << shift;
+            k_rem -= sm->above;
+          }
+        }
+      }
+      T = prefix;
+      need_eq = k_rem;
     }
-    T = prefix;
-    need_eq = k_rem;
   }
   // output: one scan of packed (count > T, count == T); both fit 16 bits
   uint32_t ngt = 0, neq = 0;
@@ -406,7 +484,12 @@ __device__ __forceinline__ void topk_registers(const float* __restrict__ srow, i
     const uint32_t kj = key[j];
     bool sel = kj != 0u && kj > T;
     if (kj != 0u && kj == T) sel = eq_rank++ < need_eq;
-    if (sel && slot < (uint32_t)k) orow[slot++] = map_out<SRC>(lo + j, pool_row);
+    if (sel && slot < (uint32_t)k) {
+      int32_t o;
+      if (SRC == SRC_POOL) o = (j < 8 ? pb0 : pb1) * kBlock + (int32_t)((lo + j) & 7);
+      else o = (int32_t)(lo + j);
+      orow[slot++] = o;
+    }
   }
   const uint32_t total = tot_gt + min(tot_eq, need_eq);
   for (int64_t s = (int64_t)total + tid; s < k; s += kTopkThreads) orow[s] = -1;
@@ -584,7 +667,8 @@ cudaError_t launch_score(int src, const CacheView& c, const uint16_t* idx_q, con
   // 32-unit stages, at most 256
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t per_query = nq > 0 ? ((int64_t)2 * sms + nq - 1) / nq : 1;   // CTAs per query wanted
+  int64_t per_query = nq > 0 ? ((int64_t)2 * sms) / nq : 1;   // CTAs per query that fit in one wave
+  if (per_query < 1) per_query = 1;
   int64_t upc = (max_units + per_query - 1) / per_query;
   upc = (upc + kStageUnits - 1) / kStageUnits * kStageUnits;
   if (upc > kUnitsPerCta) upc = kUnitsPerCta;
