@@ -60,13 +60,21 @@ class IndexSetStruct(ctypes.Structure):
         ("pool_layer", ctypes.c_int32),
         ("cache_id", ctypes.c_uint64),
         ("nq", ctypes.c_int32),
+        ("attn_rows", ctypes.c_void_p),
+        ("rows_layer", ctypes.c_int32),
+        ("rows_split", ctypes.c_int32),
+        ("rows_nq", ctypes.c_int32),
     ]
+
+
+ATTN_ROWS_INTS = 648
 
 
 # every entry point declared in include/csa2.h, with its ctypes signature
 _VP, _I32, _I64, _F32, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "csa2_indexset_init": (None, [_VP, _VP, _VP, _I32]),
+    "csa2_indexset_attach_rows": (None, [_VP, _VP]),
     "csa2_kv_quant_append": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _I32, _I32, _VP]),
     "csa2_indexer_score_topk": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _I32, _I64, _I32, _I32, _I32,
                                                _VP, _VP, _SZ, _VP]),
@@ -169,15 +177,24 @@ class Cache:
 
 
 class IndexSet:
-    """Device index rows [rows, 512] + pool rows [rows, 2048] and their mode tags."""
+    """Device index rows [rows, 512] + pool rows [rows, 2048], the attention row
+    cache [rows, ATTN_ROWS_INTS] (row_cache=False leaves it out) and the mode tags."""
 
-    def __init__(self, rows: int, device="cuda"):
+    def __init__(self, rows: int, device="cuda", row_cache: bool = True):
         dev = torch.device(device)
         self.idx = torch.full((rows, TOP_K), -1, dtype=torch.int32, device=dev)
         self.pool_blocks = torch.full((rows, POOL_BLOCKS), -1, dtype=torch.int32, device=dev)
         self.struct = IndexSetStruct()
         lib().csa2_indexset_init(ctypes.byref(self.struct), self.idx.data_ptr(),
                                  self.pool_blocks.data_ptr(), rows)
+        self.attn_rows = None
+        if row_cache:
+            self.attn_rows = torch.zeros((rows, ATTN_ROWS_INTS), dtype=torch.int32, device=dev)
+            lib().csa2_indexset_attach_rows(ctypes.byref(self.struct), self.attn_rows.data_ptr())
+
+    def detach_rows(self):
+        lib().csa2_indexset_attach_rows(ctypes.byref(self.struct), None)
+        self.attn_rows = None
 
     def ref(self):
         return ctypes.byref(self.struct)

@@ -19,8 +19,10 @@ cudaError_t launch_topk(int, const CacheView&, const float*, int64_t, const int3
 cudaError_t indexer_set_attributes();
 cudaError_t attention_set_attributes();
 size_t attn_workspace_bytes(int nq, int H);
+int attn_splits_for(int nq);
 cudaError_t launch_attention(const CacheView&, const uint16_t*, int, float, const int32_t*,
-                             const int32_t*, const int32_t*, int, uint16_t*, void*, cudaStream_t);
+                             const int32_t*, const int32_t*, int, uint16_t*, void*, int32_t*, int, int,
+                             cudaStream_t);
 }  // namespace csa2
 
 using namespace csa2;
@@ -98,6 +100,16 @@ void csa2_indexset_init(csa2_indexset* set, int32_t* idx, int32_t* pool_blocks, 
   set->pool_layer = -1;
   set->cache_id = 0;
   set->nq = 0;
+  set->attn_rows = nullptr;
+  set->rows_layer = -1;
+  set->rows_split = 0;
+  set->rows_nq = 0;
+}
+
+void csa2_indexset_attach_rows(csa2_indexset* set, int32_t* attn_rows) {
+  if (!set) return;
+  set->attn_rows = attn_rows;
+  set->rows_layer = -1;
 }
 
 int csa2_kv_quant_append(const csa2_cache* cache, const uint16_t* kv, const uint16_t* idxk,
@@ -177,6 +189,7 @@ int csa2_indexer_score_topk(const csa2_cache* cache, const uint16_t* idx_q, cons
   set->layer = layer;
   set->mode = mode;
   set->cache_id = cache->cache_id;
+  set->rows_layer = -1;   // the attention row cache belongs to the previous set
   if (mode == CSA2_FULL) {
     set->nq = nq;
     set->pool_layer = hier ? layer : -1;
@@ -186,7 +199,7 @@ int csa2_indexer_score_topk(const csa2_cache* cache, const uint16_t* idx_q, cons
 
 int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int32_t heads, float sm_scale,
                      const int32_t* q_seq, const int32_t* q_visible, int32_t nq, int32_t mode,
-                     int32_t layer, const csa2_indexset* set, uint16_t* out, void* workspace,
+                     int32_t layer, csa2_indexset* set, uint16_t* out, void* workspace,
                      size_t workspace_bytes, csa2_stream_t stream) {
   CacheView v;
   int st = make_view(cache, &v);
@@ -209,10 +222,29 @@ int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int32_t heads, 
   const size_t need = csa2_workspace_bytes(CSA2_OP_ATTENTION, nq, heads, 0, 0);
   if (nq > 0 && need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16)))
     return CSA2_ERR_WORKSPACE;
+  if (!aligned(set->attn_rows, 4)) return CSA2_ERR_ALIGNMENT;
   if (nq == 0) return CSA2_OK;
   if ((st = ensure_device_setup())) return st;
-  return from_cuda(launch_attention(v, q, heads, sm_scale, q_seq, q_visible, set->idx, nq, out,
-                                    workspace, (cudaStream_t)stream));
+  // row cache: Full / Reindex record the resolved rows, Reuse reads them when they
+  // come from the set's current indexer layer with the same queries and ranges
+  const int split = attn_splits_for(nq);
+  int rmode = 0;
+  if (set->attn_rows) {
+    if (mode != CSA2_REUSE) rmode = 1;
+    else if (set->rows_layer == set->layer && set->rows_nq == nq && set->rows_split == split) rmode = 2;
+  }
+  const int e = from_cuda(launch_attention(v, q, heads, sm_scale, q_seq, q_visible, set->idx, nq, out,
+                                           workspace, set->attn_rows, rmode, split, (cudaStream_t)stream));
+  if (rmode == 1) {
+    if (e == CSA2_OK) {
+      set->rows_layer = layer;
+      set->rows_nq = nq;
+      set->rows_split = split;
+    } else {
+      set->rows_layer = -1;
+    }
+  }
+  return e;
 }
 
 int csa2_swa_replay(const csa2_cache* cache, const uint16_t* kv_last, const uint16_t* idxk_last,

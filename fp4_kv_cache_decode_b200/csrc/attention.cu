@@ -70,6 +70,8 @@ constexpr uint32_t kTmemCols = 512;                    // S^T 2x64 + O^T 4x64 + 
 constexpr uint32_t kColO = 128;                        // first O^T column
 constexpr uint32_t kColL = 384;                        // l row (TMEM lane 0)
 constexpr uint32_t kNoRow = 0xFFFFFFFFu;
+constexpr int kRowCacheInts = CSA2_ATTN_ROWS_INTS;      // 640 row ids + 8 range counts per query
+static_assert(kRowCacheInts >= kMaxRows + 8, "row cache layout");
 constexpr float kSlack2 = 12.0f;                       // base-2 headroom before the max moves
 static_assert(kPipeSmem <= 232448, "shared memory budget");
 
@@ -360,7 +362,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
 attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_scale,
                  const int32_t* __restrict__ q_seq, const int32_t* __restrict__ q_vis,
                  const int32_t* __restrict__ idx, int nsplit, int range_slots, uint16_t* __restrict__ out,
-                 uint16_t* __restrict__ part) {
+                 uint16_t* __restrict__ part, int32_t* __restrict__ rcache, int rmode) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw_s = (uint32_t)__cvta_generic_to_shared(smem_raw);
   const uint32_t sb = (raw_s + 1023u) & ~1023u;            // 1024-B aligned base (swizzle atoms)
@@ -411,30 +413,43 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
   const int lo = split * range_slots;
   const int hi = min(lo + range_slots, kMaxRows);
   const int s0 = lo + 2 * tid;
-  int32_t e0 = -1, e1 = -1;
-  if (s0 < hi && s0 < kTopK) e0 = idx_row[s0];
-  if (s0 + 1 < hi && s0 + 1 < kTopK) e1 = idx_row[s0 + 1];
-  const int seq = q_seq[r];
-  const int64_t v = q_vis ? (int64_t)q_vis[r] : (int64_t)seq_len_of(c, seq);
-  const int64_t w0 = v > kWindow ? v - kWindow : 0;
-  auto slot_pos = [&](int sl, int32_t e) -> int64_t {   // attended position of a slot, -1 if unused
-    if (sl >= hi) return -1;
-    if (sl < kTopK) {
-      if (e >= v) raise_error(c.err, CSA2_DEVERR_POS);
-      return (e >= 0 && e < w0) ? (int64_t)e : -1;
-    }
-    const int64_t p = w0 + (sl - kTopK);
-    return p < v ? p : -1;
-  };
-  const int64_t p0 = slot_pos(s0, e0), p1 = slot_pos(s0 + 1, e1);
+  // row cache of this query: ids of range j at [j * range_slots ...), counts at [640 + j]
+  int32_t* const rc_row = rcache ? rcache + (int64_t)r * kRowCacheInts : nullptr;
+  bool u0 = false, u1 = false;   // slot used
   uint32_t id0 = kNoRow, id1 = kNoRow;
-  if (p0 >= 0) {
-    const int64_t pg = page_of(c, seq, p0);
-    if (pg >= 0) id0 = (uint32_t)(pg * kPageTokens + (p0 & (kPageTokens - 1)));
-  }
-  if (p1 >= 0) {
-    const int64_t pg = page_of(c, seq, p1);
-    if (pg >= 0) id1 = (uint32_t)(pg * kPageTokens + (p1 & (kPageTokens - 1)));
+  if (rmode == 2) {   // the rows a Full / Reindex call resolved for this set and range
+    const int nrow_c = rc_row[kMaxRows + split];
+    u0 = s0 < hi && s0 - lo < nrow_c;
+    u1 = s0 + 1 < hi && s0 + 1 - lo < nrow_c;
+    if (u0) id0 = (uint32_t)rc_row[s0];
+    if (u1) id1 = (uint32_t)rc_row[s0 + 1];
+  } else {
+    int32_t e0 = -1, e1 = -1;
+    if (s0 < hi && s0 < kTopK) e0 = idx_row[s0];
+    if (s0 + 1 < hi && s0 + 1 < kTopK) e1 = idx_row[s0 + 1];
+    const int seq = q_seq[r];
+    const int64_t v = q_vis ? (int64_t)q_vis[r] : (int64_t)seq_len_of(c, seq);
+    const int64_t w0 = v > kWindow ? v - kWindow : 0;
+    auto slot_pos = [&](int sl, int32_t e) -> int64_t {   // attended position of a slot, -1 if unused
+      if (sl >= hi) return -1;
+      if (sl < kTopK) {
+        if (e >= v) raise_error(c.err, CSA2_DEVERR_POS);
+        return (e >= 0 && e < w0) ? (int64_t)e : -1;
+      }
+      const int64_t p = w0 + (sl - kTopK);
+      return p < v ? p : -1;
+    };
+    const int64_t p0 = slot_pos(s0, e0), p1 = slot_pos(s0 + 1, e1);
+    u0 = p0 >= 0;
+    u1 = p1 >= 0;
+    if (u0) {
+      const int64_t pg = page_of(c, seq, p0);
+      if (pg >= 0) id0 = (uint32_t)(pg * kPageTokens + (p0 & (kPageTokens - 1)));
+    }
+    if (u1) {
+      const int64_t pg = page_of(c, seq, p1);
+      if (pg >= 0) id1 = (uint32_t)(pg * kPageTokens + (p1 & (kPageTokens - 1)));
+    }
   }
   // largest |q| of the warp (the loads above were in flight meanwhile)
   uint32_t qmax = 0;   // as bf16 bits: magnitudes order like their bit patterns
@@ -451,7 +466,7 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
     for (int o = 16; o > 0; o >>= 1) qmax = max(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
   }
   // compact the used slots (in slot order) into rows_s
-  const uint32_t cnt = (p0 >= 0 ? 1u : 0u) + (p1 >= 0 ? 1u : 0u);
+  const uint32_t cnt = (u0 ? 1u : 0u) + (u1 ? 1u : 0u);
   uint32_t incl = cnt;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -490,8 +505,13 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
   }
   {
     const uint32_t at = before + incl - cnt;
-    if (p0 >= 0) rows_s[at] = id0;
-    if (p1 >= 0) rows_s[at + (p0 >= 0 ? 1u : 0u)] = id1;
+    if (u0) rows_s[at] = id0;
+    if (u1) rows_s[at + (u0 ? 1u : 0u)] = id1;
+    if (rmode == 1) {   // record them for the Reuse layers
+      if (u0) rc_row[lo + at] = (int32_t)id0;
+      if (u1) rc_row[lo + at + (u0 ? 1u : 0u)] = (int32_t)id1;
+      if (tid == 0) rc_row[kMaxRows + split] = (int32_t)total;
+    }
     // start the rows on their way into L2 while the pipeline sets up
     if (id0 != kNoRow) l2_prefetch_bulk(c.kv + (int64_t)id0 * kRowBytes, kRowBytes);
     if (id1 != kNoRow) l2_prefetch_bulk(c.kv + (int64_t)id1 * kRowBytes, kRowBytes);
@@ -911,12 +931,15 @@ cudaError_t attention_set_attributes() {
   return cudaSuccess;
 }
 
+int attn_splits_for(int nq) { return attn_splits(nq); }
+
 cudaError_t launch_attention(const CacheView& c, const uint16_t* q, int H, float sm_scale,
                              const int32_t* q_seq, const int32_t* q_vis, const int32_t* idx, int nq,
-                             uint16_t* out, void* ws, cudaStream_t st) {
+                             uint16_t* out, void* ws, int32_t* rcache, int rmode, int s, cudaStream_t st) {
   if (nq == 0) return cudaSuccess;
   if (H % 16 != 0 || H < 16 || H > kHeadsMma) return cudaErrorInvalidValue;
-  const int s = attn_splits(nq);
+  if (s != 1 && s != 2 && s != 4 && s != 8) return cudaErrorInvalidValue;
+  if (!rcache) rmode = 0;
   const int range = (kMaxRows + s - 1) / s;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(s, nq);
@@ -931,7 +954,7 @@ cudaError_t launch_attention(const CacheView& c, const uint16_t* q, int H, float
   cfg.attrs = at;
   cfg.numAttrs = s > 1 ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, attn_pipe_kernel, c, q, H, sm_scale, q_seq, q_vis, idx, s, range, out,
-                            reinterpret_cast<uint16_t*>(ws));
+                            reinterpret_cast<uint16_t*>(ws), rcache, rmode);
 }
 
 }  // namespace csa2

@@ -113,10 +113,32 @@ typedef struct {
   int32_t pool_layer;    /* layer whose hierarchical Full call wrote pool_blocks    */
   uint64_t cache_id;     /* cache the sets were computed on                         */
   int32_t nq;            /* queries written by the last indexer call                */
+  int32_t* attn_rows;    /* optional int32 [rows][CSA2_ATTN_ROWS_INTS] (NULL: none):
+                            attended rows resolved by the last Full / Reindex
+                            attention call, reused by Reuse calls                   */
+  int32_t rows_layer;    /* layer of the attention call that wrote attn_rows (-1)   */
+  int32_t rows_split;    /* row ranges per query of that call                       */
+  int32_t rows_nq;       /* queries of that call                                    */
 } csa2_indexset;
+
+/* int32 per query of an index set's attention row cache: 640 physical row ids
+ * (page * 64 + slot, in the order attention visits them) and 8 range counts. */
+#define CSA2_ATTN_ROWS_INTS 648
 
 /* Reset an index set's tags (no device work). */
 void csa2_indexset_init(csa2_indexset* set, int32_t* idx, int32_t* pool_blocks, int32_t rows);
+
+/* Attach (or, with NULL, detach) a caller-owned device buffer of
+ * rows * CSA2_ATTN_ROWS_INTS int32 (4-B aligned) in which attention keeps the
+ * physical rows it resolved.  A Full or Reindex csa2_sparse_attn call writes
+ * them; a following Reuse call on the same set with the same queries (nq,
+ * q_seq, q_visible) and the cache unchanged reads them instead of resolving
+ * the selected positions and the window through the page table again.  Any
+ * indexer call on the set discards them.  This is a schedule of the same
+ * computation (the attended positions of a Reuse layer are those of the
+ * latest Full / Reindex layer: agentnet.co.il, "CSA2: דחיסה לאורך ציר
+ * השכבות"); it changes no result. */
+void csa2_indexset_attach_rows(csa2_indexset* set, int32_t* attn_rows);
 
 /*
  * csa2_kv_quant_append -- write new entries into the FP4 cache.
@@ -186,11 +208,13 @@ int csa2_indexer_score_topk(const csa2_cache* cache, const uint16_t* idx_q, cons
  * CSA2_REUSE needs set->layer < layer (the latest Full or Reindex set).  An
  * empty set gives a zero output.  Workspace: csa2_workspace_bytes(
  * CSA2_OP_ATTENTION, nq, heads, 0, 0) (0 when a query's rows are not split
- * across CTAs; workspace may then be NULL).
+ * across CTAs; workspace may then be NULL).  With a row cache attached
+ * (csa2_indexset_attach_rows), Full / Reindex calls record the resolved rows
+ * in it (host tags rows_*) and Reuse calls read them.
  */
 int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int32_t heads, float sm_scale,
                      const int32_t* q_seq, const int32_t* q_visible, int32_t nq, int32_t mode,
-                     int32_t layer, const csa2_indexset* set, uint16_t* out, void* workspace,
+                     int32_t layer, csa2_indexset* set, uint16_t* out, void* workspace,
                      size_t workspace_bytes, csa2_stream_t stream);
 
 /*

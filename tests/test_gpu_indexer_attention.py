@@ -130,3 +130,30 @@ def test_mode_errors_through_binding(ragged):
     with pytest.raises(csa2.Csa2Error) as e:
         csa2.csa2_sparse_attn(cache, q, qs, csa2.REUSE, 1, iset, out, ws)
     assert e.value.status == 4
+
+
+def test_row_cache_changes_no_result(ragged):
+    """Reuse layers read the rows the Full attention call resolved (row cache) or
+    resolve them again (no cache): the outputs are the same bits either way, and an
+    indexer call on the set discards the cached rows."""
+    csa2, syn, w, cache, oseqs = ragged
+    from workload import device as wdev
+    B = len(LENGTHS)
+    sets = {"cached": csa2.IndexSet(B), "plain": csa2.IndexSet(B, row_cache=False)}
+    ws = torch.empty(csa2.csa2_workspace_bytes(csa2.OP_ATTENTION, B, 64), dtype=torch.uint8, device="cuda")
+    outs = {}
+    for name, s in sets.items():
+        qs = _run_indexer(csa2, cache, w, csa2.FULL, 0, s, B, max(LENGTHS))
+        outs[name] = []
+        for layer, mode in ((0, csa2.FULL), (2, csa2.REUSE), (3, csa2.REUSE)):
+            o = torch.empty((B, 64, 512), dtype=torch.bfloat16, device="cuda")
+            csa2.csa2_sparse_attn(cache, wdev.q_batch(w.seed, layer, 0, B, 64), qs, mode, layer, s, o, ws)
+            outs[name].append(o)
+        assert csa2.csa2_check_device_error(cache) == 0
+    for a, b in zip(outs["cached"], outs["plain"]):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    st = sets["cached"].struct
+    assert st.rows_layer == 0 and st.rows_nq == B and st.rows_split in (1, 2, 4, 8)
+    assert sets["plain"].struct.rows_layer == -1
+    _run_indexer(csa2, cache, w, csa2.REINDEX, 4, sets["cached"], B, max(LENGTHS))
+    assert sets["cached"].struct.rows_layer == -1
