@@ -264,10 +264,6 @@ __device__ __forceinline__ void max_scatter32x16(float (&v)[32], int lane) {
   }
 }
 
-// Bulk prefetch of a 16-B aligned range (size a multiple of 16) into L2.
-__device__ __forceinline__ void l2_prefetch_bulk(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
 
 // Thread-block cluster: barrier over all threads of the cluster, address of
 // the same shared-memory offset in CTA `rank`, and accesses through it.
@@ -404,10 +400,12 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
       qv[i] = (e < kQChunks && (e >> 6) < H) ? ld_nc16(qsrc + e) : make_uint4(0, 0, 0, 0);
     }
   }
-  // ones row for the softmax denominator: row 0 of a K-major [64 x 64] f16 tile
+  // ones row for the softmax denominator: row 0 of a K-major [64 x 64] f16 tile,
+  // fenced for the tensor core
   for (int e = tid; e < (int)(kOnesBytes / 16); e += kPipeThreads)
     *reinterpret_cast<uint4*>(sp + kOffOnes + 16 * e) =
         e < 8 ? make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u) : make_uint4(0, 0, 0, 0);
+  fence_async_smem();
 
   // this CTA's candidate slots; thread tid takes slots lo + 2 tid and lo + 2 tid + 1
   const int lo = split * range_slots;
@@ -512,9 +510,6 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
       if (u1) rc_row[lo + at + (u0 ? 1u : 0u)] = (int32_t)id1;
       if (tid == 0) rc_row[kMaxRows + split] = (int32_t)total;
     }
-    // start the rows on their way into L2 while the pipeline sets up
-    if (id0 != kNoRow) l2_prefetch_bulk(c.kv + (int64_t)id0 * kRowBytes, kRowBytes);
-    if (id1 != kNoRow) l2_prefetch_bulk(c.kv + (int64_t)id1 * kRowBytes, kRowBytes);
   }
   // Q in f16 scaled by 2^qexp so that the largest |q| lies in [2^14, 2^15):
   // exact for every element of magnitude >= 2^-28 of the largest; the scores
@@ -543,8 +538,7 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
   const int nrow = (int)total;
   const int nt = (nrow + kRowTile - 1) / kRowTile;
   const uint32_t tmem = misc[0];
-  fence_async_smem();
-  __syncthreads();
+  __syncthreads();   // rows_s complete
   bool ok = true;
 
   if (warp >= kSoftmaxWarps && warp < kMmaWarp) {
