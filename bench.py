@@ -122,6 +122,55 @@ def _attended_rows(idx: np.ndarray, L: int) -> int:
     return int(sel.size + (L - w0))
 
 
+# ---------------------------------------------------------------------------
+# ranks (one process per GPU under torchrun; the host logic is tested with gloo)
+# ---------------------------------------------------------------------------
+
+def rank_env() -> tuple[int, int, int]:
+    """(world, rank, local_rank) from the torchrun environment (1, 0, 0 alone)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_ranks(world: int, backend: str = "nccl", device=None) -> None:
+    """Join the process group (nothing to do alone).  A short timeout makes ranks
+    that wait on a missing peer fail instead of hanging."""
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        kw = {"device_id": device} if device is not None else {}
+        dist.init_process_group(backend, timeout=timedelta(seconds=120), **kw)
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Every rank draws its own batch (weak scaling: no data is shared)."""
+    return seed + 1000 * rank
+
+
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The slowest rank's time: the job is done when its last rank is."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int) -> None:
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def finish_ranks(world: int) -> None:
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -129,19 +178,13 @@ def run_gpu(args):
     import workload as wl
     from fp4_kv_cache_decode_b200 import _build, csa2, synthetic
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     if not os.path.exists(_build.LIB):
         raise SystemExit("libcsa2.so is not built: run `python -c 'import __graft_entry__ as g; g.build()'`")
     torch.cuda.set_device(local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+    init_ranks(world, "nccl", torch.device("cuda", local))
     w = wl.workload(CONFIG_ID)
-    if world > 1:
-        w.seed = w.seed + 1000 * rank          # every rank gets its own batch
+    w.seed = rank_seed(w.seed, rank)
     if args.pool_pages:
         # profiling case only: a pool of exactly the pages the batch uses (same work per
         # call, compact addresses, ~1 GB on the device instead of ~5 GB)
@@ -187,24 +230,21 @@ def run_gpu(args):
         flush.fill_(1)
         graph.replay()
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    barrier(world)
 
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    barrier(world)
     for k in range(args.steps):
         flush.fill_(k & 0xFF)          # outside the events: the step starts with a cold L2
         events[k][0].record(stream)
         graph.replay()
         events[k][1].record(stream)
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    barrier(world)
     clocks = sampler.stop()
     step_ms = np.array([events[k][0].elapsed_time(events[k][1]) for k in range(args.steps)])
     total_ms = float(step_ms.sum())
@@ -239,10 +279,7 @@ def run_gpu(args):
         torch.cuda.synchronize()
         attn_ms.append(a0.elapsed_time(a1) / n_attn)
     attn_launch_ms = float(np.median(attn_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world)
     assert csa2.csa2_check_device_error(cache) == 0
 
     # --- algorithmic work of one step (from the sets the step produced) ---
@@ -301,10 +338,7 @@ def run_gpu(args):
 
     # --- end to end through the C ABI with host buffers ---
     e2e = run_e2e(args, w, step, stream, flush)
-    if world > 1:
-        t = torch.tensor([e2e["ms"]], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e["ms"] = float(t.item())
+    e2e["ms"] = max_over_ranks(e2e["ms"], world)
     e2e_value = len(w.layers) * args.steps * world / (e2e["ms"] * 1e-3)
 
     result = {
@@ -325,9 +359,7 @@ def run_gpu(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args, seqs=tuple(range(w.batch)))
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    finish_ranks(world)
     if rank == 0:
         print(json.dumps(result), flush=True)
 
@@ -448,8 +480,7 @@ def cpu_baseline(args, seqs=(0,)):
 
 
 def run_reference(args):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
+    world, rank, _ = rank_env()
     if rank != 0:
         return
     import workload as wl

@@ -220,7 +220,7 @@ constexpr int kTopkSmemKeys = 16384;   // keys cached in shared memory up to thi
 constexpr int kCandCap = 4096;         // boundary-bucket candidates kept for refinement
 constexpr int kRankCand = 1024;        // up to this many are ranked by pairwise counting
 
-// Exclusive scan of one value per thread across the CTA (1024 threads).
+// Exclusive scan of one value per thread across the CTA (kTopkThreads threads).
 // Returns the exclusive prefix; *total receives the CTA-wide sum.
 __device__ __forceinline__ uint32_t cta_exclusive_scan(uint32_t v, uint32_t* warp_sums, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -233,7 +233,7 @@ __device__ __forceinline__ uint32_t cta_exclusive_scan(uint32_t v, uint32_t* war
   if (lane == 31) warp_sums[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    uint32_t s = warp_sums[lane];
+    uint32_t s = lane < kTopkThreads / 32 ? warp_sums[lane] : 0u;
     uint32_t t = s;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -267,10 +267,10 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool pred
 // `nbins` bins (larger bin = larger key).  Sets sm->bucket and sm->above
 // (elements in higher bins).
 __device__ __forceinline__ void find_bucket(TopkSmem* sm, int nbins, uint32_t k_rem) {
-  const int per = 4;
+  const int per = (nbins + kTopkThreads - 1) / kTopkThreads;   // bins per thread
   const int t = threadIdx.x;
   uint32_t local = 0;
-  const int hi = nbins - per * t;   // this thread's bins: [hi-4, hi), counted from the top
+  const int hi = nbins - per * t;   // this thread's bins: [hi-per, hi), counted from the top
   if (hi > 0) {
 #pragma unroll
     for (int j = 1; j <= per; ++j)
@@ -302,6 +302,7 @@ __device__ __forceinline__ int32_t map_out(int64_t i, const int32_t* pool_row) {
 }
 
 constexpr int kKeysPerThread = kTopkSmemKeys / kTopkThreads;   // 16
+static_assert(kKeysPerThread == 16, "a thread's positions span exactly two 8-token pool blocks");
 
 // Top-k of up to 16,384 entries with every key held in registers: thread t
 // owns positions [16t, 16t+16).
@@ -366,7 +367,9 @@ __device__ __forceinline__ void topk_registers(const float* __restrict__ srow, i
   for (int i = tid; i < 4096; i += kTopkThreads) sm->hist[i] = 0;
   __syncthreads();
   {
-    const uint32_t a = red[lane], bmax = red[32 + lane], bmin = red[64 + lane];
+    const bool in = lane < kTopkThreads / 32;
+    const uint32_t a = in ? red[lane] : 0u, bmax = in ? red[32 + lane] : 0u,
+                   bmin = in ? red[64 + lane] : 0xFFFFFFFFu;
     nv = __reduce_add_sync(0xffffffffu, a);
     kmax = __reduce_max_sync(0xffffffffu, bmax);
     kmin = __reduce_min_sync(0xffffffffu, bmin);
