@@ -354,6 +354,53 @@ __device__ __forceinline__ void raw_decode(const RawTile& R, uint8_t* sp, uint32
   }
 }
 
+// Rank `split` of a query's cluster sums channels [split C, (split + 1) C),
+// C = 512 / S, of the S f16 slices [S][H][512] in `part` and writes them as
+// bf16.  Task = (head, 8 channels); a thread's tasks are tid + 416 t, and all
+// of their loads (at most 16 x 16 B) are in flight before any sum is formed.
+template <int S>
+__device__ __forceinline__ void reduce_slices(const uint16_t* __restrict__ part, uint16_t* __restrict__ out,
+                                              int r, int split, int H, int tid) {
+  constexpr int nch = kD / S, c8n = nch / 8;
+  constexpr int kTasks = (kHeadsMma * c8n + kPipeThreads - 1) / kPipeThreads;   // per thread at H = 64
+  const int ntask = H * c8n;
+  uint4 xs[kTasks][S];
+#pragma unroll
+  for (int t = 0; t < kTasks; ++t) {
+    const int task = tid + t * kPipeThreads;
+    if (task < ntask) {
+      const int h = task / c8n, ch0 = split * nch + 8 * (task % c8n);
+#pragma unroll
+      for (int j = 0; j < S; ++j)   // L2 only: written by this grid
+        xs[t][j] = __ldcg(reinterpret_cast<const uint4*>(part + (((int64_t)r * S + j) * H + h) * kD + ch0));
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < kTasks; ++t) {
+    const int task = tid + t * kPipeThreads;
+    if (task < ntask) {
+      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+      for (int j = 0; j < S; ++j) {
+        const uint32_t w[4] = {xs[t][j].x, xs[t][j].y, xs[t][j].z, xs[t][j].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+          acc[2 * k] += f2.x;
+          acc[2 * k + 1] += f2.y;
+        }
+      }
+      const int h = task / c8n, ch0 = split * nch + 8 * (task % c8n);
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      *reinterpret_cast<uint4*>(out + ((int64_t)r * H + h) * kD + ch0) = o;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kPipeThreads, 1)
 attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_scale,
                  const int32_t* __restrict__ q_seq, const int32_t* __restrict__ q_vis,
@@ -819,42 +866,10 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
     }
   }
   if (nsplit > 1) {
-    const int nch = kD / nsplit, c8n = nch / 8, ntask = H * c8n;
     cluster_sync_all();   // every rank's slice is in global memory
-    // task = (head, 8 channels); the next task's loads are issued before this one is summed
-    auto load_task = [&](int task, uint4 (&xs)[8]) {
-      const int h = task / c8n, ch0 = split * nch + 8 * (task % c8n);
-#pragma unroll
-      for (int j = 0; j < 8; ++j)   // L2 only: written by this grid
-        if (j < nsplit) xs[j] = __ldcg(reinterpret_cast<const uint4*>(part + (((int64_t)r * nsplit + j) * H + h) * kD + ch0));
-    };
-    uint4 xa[8], xb[8];
-    if (tid < ntask) load_task(tid, xa);
-    for (int task = tid; task < ntask; task += kPipeThreads) {
-      if (task + kPipeThreads < ntask) load_task(task + kPipeThreads, xb);
-      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j < nsplit) {
-          const uint32_t w[4] = {xa[j].x, xa[j].y, xa[j].z, xa[j].w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
-            acc[2 * k] += f2.x;
-            acc[2 * k + 1] += f2.y;
-          }
-        }
-      }
-      const int h = task / c8n, ch0 = split * nch + 8 * (task % c8n);
-      uint4 o;
-      o.x = pack_bf16x2(acc[0], acc[1]);
-      o.y = pack_bf16x2(acc[2], acc[3]);
-      o.z = pack_bf16x2(acc[4], acc[5]);
-      o.w = pack_bf16x2(acc[6], acc[7]);
-      *reinterpret_cast<uint4*>(out + ((int64_t)r * H + h) * kD + ch0) = o;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) xa[j] = xb[j];
-    }
+    if (nsplit == 2) reduce_slices<2>(part, out, r, split, H, tid);
+    else if (nsplit == 4) reduce_slices<4>(part, out, r, split, H, tid);
+    else reduce_slices<8>(part, out, r, split, H, tid);
   }
 
   // teardown
