@@ -281,20 +281,7 @@ def run_gpu(args):
     attn_launch_ms = float(np.median(attn_ms))
 
     def graph_ms(fn, reps=5):
-        """Median device time of fn() captured as a CUDA graph (L2 flushed first)."""
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            fn()
-        ts = []
-        for k in range(reps):
-            flush.fill_(k & 0xFF)
-            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a0.record(stream)
-            g.replay()
-            a1.record(stream)
-            torch.cuda.synchronize()
-            ts.append(a0.elapsed_time(a1))
-        return float(np.median(ts))
+        return _graph_ms(fn, flush, stream, reps)
 
     # the indexer calls alone, each as its own graph (Full at layer 0, then the
     # Reindex layer on the Full's pool)
@@ -381,11 +368,96 @@ def run_gpu(args):
         "gpu_launches": args.steps * launches_per_step(w),
         "clocks": clocks,
     }
+    result["window_store"] = measure_window_store(w, cache, step, stream, flush, peaks, reuse_ms)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args, seqs=tuple(range(w.batch)))
     finish_ranks(world)
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+def _graph_ms(fn, flush, stream, reps=5):
+    """Median device time of fn() captured as a CUDA graph (L2 flushed first)."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    ts = []
+    for k in range(reps):
+        flush.fill_(k & 0xFF)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        g.replay()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a0.elapsed_time(a1))
+    return float(np.median(ts))
+
+
+def measure_window_store(w, cache, step, stream, flush, peaks, attn_global_ms):
+    """The separate sliding-window store on the bench batch, outside the timed
+    region: bounded replay (every sequence flagged) into the store at ratio 1 and 2
+    and into the global cache at ratio 1, and the Reuse attention launch reading
+    its window from the store.  The store is filled with the same entries as the
+    global cache, so the step's outputs must not change by a bit."""
+    import torch
+
+    import workload as wl
+    from workload import device as wdev
+    from fp4_kv_cache_decode_b200 import csa2
+    B = w.batch
+    col = torch.from_numpy(wl.kv_col_scale(w.seed)).cuda()
+    kv1 = torch.zeros((B, 128, 512), dtype=torch.bfloat16, device="cuda")
+    k1 = torch.zeros((B, 128, 64), dtype=torch.bfloat16, device="cuda")
+    kv2 = torch.zeros((B, 256, 512), dtype=torch.bfloat16, device="cuda")
+    n_blocks = 0
+    for b, L in enumerate(w.lengths):
+        n = min(128, L)
+        wdev.kv_rows(w.seed, b, L - n, n, out=kv1[b, 128 - n:], col_scale=col)
+        wdev.idxk_rows(w.seed, b, L - n, n, out=k1[b, 128 - n:])
+        wdev.kv_rows(w.seed + 1, b, 0, 2 * n, out=kv2[b, 256 - 2 * n:], col_scale=col)
+        n_blocks += (L - 1) // 8 - (L - n) // 8 + 1
+    n_entries = sum(min(128, L) for L in w.lengths)
+    miss = torch.ones(B, dtype=torch.uint8, device="cuda")
+    ref_out = [o.clone() for o in step.out]
+    hbm = peaks["hbm_gbs"]
+
+    def leg(ms, nbytes, launches):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return {"ms": ms, "algorithmic_bytes": nbytes, "gbs": gbs, "frac_of_hbm": gbs / hbm,
+                "launches": launches}
+
+    # global cache, ratio 1: rows, keys and touched block keys rewritten (same values)
+    t_glob = _graph_ms(lambda: csa2.csa2_swa_replay(cache, kv1, k1, miss), flush, stream)
+    glob_bytes = n_entries * (1024 + 128 + 288 + 128) + n_blocks * (8 * 128 + 128)
+    cache.swa_rows = torch.zeros((B, 128, 288), dtype=torch.uint8, device="cuda")
+    cache.refresh()
+    try:
+        t_st1 = _graph_ms(lambda: csa2.csa2_swa_replay(cache, kv1, None, miss), flush, stream)
+        step.run(append=False)             # sets and row caches resolved with the store attached
+        torch.cuda.synchronize()
+        same = all(torch.equal(a.view(torch.int16), b.view(torch.int16)) for a, b in zip(step.out, ref_out))
+        reuse = [i for i, m in enumerate(w.layers) if m == "R" and i > w.layers.index("RI")]
+
+        def reuse_calls():
+            for _ in range(2):
+                for i in reuse:
+                    step.layer(i)
+        t_attn = _graph_ms(reuse_calls, flush, stream) / (2 * len(reuse))
+        t_st2 = _graph_ms(lambda: csa2.csa2_swa_replay(cache, kv2, None, miss, compress=2), flush, stream)
+        assert csa2.csa2_check_device_error(cache) == 0
+    finally:
+        cache.swa_rows = None
+        cache.refresh()
+    return {
+        "replay_global_ratio1": leg(t_glob, glob_bytes, 2),
+        "replay_store_ratio1": leg(t_st1, n_entries * (1024 + 288), 1),
+        "replay_store_ratio2": leg(t_st2, n_entries * (2048 + 288), 1),
+        "attention_reuse_launch_ms": {"window_from_store": t_attn, "window_from_global_cache": attn_global_ms},
+        "step_outputs_bit_identical": bool(same),
+        "note": "CUDA graphs of one call (replay) or 2 x 3 Reuse calls (attention), L2 flushed first; "
+                "bytes: bf16 rows read + FP4 rows (and keys) written",
+    }
 
 
 def launches_per_step(w) -> int:

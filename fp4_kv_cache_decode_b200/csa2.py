@@ -25,6 +25,7 @@ BK_PAGE_BYTES = 8 * 128
 TOP_K = 512
 POOL_BLOCKS = 2048
 WINDOW = 128
+REPLAY = 128          # entries rewritten by bounded replay; slots of the sliding-window store
 
 DEVERR_PAGE, DEVERR_POS, DEVERR_SEQ = 1, 2, 4
 
@@ -47,6 +48,7 @@ class CacheStruct(ctypes.Structure):
         ("seq_lens", ctypes.c_void_p),
         ("error_word", ctypes.c_void_p),
         ("cache_id", ctypes.c_uint64),
+        ("swa_rows", ctypes.c_void_p),
     ]
 
 
@@ -82,7 +84,7 @@ SIGNATURES = {
                                         _VP, _SZ, _VP]),
     "csa2_indexer_score_topk_noalloc": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _I32, _I64, _I32, _I32,
                                                        _I32, _VP, _VP]),
-    "csa2_swa_replay": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP]),
+    "csa2_swa_replay": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int32, _VP]),
     "csa2_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I64, _I32]),
     "csa2_check_device_error": (ctypes.c_int, [_VP, _VP, ctypes.POINTER(ctypes.c_uint32)]),
     "csa2_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -144,9 +146,11 @@ _I32T = (torch.int32,)
 
 
 class Cache:
-    """Paged FP4 cache: three page pools, page table, lengths, error word."""
+    """Paged FP4 cache: three page pools, page table, lengths, error word, and
+    (swa_store=True) a separate sliding-window store [batch, 128, 288] bytes."""
 
-    def __init__(self, n_pages: int, batch: int, max_pages: int, device="cuda", cache_id: int = 1):
+    def __init__(self, n_pages: int, batch: int, max_pages: int, device="cuda", cache_id: int = 1,
+                 swa_store: bool = False):
         dev = torch.device(device)
         self.n_pages, self.batch, self.max_pages = n_pages, batch, max_pages
         self.kv_pool = torch.zeros(n_pages * PAGE_BYTES, dtype=torch.uint8, device=dev)
@@ -156,6 +160,8 @@ class Cache:
         self.seq_lens = torch.zeros(batch, dtype=torch.int32, device=dev)
         self.error_word = torch.zeros(1, dtype=torch.int32, device=dev)
         self.cache_id = cache_id
+        self.swa_rows = (torch.zeros((batch, REPLAY, ROW_BYTES), dtype=torch.uint8, device=dev)
+                         if swa_store else None)
         self.struct = CacheStruct()
         self.refresh()
 
@@ -171,6 +177,7 @@ class Cache:
         s.seq_lens = self.seq_lens.data_ptr()
         s.error_word = self.error_word.data_ptr()
         s.cache_id = self.cache_id
+        s.swa_rows = None if self.swa_rows is None else self.swa_rows.data_ptr()
 
     def ref(self):
         return ctypes.byref(self.struct)
@@ -272,13 +279,13 @@ def csa2_sparse_attn(cache: Cache, q: torch.Tensor, q_seq: torch.Tensor, mode: i
     _check(st, "csa2_sparse_attn")
 
 
-def csa2_swa_replay(cache: Cache, kv_last: torch.Tensor, idxk_last: torch.Tensor, miss: torch.Tensor,
-                    stream=None):
+def csa2_swa_replay(cache: Cache, kv_last: torch.Tensor, idxk_last: torch.Tensor | None, miss: torch.Tensor,
+                    compress: int = 1, stream=None):
     b = cache.batch
     st = lib().csa2_swa_replay(
-        cache.ref(), _ptr(kv_last, _BF16, "kv_last", b * 128 * LATENT_DIM),
-        _ptr(idxk_last, _BF16, "idxk_last", b * 128 * 64),
-        _ptr(miss, (torch.uint8, torch.bool), "miss", b), _stream(stream))
+        cache.ref(), _ptr(kv_last, _BF16, "kv_last", b * REPLAY * compress * LATENT_DIM),
+        _ptr(idxk_last, _BF16, "idxk_last", b * REPLAY * compress * 64),
+        _ptr(miss, (torch.uint8, torch.bool), "miss", b), compress, _stream(stream))
     _check(st, "csa2_swa_replay")
 
 

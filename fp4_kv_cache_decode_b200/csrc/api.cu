@@ -11,7 +11,7 @@ namespace csa2 {
 cudaError_t launch_append(const CacheView&, const uint16_t*, const uint16_t*, const int32_t*,
                           const int32_t*, int, int, cudaStream_t);
 cudaError_t launch_replay(const CacheView&, const uint16_t*, const uint16_t*, const uint8_t*,
-                          cudaStream_t);
+                          int, cudaStream_t);
 cudaError_t launch_score(int, const CacheView&, const uint16_t*, const float*, const int32_t*,
                          const int32_t*, const int32_t*, int, int64_t, int64_t, float*, cudaStream_t);
 cudaError_t launch_topk(int, const CacheView&, const float*, int64_t, const int32_t*, const int32_t*,
@@ -55,9 +55,12 @@ int make_view(const csa2_cache* c, CacheView* v) {
       !c->error_word)
     return CSA2_ERR_INVALID_ARG;
   if (c->n_pages <= 0 || c->max_pages <= 0 || c->batch <= 0) return CSA2_ERR_SHAPE;
-  if (c->n_pages > ((int64_t)1 << 31)) return CSA2_ERR_SHAPE;
+  // attention names a physical row by a 31-bit id (page x 64 + slot, or a
+  // sliding-window slot batch x 128 + p % 128 under a flag bit)
+  if (c->n_pages > ((int64_t)1 << 25) || c->batch > (1 << 23)) return CSA2_ERR_SHAPE;
   if (!aligned(c->kv_pool, 16) || !aligned(c->idxk_pool, 16) || !aligned(c->blockkey_pool, 16) ||
-      !aligned(c->page_table, 4) || !aligned(c->seq_lens, 4) || !aligned(c->error_word, 4))
+      !aligned(c->page_table, 4) || !aligned(c->seq_lens, 4) || !aligned(c->error_word, 4) ||
+      !aligned(c->swa_rows, 16))
     return CSA2_ERR_ALIGNMENT;
   v->kv = static_cast<uint8_t*>(c->kv_pool);
   v->idxk = static_cast<uint8_t*>(c->idxk_pool);
@@ -68,6 +71,7 @@ int make_view(const csa2_cache* c, CacheView* v) {
   v->batch = c->batch;
   v->seq_lens = c->seq_lens;
   v->err = c->error_word;
+  v->swa = static_cast<uint8_t*>(c->swa_rows);
   return CSA2_OK;
 }
 
@@ -248,13 +252,14 @@ int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int32_t heads, 
 }
 
 int csa2_swa_replay(const csa2_cache* cache, const uint16_t* kv_last, const uint16_t* idxk_last,
-                    const uint8_t* miss, csa2_stream_t stream) {
+                    const uint8_t* miss, int32_t compress, csa2_stream_t stream) {
   CacheView v;
   int st = make_view(cache, &v);
   if (st) return st;
-  if (!kv_last || !idxk_last || !miss) return CSA2_ERR_INVALID_ARG;
+  if (compress != 1 && compress != 2) return CSA2_ERR_SHAPE;
+  if (!kv_last || !miss || (!idxk_last && !v.swa)) return CSA2_ERR_INVALID_ARG;
   if (!aligned(kv_last, 16) || !aligned(idxk_last, 4)) return CSA2_ERR_ALIGNMENT;
-  return from_cuda(launch_replay(v, kv_last, idxk_last, miss, (cudaStream_t)stream));
+  return from_cuda(launch_replay(v, kv_last, idxk_last, miss, compress, (cudaStream_t)stream));
 }
 
 size_t csa2_workspace_bytes(int32_t op, int32_t nq, int32_t heads, int64_t max_visible,

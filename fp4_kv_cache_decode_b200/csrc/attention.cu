@@ -70,6 +70,7 @@ constexpr uint32_t kTmemCols = 512;                    // S^T 2x64 + O^T 4x64 + 
 constexpr uint32_t kColO = 128;                        // first O^T column
 constexpr uint32_t kColL = 384;                        // l row (TMEM lane 0)
 constexpr uint32_t kNoRow = 0xFFFFFFFFu;
+constexpr uint32_t kSwaRow = 0x80000000u;              // flag: id = slot of the sliding-window store
 constexpr int kRowCacheInts = CSA2_ATTN_ROWS_INTS;      // 640 row ids + 8 range counts per query
 static_assert(kRowCacheInts >= kMaxRows + 8, "row cache layout");
 constexpr float kSlack2 = 12.0f;                       // base-2 headroom before the max moves
@@ -307,14 +308,15 @@ struct RawTile {
   uint32_t s[4];    // the 4-B scale word holding its two scale bytes
 };
 
-__device__ __forceinline__ void raw_load(RawTile& R, const uint8_t* __restrict__ kv, const uint32_t* rows_s,
+__device__ __forceinline__ void raw_load(RawTile& R, const uint8_t* __restrict__ kv,
+                                         const uint8_t* __restrict__ swa, const uint32_t* rows_s,
                                          int t, int nrow, int rsub, int piece) {
 #pragma unroll
   for (int it = 0; it < 4; ++it) {
     const int li = t * kRowTile + rsub + 16 * it;
     const uint32_t id = li < nrow ? rows_s[li] : kNoRow;
     if (id != kNoRow) {
-      const uint8_t* rp = kv + (int64_t)id * kRowBytes;
+      const uint8_t* rp = ((id & kSwaRow) ? swa : kv) + (int64_t)(id & ~kSwaRow) * kRowBytes;
       R.c[it] = ld_nc16(rp + piece * 16);
       R.s[it] = ld_nc_u32(rp + kCodeBytes + (piece >> 1) * 4);
     } else {   // zero codes and zero scales decode to zeros
@@ -487,14 +489,16 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
     const int64_t p0 = slot_pos(s0, e0), p1 = slot_pos(s0 + 1, e1);
     u0 = p0 >= 0;
     u1 = p1 >= 0;
-    if (u0) {
-      const int64_t pg = page_of(c, seq, p0);
-      if (pg >= 0) id0 = (uint32_t)(pg * kPageTokens + (p0 & (kPageTokens - 1)));
-    }
-    if (u1) {
-      const int64_t pg = page_of(c, seq, p1);
-      if (pg >= 0) id1 = (uint32_t)(pg * kPageTokens + (p1 & (kPageTokens - 1)));
-    }
+    // physical row: a sequence's last 128 entries come from the sliding-window
+    // store when there is one, every other entry from its cache page
+    const int64_t swa_from = c.swa ? (int64_t)seq_len_of(c, seq) - kReplay : INT64_MAX;
+    auto row_id = [&](int64_t p) -> uint32_t {
+      if (p >= swa_from) return kSwaRow | (uint32_t)(seq * kReplay + (int)(p & (kReplay - 1)));
+      const int64_t pg = page_of(c, seq, p);
+      return pg >= 0 ? (uint32_t)(pg * kPageTokens + (p & (kPageTokens - 1))) : kNoRow;
+    };
+    if (u0) id0 = row_id(p0);
+    if (u1) id1 = row_id(p1);
   }
   // largest |q| of the warp (the loads above were in flight meanwhile)
   uint32_t qmax = 0;   // as bf16 bits: magnitudes order like their bit patterns
@@ -600,8 +604,8 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
     // registers take tile t + 2, about one pipeline step ahead of its decode
     // (two buffers keep the loop body small: three would triple the code)
     RawTile A, B;
-    if (nt > 0) raw_load(A, c.kv, rows_s, 0, nrow, rsub, piece);
-    if (nt > 1) raw_load(B, c.kv, rows_s, 1, nrow, rsub, piece);
+    if (nt > 0) raw_load(A, c.kv, c.swa, rows_s, 0, nrow, rsub, piece);
+    if (nt > 1) raw_load(B, c.kv, c.swa, rows_s, 1, nrow, rsub, piece);
     store_q();
     auto step = [&](int t, RawTile& D) -> bool {
       const int b = t & 1;
@@ -609,7 +613,7 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
       raw_decode(D, sp, kOffK + b * kKtBytes, rsub, piece, soff);
       fence_async_smem();
       mbar_arrive(kfull(b));
-      if (t + 2 < nt) raw_load(D, c.kv, rows_s, t + 2, nrow, rsub, piece);
+      if (t + 2 < nt) raw_load(D, c.kv, c.swa, rows_s, t + 2, nrow, rsub, piece);
       return true;
     };
 #pragma unroll 1

@@ -41,6 +41,7 @@ struct CacheView {
   int32_t batch;
   const int32_t* seq_lens;
   uint32_t* err;
+  uint8_t* swa;   // separate sliding-window store [batch][128][288 B], or nullptr
 };
 
 __device__ __forceinline__ void raise_error(uint32_t* err, uint32_t bits) { atomicOr(err, bits); }

@@ -65,34 +65,36 @@ __device__ __forceinline__ void unpack8(const uint4& v, float* out) {
   out[6] = bf16_lo(v.w); out[7] = bf16_hi(v.w);
 }
 
-// One warp: encode input row(s) `src` (compress 1 or 2 consecutive bf16 rows of
-// 512) into the cache row at (seq, pos), and store the indexer key.
-__device__ __forceinline__ void encode_entry_warp(const CacheView& c, int lane,
-                                                 const uint16_t* __restrict__ kv_src,
-                                                 const uint16_t* __restrict__ idxk_src,
-                                                 int compress, int seq, int64_t pos) {
-  const int64_t page = page_of(c, seq, pos);
-  if (page < 0) return;
+// One warp: the FP4 code of an entry made of `compress` (1 or 2) consecutive
+// bf16 rows of 512 at kv_src (pair mean in fp32 at ratio 2); lane l gets
+// scale group l.
+__device__ __forceinline__ GroupCode encode_src_warp(int lane, const uint16_t* __restrict__ kv_src,
+                                                     int compress) {
   float x[16];
-  {
-    const uint4* r0 = reinterpret_cast<const uint4*>(kv_src) + lane * 2;
-    unpack8(__ldg(r0), x);
-    unpack8(__ldg(r0 + 1), x + 8);
-    if (compress == 2) {
-      float y[16];
-      const uint4* r1 = reinterpret_cast<const uint4*>(kv_src + kD) + lane * 2;
-      unpack8(__ldg(r1), y);
-      unpack8(__ldg(r1 + 1), y + 8);
+  const uint4* r0 = reinterpret_cast<const uint4*>(kv_src) + lane * 2;
+  unpack8(__ldg(r0), x);
+  unpack8(__ldg(r0 + 1), x + 8);
+  if (compress == 2) {
+    float y[16];
+    const uint4* r1 = reinterpret_cast<const uint4*>(kv_src + kD) + lane * 2;
+    unpack8(__ldg(r1), y);
+    unpack8(__ldg(r1 + 1), y + 8);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) x[j] = __fmul_rn(__fadd_rn(x[j], y[j]), 0.5f);
-    }
+    for (int j = 0; j < 16; ++j) x[j] = __fmul_rn(__fadd_rn(x[j], y[j]), 0.5f);
   }
-  const GroupCode g = encode_group(x);
-  uint8_t* row = c.kv + page * kPageBytes + (pos & (kPageTokens - 1)) * kRowBytes;
+  return encode_group(x);
+}
+
+// One warp: store a row's codes (256 B) and scales (32 B tail).
+__device__ __forceinline__ void store_row_warp(uint8_t* row, int lane, const GroupCode& g) {
   reinterpret_cast<uint2*>(row)[lane] = g.codes;
   row[kCodeBytes + lane] = (uint8_t)g.scale;
+}
 
-  // indexer key: lane owns dims 2*lane, 2*lane+1
+// One warp: the stored indexer key of an entry (lane owns dims 2 lane, 2 lane + 1;
+// pair mean rounded to bf16 at ratio 2).
+__device__ __forceinline__ uint32_t idxk_src_warp(int lane, const uint16_t* __restrict__ idxk_src,
+                                                  int compress) {
   uint32_t kw = __ldg(reinterpret_cast<const uint32_t*>(idxk_src) + lane);
   if (compress == 2) {
     const uint32_t kw2 = __ldg(reinterpret_cast<const uint32_t*>(idxk_src + kIdxDim) + lane);
@@ -100,6 +102,27 @@ __device__ __forceinline__ void encode_entry_warp(const CacheView& c, int lane,
     const float b = __fmul_rn(__fadd_rn(bf16_hi(kw), bf16_hi(kw2)), 0.5f);
     kw = (uint32_t)f32_to_bf16_rne(a) | ((uint32_t)f32_to_bf16_rne(b) << 16);
   }
+  return kw;
+}
+
+// Slot of position pos of sequence seq in the sliding-window store.
+__device__ __forceinline__ uint8_t* swa_row(const CacheView& c, int seq, int64_t pos) {
+  return c.swa + ((int64_t)seq * kReplay + (pos & (kReplay - 1))) * kRowBytes;
+}
+
+// One warp: encode an entry into the cache row at (seq, pos) and store its
+// indexer key; with a sliding-window store, an entry among the sequence's
+// last 128 positions (pos >= len - 128) is also written to its slot there.
+__device__ __forceinline__ void encode_entry_warp(const CacheView& c, int lane,
+                                                 const uint16_t* __restrict__ kv_src,
+                                                 const uint16_t* __restrict__ idxk_src,
+                                                 int compress, int seq, int64_t pos, int64_t len) {
+  const int64_t page = page_of(c, seq, pos);
+  if (page < 0) return;
+  const GroupCode g = encode_src_warp(lane, kv_src, compress);
+  store_row_warp(c.kv + page * kPageBytes + (pos & (kPageTokens - 1)) * kRowBytes, lane, g);
+  if (c.swa && pos >= len - kReplay) store_row_warp(swa_row(c, seq, pos), lane, g);
+  const uint32_t kw = idxk_src_warp(lane, idxk_src, compress);
   uint8_t* krow = c.idxk + page * kIdxPageBytes + (pos & (kPageTokens - 1)) * kIdxRowBytes;
   reinterpret_cast<uint32_t*>(krow)[lane] = kw;
 }
@@ -143,12 +166,13 @@ __global__ void __launch_bounds__(256) append_rows_kernel(CacheView c, const uin
     if (lane == 0) raise_error(c.err, CSA2_DEVERR_SEQ);
     return;
   }
-  if (pos < 0 || pos >= c.seq_lens[seq]) {
+  const int64_t len = c.seq_lens[seq];
+  if (pos < 0 || pos >= len) {
     if (lane == 0) raise_error(c.err, CSA2_DEVERR_POS);
     return;
   }
   encode_entry_warp(c, lane, kv + (int64_t)i * compress * kD, idxk + (int64_t)i * compress * kIdxDim,
-                    compress, seq, pos);
+                    compress, seq, pos, len);
 }
 
 // Block keys of the blocks touched by an append.  Entry i recomputes its
@@ -171,10 +195,13 @@ __global__ void __launch_bounds__(256) append_block_keys_kernel(CacheView c,
   block_key_warp(c, lane, seq, blk, len);
 }
 
-// Replay: warp (b, r) handles row r of the supplied last-128 block of seq b.
+// Replay: warp (b, r) handles entry r of the supplied last-128 block of seq b
+// (raw rows [compress r, compress r + compress) of that block).  With a
+// sliding-window store only its slot is rewritten; otherwise the cache row and
+// the indexer key.
 __global__ void __launch_bounds__(256) replay_rows_kernel(CacheView c, const uint16_t* __restrict__ kv_last,
                                                           const uint16_t* __restrict__ idxk_last,
-                                                          const uint8_t* __restrict__ miss) {
+                                                          const uint8_t* __restrict__ miss, int compress) {
   const int lane = threadIdx.x & 31;
   const int b = blockIdx.y;
   const int r = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
@@ -183,8 +210,12 @@ __global__ void __launch_bounds__(256) replay_rows_kernel(CacheView c, const uin
   const int64_t nrep = miss[b] ? (len < kReplay ? len : (int64_t)kReplay) : (len > 0 ? 1 : 0);
   if (r < kReplay - nrep) return;
   const int64_t pos = len - kReplay + r;
-  const int64_t row = (int64_t)b * kReplay + r;
-  encode_entry_warp(c, lane, kv_last + row * kD, idxk_last + row * kIdxDim, 1, b, pos);
+  const int64_t row = ((int64_t)b * kReplay + r) * compress;
+  if (c.swa) {
+    store_row_warp(swa_row(c, b, pos), lane, encode_src_warp(lane, kv_last + row * kD, compress));
+    return;
+  }
+  encode_entry_warp(c, lane, kv_last + row * kD, idxk_last + row * kIdxDim, compress, b, pos, len);
 }
 
 // Replay block keys: warp (b, j) recomputes the j-th block touched in seq b.
@@ -215,9 +246,10 @@ cudaError_t launch_append(const CacheView& c, const uint16_t* kv, const uint16_t
 }
 
 cudaError_t launch_replay(const CacheView& c, const uint16_t* kv_last, const uint16_t* idxk_last,
-                          const uint8_t* miss, cudaStream_t st) {
+                          const uint8_t* miss, int compress, cudaStream_t st) {
   dim3 g1(kReplay / kWarpsPerCta, c.batch);
-  replay_rows_kernel<<<g1, 256, 0, st>>>(c, kv_last, idxk_last, miss);
+  replay_rows_kernel<<<g1, 256, 0, st>>>(c, kv_last, idxk_last, miss, compress);
+  if (c.swa) return cudaGetLastError();   // the global cache's keys are untouched
   // a 128-token window touches at most 17 blocks of 8
   dim3 g2((kReplay / kBlock + 1 + kWarpsPerCta - 1) / kWarpsPerCta, c.batch);
   replay_block_keys_kernel<<<g2, 256, 0, st>>>(c, miss);

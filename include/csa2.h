@@ -92,13 +92,17 @@ typedef struct {
   void* kv_pool;              /* n_pages * 18432 B, 16-B aligned               */
   void* idxk_pool;            /* n_pages * 8192 B, 16-B aligned                */
   void* blockkey_pool;        /* n_pages * 1024 B, 16-B aligned                */
-  int64_t n_pages;
+  int64_t n_pages;            /* 1 .. 2^25 (attention names rows by 31 bits)   */
   const int32_t* page_table;  /* int32 [batch][max_pages]                      */
   int32_t max_pages;
-  int32_t batch;
+  int32_t batch;              /* 1 .. 2^23                                     */
   const int32_t* seq_lens;    /* int32 [batch]: entries present per sequence   */
   uint32_t* error_word;       /* one uint32, zeroed by the caller              */
   uint64_t cache_id;          /* caller-chosen identity used by mode checks    */
+  void* swa_rows;             /* optional separate sliding-window store, NULL:
+                                 none (the window is read from kv_pool); else
+                                 [batch][128][288 B] FP4 rows, 16-B aligned,
+                                 position p of sequence b in slot p % 128      */
 } csa2_cache;
 
 /* Index sets produced by the indexer and consumed by attention.  Device
@@ -156,7 +160,9 @@ void csa2_indexset_attach_rows(csa2_indexset* set, int32_t* attn_rows);
  * indexer key is stored as bf16; the block key of every touched 8-token block
  * is recomputed as bf16(fp32 mean of the block's present keys, ascending
  * order).  seq_lens must already count the new entries (entry_pos[i] <
- * seq_lens[seq]).  kv and idxk must be 16-B aligned.
+ * seq_lens[seq]).  kv and idxk must be 16-B aligned.  With a sliding-window
+ * store (cache->swa_rows), entries among their sequence's last 128 positions
+ * are also written to their slot there.
  */
 int csa2_kv_quant_append(const csa2_cache* cache, const uint16_t* kv, const uint16_t* idxk,
                          const int32_t* entry_seq, const int32_t* entry_pos, int32_t n,
@@ -222,15 +228,23 @@ int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int32_t heads, 
  *
  * On a cache miss only the last 128 tokens are recomputed (ai-wave.ru, second
  * paragraph; news.hamidun.com, section "Три механизма экономии памяти";
- * agentnet.co.il, section "ארכיטקטורה שחותכת בחצי את הפריפיל").  For every
- * sequence b with L = seq_lens[b]: if miss[b] != 0, positions
- * [L - min(128, L), L) are re-encoded from the last min(128, L) rows of
- * kv_last[b] (bf16 [batch][128][512]) and idxk_last[b] (bf16
- * [batch][128][64]); otherwise only position L-1 is written, from row 127.
- * Same codec and block-key rule as csa2_kv_quant_append (ratio 1).
+ * agentnet.co.il, section "ארכיטקטורה שחותכת בחצי את הפריפיל"), in the decoder
+ * and in the encoder (same agentnet.co.il section: 128 tokens instead of
+ * layers x window).  For every sequence b with L = seq_lens[b] entries: if
+ * miss[b] != 0, entries [L - min(128, L), L) are re-encoded from the last
+ * min(128, L) entries' raw rows of kv_last[b] (bf16 [batch][128 compress][512],
+ * entry r of the block made of raw rows [compress r, compress r + compress),
+ * averaged in fp32 when compress == 2) and idxk_last[b] (bf16
+ * [batch][128 compress][64]); otherwise only entry L-1 is written, from the
+ * block's last entry.  Same codec as csa2_kv_quant_append.  Without a
+ * sliding-window store the rows, indexer keys and block keys of kv_pool are
+ * rewritten; with one (cache->swa_rows) only its slots are rewritten -- the
+ * window lives apart from the global cache (ai-wave.ru, fourth paragraph;
+ * agentnet.co.il, section "קוונטיזציה ופריסה: FP4 ו-DRAM במקום SSD") -- and
+ * idxk_last may be NULL.
  */
 int csa2_swa_replay(const csa2_cache* cache, const uint16_t* kv_last, const uint16_t* idxk_last,
-                    const uint8_t* miss, csa2_stream_t stream);
+                    const uint8_t* miss, int32_t compress, csa2_stream_t stream);
 
 /*
  * csa2_indexer_score_topk_noalloc -- csa2_indexer_score_topk without a

@@ -16,19 +16,34 @@ What the pages fix (agentnet.co.il, "דיפסיק משיקה את V4.1-פלאש 
 
 Bounded replay: on a cache miss only the last 128 tokens are recomputed
 (ai-wave.ru, second paragraph; agentnet.co.il, sections "ארכיטקטורה שחותכת
-בחצי את הפריפיל" and "קוונטיזציה ופריסה: FP4 ו-DRAM במקום SSD").  Reading:
-a flagged sequence rewrites its last min(128, L) rows from freshly supplied
-bf16 rows; an unflagged one writes only its newest row (position L-1).
+בחצי את הפריפיל" and "קוונטיזציה ופריסה: FP4 ו-DRAM במקום SSD"), in the
+decoder and in the encoder (the latter section: 128 tokens instead of layers
+x window).  Reading: a flagged sequence rewrites its last min(128, L) entries
+from freshly supplied bf16 rows; an unflagged one writes only its newest entry
+(position L-1).  At compression ratio 2 (encoder) an entry is made of two raw
+rows, so the supplied block holds 2 x 128 raw rows.
+
+Sliding-window store: the window's KV is kept apart from the global cache
+(ai-wave.ru, fourth paragraph; agentnet.co.il, section "קוונטיזציה ופריסה: FP4
+ו-DRAM במקום SSD": a separate pool with a short lifetime, never written to
+disk).  Reading: the store holds each sequence's last 128 entries, entry p in
+slot p mod 128, in the cache's FP4 row format; attention reads those entries
+from the store and every older entry from the global cache; replay with a
+store rewrites only the store.
 
 Pinned by tests/test_oracle_modes.py (Reuse reproduces the preceding set
 exactly; Reindex with the Full layer's own query reproduces the Full set;
-group patterns; replay idempotence and poisoned-row restore).
+group patterns; replay idempotence and poisoned-row restore; ratio-2 replay of
+an intact sequence reproduces its entries, and of duplicated raw rows equals
+ratio 1; the store's slots against a first-in first-out queue of the last 128
+appended entries).
 """
 from __future__ import annotations
 
 import numpy as np
 
 from . import attention as attn_mod
+from . import codec as codec_mod
 from . import indexer as idx_mod
 
 DECODER_PATTERN = ["F", "R", "R", "R"] + ["RI", "R", "R", "R"] * 4
@@ -75,3 +90,36 @@ def replay_positions(length: int, miss: bool, window: int = REPLAY) -> tuple[np.
         n = min(window, length)
         return np.arange(length - n, length), np.arange(window - n, window)
     return np.array([length - 1]), np.array([window - 1])
+
+
+def replay_entries(kv_last_bits: np.ndarray, length: int, miss: bool, compress: int = 1,
+                   window: int = REPLAY) -> tuple[np.ndarray, np.ndarray]:
+    """(entry positions rewritten, their packed 288-B rows) for one sequence.
+    kv_last_bits: the raw bf16 rows [window * compress, 512] behind the
+    sequence's last `window` entries; entry r is made of raw rows
+    [compress r, compress r + compress)."""
+    pos, used = replay_positions(length, miss, window)
+    raw = np.asarray(kv_last_bits, dtype=np.uint16).reshape(window, compress, -1)[used]
+    return pos, codec_mod.encode_entries(raw.reshape(-1, raw.shape[-1]), compress)
+
+
+def replay_keys(idxk_last_bits: np.ndarray, length: int, miss: bool, compress: int = 1,
+                window: int = REPLAY) -> tuple[np.ndarray, np.ndarray]:
+    """(entry positions rewritten, their stored bf16 indexer keys) for one
+    sequence replayed without a sliding-window store."""
+    pos, used = replay_positions(length, miss, window)
+    raw = np.asarray(idxk_last_bits, dtype=np.uint16).reshape(window, compress, -1)[used]
+    return pos, codec_mod.idxk_entries(raw.reshape(-1, raw.shape[-1]), compress)
+
+
+def window_store_slots(length: int, window: int = REPLAY) -> tuple[np.ndarray, np.ndarray]:
+    """(entry positions the sliding-window store holds for a sequence of
+    `length` entries, their slots)."""
+    pos = np.arange(max(0, length - window), length, dtype=np.int64)
+    return pos, pos % window
+
+
+def from_window_store(positions, length: int, window: int = REPLAY) -> np.ndarray:
+    """Mask of the attended positions that are read from the sliding-window
+    store rather than the global cache."""
+    return np.asarray(positions, dtype=np.int64) >= length - window

@@ -157,3 +157,20 @@ def test_mode_order_state_machine(csa2_lib):
                                      f.p(), 16, None) == 5
     assert L.csa2_indexer_score_topk(B(c), f.p(8), None, f.p(), None, 2, 65536, FULL, 1, 9, B(s),
                                      f.p(), 1 << 30, None) == 3
+
+
+def test_replay_and_cache_argument_checks(csa2_lib):
+    L = csa2_lib.lib()
+    f = _Fake()
+    c = _cache(csa2_lib, f)
+    B = ctypes.byref
+    rep = lambda cache, kv, k, miss, comp: L.csa2_swa_replay(B(cache), kv, k, miss, comp, None)
+    assert rep(c, f.p(), f.p(), f.p(), 3) == 2                 # compression ratio 1 or 2
+    assert rep(c, f.p(), f.p(), f.p(), 0) == 2
+    assert rep(c, f.p(), None, f.p(), 1) == 1                  # keys needed without a window store
+    assert rep(c, None, f.p(), f.p(), 1) == 1
+    assert rep(c, f.p(8), f.p(), f.p(), 2) == 3
+    assert rep(_cache(csa2_lib, f, swa_rows=f.p(8)), f.p(), None, f.p(), 1) == 3   # store 16-B aligned
+    # attention names rows by 31-bit ids: the pool and batch limits
+    assert rep(_cache(csa2_lib, f, n_pages=(1 << 25) + 1), f.p(), f.p(), f.p(), 1) == 2
+    assert rep(_cache(csa2_lib, f, batch=(1 << 23) + 1), f.p(), f.p(), f.p(), 1) == 2

@@ -96,3 +96,60 @@ def test_replay_idempotent_and_restores_poisoned_rows():
     again = poisoned.copy()
     again[pos] = codec.encode_bf16_rows(last[src])
     np.testing.assert_array_equal(again, cache)
+
+
+@pytest.mark.parametrize("L", [300, 50, 128, 1])
+def test_ratio2_replay_of_an_intact_sequence_reproduces_its_entries(L):
+    """Encoder replay at compression ratio 2: the supplied block holds the raw
+    rows of the last 128 entries (two per entry, zero rows ahead of a short
+    sequence); re-encoding them gives back the entries the append made."""
+    rng = np.random.default_rng(L)
+    raw = _bf16(rng.standard_normal((2 * L, 512)))
+    rawk = _bf16(rng.standard_normal((2 * L, 64)))
+    entries = codec.encode_entries(raw, 2)
+    keys = codec.idxk_entries(rawk, 2)
+    n = min(128, L)
+    block = np.zeros((256, 512), np.uint16)
+    block[256 - 2 * n:] = raw[2 * (L - n):]
+    kblock = np.zeros((256, 64), np.uint16)
+    kblock[256 - 2 * n:] = rawk[2 * (L - n):]
+    for miss in (True, False):
+        pos, rows = modes.replay_entries(block, L, miss, compress=2)
+        kpos, krows = modes.replay_keys(kblock, L, miss, compress=2)
+        np.testing.assert_array_equal(pos, np.arange(L - n, L) if miss else [L - 1])
+        np.testing.assert_array_equal(kpos, pos)
+        np.testing.assert_array_equal(rows, entries[pos])
+        np.testing.assert_array_equal(krows, keys[pos])
+
+
+def test_ratio2_replay_of_duplicated_rows_equals_ratio1():
+    """The pair mean of two equal bf16 rows is the row itself (exact in fp32),
+    so a block whose raw rows come in equal pairs replays to the ratio-1
+    encoding of one row of each pair."""
+    rng = np.random.default_rng(3)
+    x = _bf16(rng.standard_normal((128, 512)) * rng.uniform(0.01, 50, (128, 1)))
+    k = _bf16(rng.standard_normal((128, 64)))
+    pos, rows = modes.replay_entries(np.repeat(x, 2, axis=0), 700, True, compress=2)
+    np.testing.assert_array_equal(pos, np.arange(572, 700))
+    np.testing.assert_array_equal(rows, codec.encode_bf16_rows(x))
+    _, krows = modes.replay_keys(np.repeat(k, 2, axis=0), 700, True, compress=2)
+    np.testing.assert_array_equal(krows, k)
+    # ratio 1 reads the block row by row
+    _, rows1 = modes.replay_entries(x, 700, True, compress=1)
+    np.testing.assert_array_equal(rows1, codec.encode_bf16_rows(x))
+
+
+def test_window_store_holds_the_last_128_entries():
+    """Against a first-in first-out queue of capacity 128 fed one entry at a
+    time: the store's positions are the queue's content, each in its own slot,
+    and the attended positions read from the store are exactly those."""
+    import collections
+    fifo = collections.deque(maxlen=128)
+    for L in range(1, 700):
+        fifo.append(L - 1)
+        if L in (1, 2, 127, 128, 129, 255, 256, 300, 699):
+            pos, slot = modes.window_store_slots(L)
+            np.testing.assert_array_equal(pos, np.array(fifo))
+            assert len(set(slot.tolist())) == pos.size and slot.min() >= 0 and slot.max() < 128
+            probe = np.arange(L)
+            np.testing.assert_array_equal(modes.from_window_store(probe, L), np.isin(probe, list(fifo)))
