@@ -65,20 +65,37 @@ __device__ __forceinline__ void unpack8(const uint4& v, float* out) {
   out[6] = bf16_lo(v.w); out[7] = bf16_hi(v.w);
 }
 
-// One warp: the FP4 code of an entry made of `compress` (1 or 2) consecutive
-// bf16 rows of 512 at kv_src (pair mean in fp32 at ratio 2); lane l gets
-// scale group l.
-__device__ __forceinline__ GroupCode encode_src_warp(int lane, const uint16_t* __restrict__ kv_src,
-                                                     int compress) {
-  float x[16];
+// One lane's share of an entry's source: scale group `lane` of the one or two
+// (compress 1 or 2) consecutive bf16 rows of 512 at kv_src.  Loaded before the
+// entry's position is known, so that these loads overlap the lookups.
+struct SrcWords {
+  uint4 a0, a1, b0, b1;
+};
+
+__device__ __forceinline__ SrcWords load_src_lane(int lane, const uint16_t* __restrict__ kv_src, int compress) {
+  SrcWords w;
   const uint4* r0 = reinterpret_cast<const uint4*>(kv_src) + lane * 2;
-  unpack8(__ldg(r0), x);
-  unpack8(__ldg(r0 + 1), x + 8);
+  w.a0 = __ldg(r0);
+  w.a1 = __ldg(r0 + 1);
+  if (compress == 2) {
+    const uint4* r1 = reinterpret_cast<const uint4*>(kv_src + kD) + lane * 2;
+    w.b0 = __ldg(r1);
+    w.b1 = __ldg(r1 + 1);
+  } else {
+    w.b0 = w.b1 = make_uint4(0, 0, 0, 0);
+  }
+  return w;
+}
+
+// The FP4 code of scale group `lane` of an entry (pair mean in fp32 at ratio 2).
+__device__ __forceinline__ GroupCode encode_src_lane(const SrcWords& w, int compress) {
+  float x[16];
+  unpack8(w.a0, x);
+  unpack8(w.a1, x + 8);
   if (compress == 2) {
     float y[16];
-    const uint4* r1 = reinterpret_cast<const uint4*>(kv_src + kD) + lane * 2;
-    unpack8(__ldg(r1), y);
-    unpack8(__ldg(r1 + 1), y + 8);
+    unpack8(w.b0, y);
+    unpack8(w.b1, y + 8);
 #pragma unroll
     for (int j = 0; j < 16; ++j) x[j] = __fmul_rn(__fadd_rn(x[j], y[j]), 0.5f);
   }
@@ -113,13 +130,12 @@ __device__ __forceinline__ uint8_t* swa_row(const CacheView& c, int seq, int64_t
 // One warp: encode an entry into the cache row at (seq, pos) and store its
 // indexer key; with a sliding-window store, an entry among the sequence's
 // last 128 positions (pos >= len - 128) is also written to its slot there.
-__device__ __forceinline__ void encode_entry_warp(const CacheView& c, int lane,
-                                                 const uint16_t* __restrict__ kv_src,
+__device__ __forceinline__ void encode_entry_warp(const CacheView& c, int lane, const SrcWords& src,
                                                  const uint16_t* __restrict__ idxk_src,
                                                  int compress, int seq, int64_t pos, int64_t len) {
   const int64_t page = page_of(c, seq, pos);
   if (page < 0) return;
-  const GroupCode g = encode_src_warp(lane, kv_src, compress);
+  const GroupCode g = encode_src_lane(src, compress);
   store_row_warp(c.kv + page * kPageBytes + (pos & (kPageTokens - 1)) * kRowBytes, lane, g);
   if (c.swa && pos >= len - kReplay) store_row_warp(swa_row(c, seq, pos), lane, g);
   const uint32_t kw = idxk_src_warp(lane, idxk_src, compress);
@@ -160,6 +176,7 @@ __global__ void __launch_bounds__(256) append_rows_kernel(CacheView c, const uin
   const int lane = threadIdx.x & 31;
   const int i = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
   if (i >= n) return;
+  const SrcWords src = load_src_lane(lane, kv + (int64_t)i * compress * kD, compress);
   const int seq = eseq[i];
   const int64_t pos = epos[i];
   if (seq < 0 || seq >= c.batch) {
@@ -171,8 +188,7 @@ __global__ void __launch_bounds__(256) append_rows_kernel(CacheView c, const uin
     if (lane == 0) raise_error(c.err, CSA2_DEVERR_POS);
     return;
   }
-  encode_entry_warp(c, lane, kv + (int64_t)i * compress * kD, idxk + (int64_t)i * compress * kIdxDim,
-                    compress, seq, pos, len);
+  encode_entry_warp(c, lane, src, idxk + (int64_t)i * compress * kIdxDim, compress, seq, pos, len);
 }
 
 // Block keys of the blocks touched by an append.  Entry i recomputes its
@@ -211,11 +227,13 @@ __global__ void __launch_bounds__(256) replay_rows_kernel(CacheView c, const uin
   if (r < kReplay - nrep) return;
   const int64_t pos = len - kReplay + r;
   const int64_t row = ((int64_t)b * kReplay + r) * compress;
+  // the source loads and the page lookup below are in flight together
+  const SrcWords src = load_src_lane(lane, kv_last + row * kD, compress);
   if (c.swa) {
-    store_row_warp(swa_row(c, b, pos), lane, encode_src_warp(lane, kv_last + row * kD, compress));
+    store_row_warp(swa_row(c, b, pos), lane, encode_src_lane(src, compress));
     return;
   }
-  encode_entry_warp(c, lane, kv_last + row * kD, idxk_last + row * kIdxDim, compress, b, pos, len);
+  encode_entry_warp(c, lane, src, idxk_last + row * kIdxDim, compress, b, pos, len);
 }
 
 // Replay block keys: warp (b, j) recomputes the j-th block touched in seq b.

@@ -26,6 +26,10 @@ Readings taken where the pages are silent:
   output set is listed in ascending position order;
 * Reindex ranks the tokens of the pool that the Full layer built.
 
+Keys are bf16 bit patterns [n, 64] or FP8 keys (oracle.idxk_fp8.Fp8Keys):
+an FP8 key's score is its scale times the score of its code values, and
+block keys are built from the dequantised keys.
+
 The score arithmetic is fp32, as in the kernels, because its result decides
 integer outcomes (which positions are selected).
 
@@ -39,6 +43,7 @@ from __future__ import annotations
 import numpy as np
 
 from .formats import bf16_to_f32, f32_to_bf16
+from .idxk_fp8 import Fp8Keys, code_values
 
 IDX_HEADS = 4
 IDX_DIM = 64
@@ -47,10 +52,13 @@ POOL_BLOCKS = 2048  # blocks in the candidate pool
 TOP_K = 512         # indices selected per query
 
 
-def block_keys(key_bits: np.ndarray, length: int, block: int = BLOCK) -> np.ndarray:
+def block_keys(key_bits, length: int, block: int = BLOCK) -> np.ndarray:
     """Mean-pooled block keys (bf16 bits [ceil(L/block), 64]) of the first
-    `length` stored keys."""
-    k = bf16_to_f32(np.asarray(key_bits)[:length])
+    `length` stored keys (bf16 bits, or FP8 keys through their dequantised values)."""
+    if isinstance(key_bits, Fp8Keys):
+        k = key_bits[:length].dequantized()
+    else:
+        k = bf16_to_f32(np.asarray(key_bits)[:length])
     nb = (length + block - 1) // block
     acc = np.zeros((nb, k.shape[1]), dtype=np.float32)
     cnt = np.zeros(nb, dtype=np.float32)
@@ -63,10 +71,16 @@ def block_keys(key_bits: np.ndarray, length: int, block: int = BLOCK) -> np.ndar
     return f32_to_bf16(mean)
 
 
-def index_scores(q_bits: np.ndarray, key_bits: np.ndarray, w: np.ndarray | None = None) -> np.ndarray:
-    """fp32 scores [n] of one indexer query q [4,64] against keys [n,64]."""
-    q = bf16_to_f32(q_bits)
-    k = bf16_to_f32(key_bits)
+def index_scores(q_bits: np.ndarray, key_bits, w: np.ndarray | None = None) -> np.ndarray:
+    """fp32 scores [n] of one indexer query q [4,64] against keys [n,64]
+    (bf16 bits, or FP8 keys: fl32(scale x score of the code values))."""
+    if isinstance(key_bits, Fp8Keys):
+        total = _scores_f32(bf16_to_f32(q_bits), code_values(key_bits.codes), w)
+        return (key_bits.scales * total).astype(np.float32)
+    return _scores_f32(bf16_to_f32(q_bits), bf16_to_f32(key_bits), w)
+
+
+def _scores_f32(q: np.ndarray, k: np.ndarray, w) -> np.ndarray:
     heads = q.shape[0]
     wv = np.ones(heads, dtype=np.float32) if w is None else np.asarray(w, dtype=np.float32)
     total = np.zeros(k.shape[0], dtype=np.float32)
@@ -102,7 +116,8 @@ def pool_tokens(pool_blocks: np.ndarray, length: int, block: int = BLOCK) -> np.
 def select_tokens(q_bits, key_bits, candidates: np.ndarray, w=None, k: int = TOP_K):
     """Top-k token positions among `candidates` (ascending positions)."""
     cand = np.asarray(candidates, dtype=np.int64)
-    s = index_scores(q_bits, np.asarray(key_bits)[cand], w)
+    keys = key_bits if isinstance(key_bits, Fp8Keys) else np.asarray(key_bits)
+    s = index_scores(q_bits, keys[cand], w)
     sel = top_k(s, np.ones(cand.size, dtype=bool), k)
     out = np.full(k, -1, dtype=np.int64)
     m = sel >= 0
