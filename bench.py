@@ -369,6 +369,8 @@ def run_gpu(args):
         "clocks": clocks,
     }
     result["window_store"] = measure_window_store(w, cache, step, stream, flush, peaks, reuse_ms)
+    result["fp8_indexer_keys"] = measure_fp8_keys(
+        w, stream, flush, peaks, {"step": ms_per_step, "full": idx_full_ms, "reindex": idx_ri_ms})
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args, seqs=tuple(range(w.batch)))
     finish_ranks(world)
@@ -457,6 +459,49 @@ def measure_window_store(w, cache, step, stream, flush, peaks, attn_global_ms):
         "step_outputs_bit_identical": bool(same),
         "note": "CUDA graphs of one call (replay) or 2 x 3 Reuse calls (attention), L2 flushed first; "
                 "bytes: bf16 rows read + FP4 rows (and keys) written",
+    }
+
+
+def measure_fp8_keys(w, stream, flush, peaks, bf16_ms):
+    """The same decode step on a cache whose indexer keys are FP8 (64 E4M3 codes
+    + one fp32 scale, 68 B per token instead of 128 B), outside the timed region:
+    the step as one CUDA graph, and the Full and Reindex indexer calls alone."""
+    import torch
+
+    from fp4_kv_cache_decode_b200 import csa2, synthetic
+    cache = synthetic.new_cache(w, cache_id=3, idxk_format=csa2.IDXK_FP8)
+    synthetic.fill_decode_cache(w, cache)
+    step = synthetic.DecodeStep(w, cache)
+    step.run()
+    torch.cuda.synchronize()
+    assert csa2.csa2_check_device_error(cache) == 0
+    step_ms = _graph_ms(step.run, flush, stream, reps=7)
+    f_layer, ri_layer = w.layers.index("F"), w.layers.index("RI")
+    full_ms = _graph_ms(lambda: csa2.csa2_indexer_score_topk(
+        cache, step.idxq[f_layer], step.q_seq, csa2.FULL, f_layer, step.iset, step.ws_idx, step.max_visible),
+        flush, stream)
+    ri_ms = _graph_ms(lambda: csa2.csa2_indexer_score_topk(
+        cache, step.idxq[ri_layer], step.q_seq, csa2.REINDEX, ri_layer, step.iset, step.ws_idx,
+        step.max_visible), flush, stream)
+    assert csa2.csa2_check_device_error(cache) == 0
+    B, L = w.batch, w.lengths[0]
+    nb = (L + 7) // 8
+    full_bytes = B * (nb * 128 + 16384 * 68)
+    ri_bytes = B * 16384 * 68
+    del step, cache
+    torch.cuda.empty_cache()
+    return {
+        "layer_steps_per_s": len(w.layers) / (step_ms * 1e-3),
+        "step_ms": step_ms,
+        "step_ms_bf16_keys": bf16_ms["step"],
+        "indexer_full_ms": full_ms, "indexer_full_ms_bf16_keys": bf16_ms["full"],
+        "indexer_reindex_ms": ri_ms, "indexer_reindex_ms_bf16_keys": bf16_ms["reindex"],
+        "indexer_full_gbs": full_bytes / (full_ms * 1e-3) / 1e9,
+        "indexer_reindex_gbs": ri_bytes / (ri_ms * 1e-3) / 1e9,
+        "hbm_peak_gbs": peaks["hbm_gbs"],
+        "bytes_per_token": {"main_kv": 288, "indexer_key": 68, "block_key_share": 16},
+        "note": "median of CUDA-graph replays, L2 flushed first; Full bytes = block keys (bf16) + "
+                "16,384 pool keys x 68 B per query; the step's timed line above uses bf16 keys",
     }
 
 

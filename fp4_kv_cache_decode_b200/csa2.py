@@ -21,6 +21,8 @@ ROW_BYTES = 288
 PAGE_TOKENS = 64
 PAGE_BYTES = ROW_BYTES * PAGE_TOKENS
 IDX_PAGE_BYTES = 64 * 128
+IDX8_PAGE_BYTES = 64 * 64 + 64 * 4   # FP8 indexer keys: codes, then fp32 scales
+IDXK_BF16, IDXK_FP8 = 0, 1
 BK_PAGE_BYTES = 8 * 128
 TOP_K = 512
 POOL_BLOCKS = 2048
@@ -49,6 +51,7 @@ class CacheStruct(ctypes.Structure):
         ("error_word", ctypes.c_void_p),
         ("cache_id", ctypes.c_uint64),
         ("swa_rows", ctypes.c_void_p),
+        ("idxk_format", ctypes.c_int32),
     ]
 
 
@@ -146,15 +149,18 @@ _I32T = (torch.int32,)
 
 
 class Cache:
-    """Paged FP4 cache: three page pools, page table, lengths, error word, and
-    (swa_store=True) a separate sliding-window store [batch, 128, 288] bytes."""
+    """Paged FP4 cache: three page pools, page table, lengths, error word,
+    (swa_store=True) a separate sliding-window store [batch, 128, 288] bytes, and
+    the indexer-key format (IDXK_BF16 or IDXK_FP8)."""
 
     def __init__(self, n_pages: int, batch: int, max_pages: int, device="cuda", cache_id: int = 1,
-                 swa_store: bool = False):
+                 swa_store: bool = False, idxk_format: int = IDXK_BF16):
         dev = torch.device(device)
         self.n_pages, self.batch, self.max_pages = n_pages, batch, max_pages
         self.kv_pool = torch.zeros(n_pages * PAGE_BYTES, dtype=torch.uint8, device=dev)
-        self.idxk_pool = torch.zeros(n_pages * IDX_PAGE_BYTES, dtype=torch.uint8, device=dev)
+        self.idxk_format = idxk_format
+        kpage = IDX8_PAGE_BYTES if idxk_format == IDXK_FP8 else IDX_PAGE_BYTES
+        self.idxk_pool = torch.zeros(n_pages * kpage, dtype=torch.uint8, device=dev)
         self.bk_pool = torch.zeros(n_pages * BK_PAGE_BYTES, dtype=torch.uint8, device=dev)
         self.page_table = torch.full((batch, max_pages), -1, dtype=torch.int32, device=dev)
         self.seq_lens = torch.zeros(batch, dtype=torch.int32, device=dev)
@@ -178,6 +184,7 @@ class Cache:
         s.error_word = self.error_word.data_ptr()
         s.cache_id = self.cache_id
         s.swa_rows = None if self.swa_rows is None else self.swa_rows.data_ptr()
+        s.idxk_format = self.idxk_format
 
     def ref(self):
         return ctypes.byref(self.struct)

@@ -55,6 +55,7 @@ int make_view(const csa2_cache* c, CacheView* v) {
       !c->error_word)
     return CSA2_ERR_INVALID_ARG;
   if (c->n_pages <= 0 || c->max_pages <= 0 || c->batch <= 0) return CSA2_ERR_SHAPE;
+  if (c->idxk_format != CSA2_IDXK_BF16 && c->idxk_format != CSA2_IDXK_FP8) return CSA2_ERR_INVALID_ARG;
   // attention names a physical row by a 31-bit id (page x 64 + slot, or a
   // sliding-window slot batch x 128 + p % 128 under a flag bit)
   if (c->n_pages > ((int64_t)1 << 25) || c->batch > (1 << 23)) return CSA2_ERR_SHAPE;
@@ -72,6 +73,7 @@ int make_view(const csa2_cache* c, CacheView* v) {
   v->seq_lens = c->seq_lens;
   v->err = c->error_word;
   v->swa = static_cast<uint8_t*>(c->swa_rows);
+  v->idxk_fp8 = c->idxk_format == CSA2_IDXK_FP8 ? 1 : 0;
   return CSA2_OK;
 }
 

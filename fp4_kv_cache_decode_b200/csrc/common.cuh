@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "../../include/csa2.h"
 
@@ -24,6 +25,10 @@ constexpr int kIdxPageBytes = kIdxRowBytes * kPageTokens;  // 8192
 constexpr int kBlock = CSA2_BLOCK_TOKENS;             // 8
 constexpr int kBlocksPerPage = kPageTokens / kBlock;  // 8
 constexpr int kBkPageBytes = kBlocksPerPage * kIdxRowBytes;  // 1024
+// FP8 indexer keys: 64 E4M3 code bytes per token, the page's 64 fp32 scales after its codes
+constexpr int kIdx8RowBytes = kIdxDim;                          // 64
+constexpr int kIdx8ScaleOff = kIdx8RowBytes * kPageTokens;      // 4096
+constexpr int kIdx8PageBytes = kIdx8ScaleOff + 4 * kPageTokens;  // 4352
 constexpr int kPoolBlocks = CSA2_POOL_BLOCKS;         // 2048
 constexpr int kTopK = CSA2_TOP_K;                     // 512
 constexpr int kWindow = CSA2_WINDOW;                  // 128
@@ -42,6 +47,7 @@ struct CacheView {
   const int32_t* seq_lens;
   uint32_t* err;
   uint8_t* swa;   // separate sliding-window store [batch][128][288 B], or nullptr
+  int idxk_fp8;   // indexer keys: 0 bf16, 1 E4M3 codes + fp32 scale
 };
 
 __device__ __forceinline__ void raise_error(uint32_t* err, uint32_t bits) { atomicOr(err, bits); }
@@ -83,6 +89,14 @@ __device__ __forceinline__ float e4m3_pos_value(uint32_t b) {
   const uint32_t e = (b >> 3) & 0xFu, m = b & 7u;
   if (e == 0) return (float)m * 0x1p-9f;                    // subnormal m/8 * 2^-6
   return __uint_as_float(((e + 120u) << 23) | (m << 20));   // (1 + m/8) * 2^(e-7)
+}
+
+// Two E4M3 (FN) bytes, the low byte first, to their exact fp32 values (through
+// f16, which holds every E4M3 value).
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t pair) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((unsigned short)(pair & 0xFFFFu)));
+  return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
 // Magnitudes of the E2M1 codes 0..7 (bit 3 is the sign).

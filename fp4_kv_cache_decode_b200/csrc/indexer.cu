@@ -10,6 +10,9 @@
 //   BLOCKKEYS unit u = the 8 block keys stored in page slot u,
 //   POOL      unit u = the 8 tokens of pool block pool[u].
 // score(q, k) = sum_h w_h * max(0, q_h . k), fp32.
+// FP8 indexer keys (E4M3 codes + one fp32 scale s per token): a unit is the 8
+// tokens' 512 code bytes plus their 32 scale bytes, and a key scores
+// s x score(q, code values) -- s >= 0 commutes with the ReLU.
 //
 // Scoring is HBM-bound (4 heads x 64 dims = 4 FLOP per key byte): each warp
 // streams whole units with 16-B non-allocating loads, several units in flight
@@ -32,10 +35,21 @@ enum UnitSource : int { SRC_FLAT = 0, SRC_BLOCKKEYS = 1, SRC_POOL = 2 };
 constexpr int kScoreThreads = 256;
 constexpr int kScoreWarps = kScoreThreads / 32;
 constexpr int kUnitsPerCta = 256;                         // at most 256 KiB of keys per CTA
-constexpr int kStageUnits = 32;                           // 32 KiB per pipeline stage
 constexpr int kStages = 3;
-constexpr int kWarpStageUnits = kStageUnits / kScoreWarps;   // 4 units per warp per stage
-constexpr uint32_t kScoreSmem = kStages * kStageUnits * 1024u;
+
+// Pipeline geometry per key format: 32 units per stage of 1 KiB (bf16 keys) or
+// 544 B (FP8 codes + scales).  The scoring is bound by issue latency, not by
+// the bytes in flight: 64-unit FP8 stages (the same bytes per stage as bf16)
+// were measured slower.
+template <bool F8>
+struct ScoreGeom {
+  static constexpr int kUnits = 32;                           // units per stage
+  static constexpr int kWarpUnits = kUnits / kScoreWarps;     // per warp per stage
+  static constexpr uint32_t kSlot = F8 ? 544u : 1024u;        // bytes per unit slot
+  static constexpr uint32_t kSmem = kStages * kUnits * kSlot;
+};
+constexpr uint32_t kScoreSmemMax = ScoreGeom<false>::kSmem;   // 98,304 B
+static_assert(ScoreGeom<true>::kSmem <= kScoreSmemMax, "stage sizes");
 
 __device__ __forceinline__ int64_t visible_of(const CacheView& c, const int32_t* q_seq,
                                               const int32_t* q_vis, int r) {
@@ -63,7 +77,7 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
 //  3. each lane reads back exactly the bytes it copied (row l/4, dims
 //     16(l%4)..+15), forms its 4 partial head dot products, and two shuffles
 //     finish each row's dot products.  No CTA-wide barrier inside the stream.
-template <int SRC>
+template <int SRC, bool F8>
 __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView c, const uint16_t* __restrict__ idx_q,
                                                                        const float* __restrict__ head_w,
                                                                        const int32_t* __restrict__ q_seq,
@@ -72,7 +86,9 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView
                                                                        int64_t max_units, int64_t stride,
                                                                        int upc, float* __restrict__ scores) {
   extern __shared__ __align__(16) uint8_t stage[];
+  static_assert(!F8 || SRC != SRC_BLOCKKEYS, "block keys are bf16");
   __shared__ const uint8_t* ubase[kUnitsPerCta];
+  __shared__ const uint8_t* uscale[F8 ? kUnitsPerCta : 1];   // FP8: the unit's 8 scales
   __shared__ int32_t urows[kUnitsPerCta];
   const int r = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -83,7 +99,8 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView
     if (blockIdx.x == 0 && tid == 0) raise_error(c.err, CSA2_DEVERR_POS);
     nunits = max_units;
   }
-  const int64_t u0 = (int64_t)blockIdx.x * upc;   // upc <= kUnitsPerCta, a multiple of kStageUnits
+  using G = ScoreGeom<F8>;
+  const int64_t u0 = (int64_t)blockIdx.x * upc;   // upc <= kUnitsPerCta, a multiple of G::kUnits
   if (u0 >= nunits) return;
   const int64_t nb = (v + kBlock - 1) / kBlock;
   const int nu = (int)(nunits - u0 < upc ? nunits - u0 : upc);
@@ -92,12 +109,22 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView
   {
     const int64_t u = u0 + tid;
     const uint8_t* base = nullptr;
+    const uint8_t* sbase = nullptr;
     int nrows = 0;
+    // the unit's codes (and, FP8, scales) within an indexer-key page
+    auto unit_at = [&](int64_t pg, int64_t slot8) {
+      if (F8) {
+        base = c.idxk + pg * kIdx8PageBytes + slot8 * (kBlock * kIdx8RowBytes);
+        sbase = c.idxk + pg * kIdx8PageBytes + kIdx8ScaleOff + slot8 * (kBlock * 4);
+      } else {
+        base = c.idxk + pg * kIdxPageBytes + slot8 * (kBlock * kIdxRowBytes);
+      }
+    };
     if (tid < nu) {
       if (SRC == SRC_FLAT) {
         const int64_t pg = page_of(c, seq, u * kBlock);
         if (pg >= 0) {
-          base = c.idxk + pg * kIdxPageBytes + (u & (kBlocksPerPage - 1)) * (kBlock * kIdxRowBytes);
+          unit_at(pg, u & (kBlocksPerPage - 1));
           nrows = (int)(v - u * kBlock < kBlock ? v - u * kBlock : kBlock);
         }
       } else if (SRC == SRC_BLOCKKEYS) {
@@ -114,7 +141,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView
           } else {
             const int64_t pg = page_of(c, seq, (int64_t)blk * kBlock);
             if (pg >= 0) {
-              base = c.idxk + pg * kIdxPageBytes + (blk & (kBlocksPerPage - 1)) * (kBlock * kIdxRowBytes);
+              unit_at(pg, blk & (kBlocksPerPage - 1));
               nrows = (int)(v - (int64_t)blk * kBlock < kBlock ? v - (int64_t)blk * kBlock : kBlock);
             }
           }
@@ -122,6 +149,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView
       }
     }
     ubase[tid] = base;
+    if (F8) uscale[F8 ? tid : 0] = sbase;
     urows[tid] = nrows;
   }
 
@@ -143,18 +171,23 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView
   __syncthreads();
 
   const uint32_t stage_s = (uint32_t)__cvta_generic_to_shared(stage);
-  const int nstage = (nu + kStageUnits - 1) / kStageUnits;
-  // issue the copies of stage s (this warp's 4 units) into ring slot s % kStages
+  const int nstage = (nu + G::kUnits - 1) / G::kUnits;
+  // issue the copies of stage s (this warp's units) into ring slot s % kStages
   auto issue = [&](int st) {
     if (st < nstage) {
 #pragma unroll
-      for (int i = 0; i < kWarpStageUnits; ++i) {
-        const int j = st * kStageUnits + warp * kWarpStageUnits + i;
+      for (int i = 0; i < G::kWarpUnits; ++i) {
+        const int j = st * G::kUnits + warp * G::kWarpUnits + i;
         const uint8_t* base = ubase[j];
-        const uint32_t dst = stage_s + ((st % kStages) * kStageUnits + warp * kWarpStageUnits + i) * 1024u + lane * 32u;
+        const uint32_t dst = stage_s + ((st % kStages) * G::kUnits + warp * G::kWarpUnits + i) * G::kSlot;
         if (j < nu && base != nullptr) {
-          cp_async16(dst, base + lane * 32);
-          cp_async16(dst + 16, base + lane * 32 + 16);
+          if (F8) {   // 512 code bytes, then the 32 scale bytes
+            cp_async16(dst + lane * 16u, base + lane * 16);
+            if (lane < 2) cp_async16(dst + 512u + lane * 16u, uscale[F8 ? j : 0] + lane * 16);
+          } else {
+            cp_async16(dst + lane * 32u, base + lane * 32);
+            cp_async16(dst + lane * 32u + 16u, base + lane * 32 + 16);
+          }
         }
       }
     }
@@ -167,20 +200,32 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView
     issue(st + 2);
     asm volatile("cp.async.wait_group 2;" ::: "memory");
 #pragma unroll
-    for (int i = 0; i < kWarpStageUnits; ++i) {
-      const int j = st * kStageUnits + warp * kWarpStageUnits + i;
+    for (int i = 0; i < G::kWarpUnits; ++i) {
+      const int j = st * G::kUnits + warp * G::kWarpUnits + i;
       const int64_t u = u0 + j;
       const bool have = j < nu && ubase[j] != nullptr;
-      const uint8_t* sl = stage + ((st % kStages) * kStageUnits + warp * kWarpStageUnits + i) * 1024 + lane * 32;
-      uint4 ka = make_uint4(0, 0, 0, 0), kb = ka;
-      if (have) {
-        ka = *reinterpret_cast<const uint4*>(sl);
-        kb = *reinterpret_cast<const uint4*>(sl + 16);
-      }
-      const uint32_t wk[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+      const uint8_t* su = stage + ((st % kStages) * G::kUnits + warp * G::kWarpUnits + i) * G::kSlot;
       float2 k[8];
+      float srow = 1.0f;   // FP8: the row's scale
+      if (F8) {            // lane l: code bytes 16l..16l+15 = row l/4, dims 16(l%4)..
+        uint4 kc = make_uint4(0, 0, 0, 0);
+        if (have) {
+          kc = *reinterpret_cast<const uint4*>(su + lane * 16);
+          srow = *reinterpret_cast<const float*>(su + 512 + row * 4);
+        }
+        const uint32_t wc[4] = {kc.x, kc.y, kc.z, kc.w};
 #pragma unroll
-      for (int j = 0; j < 8; ++j) k[j] = make_float2(bf16_lo(wk[j]), bf16_hi(wk[j]));
+        for (int j = 0; j < 8; ++j) k[j] = e4m3x2_to_float2(wc[j >> 1] >> (16 * (j & 1)));
+      } else {
+        uint4 ka = make_uint4(0, 0, 0, 0), kb = ka;
+        if (have) {
+          ka = *reinterpret_cast<const uint4*>(su + lane * 32);
+          kb = *reinterpret_cast<const uint4*>(su + lane * 32 + 16);
+        }
+        const uint32_t wk[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) k[j] = make_float2(bf16_lo(wk[j]), bf16_hi(wk[j]));
+      }
       // partial dot products of the lane's 16 dims, even and odd dims in the two halves
       float p[kIdxHeads];
 #pragma unroll
@@ -204,6 +249,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView
       float sc = wsel * fmaxf(p[0], 0.0f);
       sc += __shfl_xor_sync(0xffffffffu, sc, 1);
       sc += __shfl_xor_sync(0xffffffffu, sc, 2);
+      if (F8) sc *= srow;
       if (j < nu && (lane & 3) == 0)
         scores[(int64_t)r * stride + u * kBlock + row] = row < urows[j] ? sc : -INFINITY;
     }
@@ -649,12 +695,12 @@ size_t topk_smem_bytes() { return sizeof(TopkSmem); }
 cudaError_t indexer_set_attributes() {
   const int smem = (int)topk_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(topk_kernel<SRC_FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(score_units_kernel<SRC_FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(score_units_kernel<SRC_BLOCKKEYS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(score_units_kernel<SRC_POOL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmem);
+  const void* score_kernels[] = {
+      (const void*)score_units_kernel<SRC_FLAT, false>, (const void*)score_units_kernel<SRC_FLAT, true>,
+      (const void*)score_units_kernel<SRC_BLOCKKEYS, false>, (const void*)score_units_kernel<SRC_POOL, false>,
+      (const void*)score_units_kernel<SRC_POOL, true>};
+  for (const void* k : score_kernels)
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmemMax);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(topk_kernel<SRC_BLOCKKEYS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess)
@@ -673,17 +719,24 @@ cudaError_t launch_score(int src, const CacheView& c, const uint16_t* idx_q, con
   int64_t per_query = nq > 0 ? ((int64_t)2 * sms) / nq : 1;   // CTAs per query that fit in one wave
   if (per_query < 1) per_query = 1;
   int64_t upc = (max_units + per_query - 1) / per_query;
-  upc = (upc + kStageUnits - 1) / kStageUnits * kStageUnits;
+  const bool f8 = c.idxk_fp8 && src != SRC_BLOCKKEYS;
+  const int stage_units = f8 ? ScoreGeom<true>::kUnits : ScoreGeom<false>::kUnits;
+  const uint32_t smem = f8 ? ScoreGeom<true>::kSmem : ScoreGeom<false>::kSmem;
+  upc = (upc + stage_units - 1) / stage_units * stage_units;
   if (upc > kUnitsPerCta) upc = kUnitsPerCta;
-  if (upc < kStageUnits) upc = kStageUnits;
+  if (upc < stage_units) upc = stage_units;
   dim3 grid((unsigned)((max_units + upc - 1) / upc), (unsigned)nq);
   if (grid.x == 0) return cudaSuccess;
-  if (src == SRC_FLAT)
-    score_units_kernel<SRC_FLAT><<<grid, kScoreThreads, kScoreSmem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores);
-  else if (src == SRC_BLOCKKEYS)
-    score_units_kernel<SRC_BLOCKKEYS><<<grid, kScoreThreads, kScoreSmem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores);
+  if (src == SRC_BLOCKKEYS)
+    score_units_kernel<SRC_BLOCKKEYS, false><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores);
+  else if (src == SRC_FLAT && f8)
+    score_units_kernel<SRC_FLAT, true><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores);
+  else if (src == SRC_FLAT)
+    score_units_kernel<SRC_FLAT, false><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores);
+  else if (f8)
+    score_units_kernel<SRC_POOL, true><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores);
   else
-    score_units_kernel<SRC_POOL><<<grid, kScoreThreads, kScoreSmem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores);
+    score_units_kernel<SRC_POOL, false><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores);
   return cudaGetLastError();
 }
 

@@ -122,6 +122,23 @@ __device__ __forceinline__ uint32_t idxk_src_warp(int lane, const uint16_t* __re
   return kw;
 }
 
+// One warp: store an indexer key (lane holds dims 2 lane, 2 lane + 1 as bf16)
+// as FP8 at slot `slot` of an FP8 key page: scale s = fl32(amax / 448), codes
+// = E4M3(fl32(k / s)) rounded to nearest even with saturation at 448.
+__device__ __forceinline__ void store_idxk_fp8(uint8_t* page, int slot, int lane, uint32_t kw) {
+  const float a = bf16_lo(kw), b = bf16_hi(kw);
+  float amax = fmaxf(fabsf(a), fabsf(b));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float s = __fdiv_rn(amax, 448.0f);
+  uint16_t code = 0;
+  if (s != 0.0f)
+    code = (uint16_t)__nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(a, s), __fdiv_rn(b, s)), __NV_SATFINITE,
+                                              __NV_E4M3);
+  reinterpret_cast<uint16_t*>(page + slot * kIdx8RowBytes)[lane] = code;
+  if (lane == 0) reinterpret_cast<float*>(page + kIdx8ScaleOff)[slot] = s;
+}
+
 // Slot of position pos of sequence seq in the sliding-window store.
 __device__ __forceinline__ uint8_t* swa_row(const CacheView& c, int seq, int64_t pos) {
   return c.swa + ((int64_t)seq * kReplay + (pos & (kReplay - 1))) * kRowBytes;
@@ -139,12 +156,17 @@ __device__ __forceinline__ void encode_entry_warp(const CacheView& c, int lane, 
   store_row_warp(c.kv + page * kPageBytes + (pos & (kPageTokens - 1)) * kRowBytes, lane, g);
   if (c.swa && pos >= len - kReplay) store_row_warp(swa_row(c, seq, pos), lane, g);
   const uint32_t kw = idxk_src_warp(lane, idxk_src, compress);
-  uint8_t* krow = c.idxk + page * kIdxPageBytes + (pos & (kPageTokens - 1)) * kIdxRowBytes;
-  reinterpret_cast<uint32_t*>(krow)[lane] = kw;
+  if (c.idxk_fp8) {
+    store_idxk_fp8(c.idxk + page * kIdx8PageBytes, (int)(pos & (kPageTokens - 1)), lane, kw);
+  } else {
+    uint8_t* krow = c.idxk + page * kIdxPageBytes + (pos & (kPageTokens - 1)) * kIdxRowBytes;
+    reinterpret_cast<uint32_t*>(krow)[lane] = kw;
+  }
 }
 
 // One warp: recompute the block key of block `blk` of sequence `seq` from the
-// stored keys of its present tokens [8*blk, min(8*blk+8, len)).
+// stored keys of its present tokens [8*blk, min(8*blk+8, len)) (FP8 keys
+// through their dequantised values fl32(s x code)).
 __device__ __forceinline__ void block_key_warp(const CacheView& c, int lane, int seq, int64_t blk,
                                                int64_t len) {
   const int64_t t0 = blk * kBlock;
@@ -152,12 +174,24 @@ __device__ __forceinline__ void block_key_warp(const CacheView& c, int lane, int
   const int64_t page = page_of(c, seq, t0);
   if (page < 0) return;
   const int64_t t1 = min(t0 + kBlock, len);
-  const uint8_t* kp = c.idxk + page * kIdxPageBytes;
   float a = 0.0f, b = 0.0f;
-  for (int64_t t = t0; t < t1; ++t) {
-    const uint32_t w = reinterpret_cast<const uint32_t*>(kp + (t & (kPageTokens - 1)) * kIdxRowBytes)[lane];
-    a = __fadd_rn(a, bf16_lo(w));
-    b = __fadd_rn(b, bf16_hi(w));
+  if (c.idxk_fp8) {
+    const uint8_t* kp = c.idxk + page * kIdx8PageBytes;
+    for (int64_t t = t0; t < t1; ++t) {
+      const int slot = (int)(t & (kPageTokens - 1));
+      const uint32_t cw = reinterpret_cast<const uint16_t*>(kp + slot * kIdx8RowBytes)[lane];
+      const float s = reinterpret_cast<const float*>(kp + kIdx8ScaleOff)[slot];
+      const float2 v = e4m3x2_to_float2(cw);
+      a = __fadd_rn(a, __fmul_rn(s, v.x));
+      b = __fadd_rn(b, __fmul_rn(s, v.y));
+    }
+  } else {
+    const uint8_t* kp = c.idxk + page * kIdxPageBytes;
+    for (int64_t t = t0; t < t1; ++t) {
+      const uint32_t w = reinterpret_cast<const uint32_t*>(kp + (t & (kPageTokens - 1)) * kIdxRowBytes)[lane];
+      a = __fadd_rn(a, bf16_lo(w));
+      b = __fadd_rn(b, bf16_hi(w));
+    }
   }
   const float n = (float)(t1 - t0);
   const uint32_t out = (uint32_t)f32_to_bf16_rne(__fdiv_rn(a, n)) |

@@ -25,12 +25,14 @@ def _pages(n_entries: int) -> int:
     return (n_entries + csa2.PAGE_TOKENS - 1) // csa2.PAGE_TOKENS
 
 
-def new_cache(w: wl.Workload, lengths=None, cache_id: int = 1, swa_store: bool = False) -> csa2.Cache:
+def new_cache(w: wl.Workload, lengths=None, cache_id: int = 1, swa_store: bool = False,
+              idxk_format: int = csa2.IDXK_BF16) -> csa2.Cache:
     lens = list(lengths if lengths is not None else w.lengths)
     pages = [_pages(L) for L in lens]
     max_pages = max(pages)
     pt = wl.page_table(w.seed, w.n_pages_pool, pages, max_pages)
-    cache = csa2.Cache(w.n_pages_pool, len(lens), max_pages, cache_id=cache_id, swa_store=swa_store)
+    cache = csa2.Cache(w.n_pages_pool, len(lens), max_pages, cache_id=cache_id, swa_store=swa_store,
+                       idxk_format=idxk_format)
     cache.page_table.copy_(torch.from_numpy(pt))
     cache.seq_lens.copy_(torch.tensor(lens, dtype=torch.int32))
     return cache

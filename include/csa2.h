@@ -35,7 +35,10 @@
  *                  Row = 256 B of E2M1 codes (channel 2j in the low nibble of
  *                  byte j, channel 2j+1 in the high nibble) followed by 32 E4M3
  *                  scale bytes (scale g covers channels 16g..16g+15).
- * - idxk_pool:     page p holds 64 indexer keys, bf16 [64][64], 8192 B/page.
+ * - idxk_pool:     page p holds 64 indexer keys.  CSA2_IDXK_BF16: bf16
+ *                  [64][64], 8192 B/page.  CSA2_IDXK_FP8: E4M3 codes
+ *                  [64][64] (byte d = dimension d) followed by the 64 fp32
+ *                  scales, 4352 B/page; key = scale x code.
  * - blockkey_pool: page p holds the 8 block keys of its 8-token blocks,
  *                  bf16 [8][64], 1024 B/page.
  * - page_table[b*max_pages + i] = page id of tokens 64i..64i+63 of sequence b.
@@ -65,6 +68,8 @@ typedef struct CUstream_st* csa2_stream_t; /* == cudaStream_t */
 #define CSA2_TOP_K 512            /* indices selected per query                     */
 #define CSA2_WINDOW 128           /* sliding-window length                          */
 #define CSA2_REPLAY 128           /* tokens recomputed by bounded replay            */
+#define CSA2_IDXK_BF16 0          /* indexer keys stored as bf16, 128 B per token   */
+#define CSA2_IDXK_FP8 1           /* 64 E4M3 codes + one fp32 scale, 68 B per token */
 
 typedef enum {
   CSA2_OK = 0,
@@ -90,7 +95,8 @@ typedef enum { CSA2_OP_INDEXER = 1, CSA2_OP_ATTENTION = 2 } csa2_op;
 /* Paged cache; every pointer is device memory owned by the caller. */
 typedef struct {
   void* kv_pool;              /* n_pages * 18432 B, 16-B aligned               */
-  void* idxk_pool;            /* n_pages * 8192 B, 16-B aligned                */
+  void* idxk_pool;            /* n_pages * 8192 B (bf16 keys) or * 4352 B (FP8
+                                 keys), 16-B aligned                           */
   void* blockkey_pool;        /* n_pages * 1024 B, 16-B aligned                */
   int64_t n_pages;            /* 1 .. 2^25 (attention names rows by 31 bits)   */
   const int32_t* page_table;  /* int32 [batch][max_pages]                      */
@@ -103,6 +109,7 @@ typedef struct {
                                  none (the window is read from kv_pool); else
                                  [batch][128][288 B] FP4 rows, 16-B aligned,
                                  position p of sequence b in slot p % 128      */
+  int32_t idxk_format;        /* CSA2_IDXK_BF16 (0) or CSA2_IDXK_FP8           */
 } csa2_cache;
 
 /* Index sets produced by the indexer and consumed by attention.  Device
@@ -157,9 +164,13 @@ void csa2_indexset_attach_rows(csa2_indexset* set, int32_t* attn_rows);
  * saturating at 448); code = sign | E2M1 nearest to |x|/scale (ties to even,
  * saturating at 6); a zero scale stores code 0.  The entry is written at
  * position entry_pos[i] of sequence entry_seq[i] (both int32 [n]); the
- * indexer key is stored as bf16; the block key of every touched 8-token block
- * is recomputed as bf16(fp32 mean of the block's present keys, ascending
- * order).  seq_lens must already count the new entries (entry_pos[i] <
+ * indexer key is stored as bf16 (the fp32 pair mean rounded to nearest even
+ * at ratio 2).  With CSA2_IDXK_FP8 that bf16 key k is stored quantised:
+ * scale s = fl32(max_d |k_d| / 448), code_d = E4M3 nearest to fl32(k_d / s)
+ * (ties to even, saturating at 448, sign kept), s == 0 stores zero codes; its
+ * dequantised value is fl32(s x code).  The block key of every touched
+ * 8-token block is recomputed as bf16(fp32 mean of the block's present
+ * (dequantised) keys, ascending order).  seq_lens must already count the new entries (entry_pos[i] <
  * seq_lens[seq]).  kv and idxk must be 16-B aligned.  With a sliding-window
  * store (cache->swa_rows), entries among their sequence's last 128 positions
  * are also written to their slot there.
@@ -180,7 +191,8 @@ int csa2_kv_quant_append(const csa2_cache* cache, const uint16_t* kv, const uint
  * q_seq[r] and visible length q_visible[r] (or seq_lens[q_seq[r]] if
  * q_visible == NULL); max_visible >= every visible length (host-known bound
  * that sizes the grid and the workspace); nq <= 65535.
- * score(q, k) = sum_h w_h * max(0, q_h . k) in fp32.
+ * score(q, k) = sum_h w_h * max(0, q_h . k) in fp32; an FP8 key scores
+ * s x score(q, code values).  Block keys are bf16 in both formats.
  *  - CSA2_FULL, hierarchical != 0 (decoder): if ceil(v/8) > 2048 the 2,048
  *    best block keys form the pool, else every block does; writes
  *    set->pool_blocks[r] and the 512 best pool tokens to set->idx[r].

@@ -32,6 +32,19 @@ def cache_keys(cache, seq: int, positions) -> np.ndarray:
     return cache.idxk_pool[idx].cpu().numpy().view(np.uint16).reshape(-1, 64)
 
 
+def cache_keys_fp8(cache, seq: int, positions) -> tuple[np.ndarray, np.ndarray]:
+    """(E4M3 codes [n, 64], fp32 scales [n]) of the given positions of an FP8 key cache."""
+    pt = cache.page_table[seq].cpu().numpy()
+    pos = np.asarray(positions, dtype=np.int64)
+    pages = pt[pos >> 6].astype(np.int64)
+    cidx = (pages * 4352 + (pos & 63) * 64)[:, None] + np.arange(64)[None, :]
+    sidx = (pages * 4352 + 4096 + (pos & 63) * 4)[:, None] + np.arange(4)[None, :]
+    pool = cache.idxk_pool
+    codes = pool[torch.from_numpy(cidx).cuda()].cpu().numpy()
+    scales = pool[torch.from_numpy(sidx).cuda()].cpu().numpy().copy().view(np.float32).reshape(-1)
+    return codes, scales
+
+
 def cache_block_keys(cache, seq: int, blocks) -> np.ndarray:
     pt = cache.page_table[seq].cpu().numpy()
     blk = np.asarray(blocks, dtype=np.int64)

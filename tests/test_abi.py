@@ -174,3 +174,14 @@ def test_replay_and_cache_argument_checks(csa2_lib):
     # attention names rows by 31-bit ids: the pool and batch limits
     assert rep(_cache(csa2_lib, f, n_pages=(1 << 25) + 1), f.p(), f.p(), f.p(), 1) == 2
     assert rep(_cache(csa2_lib, f, batch=(1 << 23) + 1), f.p(), f.p(), f.p(), 1) == 2
+
+
+def test_indexer_key_format_is_checked(csa2_lib):
+    L = csa2_lib.lib()
+    f = _Fake()
+    B = ctypes.byref
+    rep = lambda cache: L.csa2_swa_replay(B(cache), f.p(), f.p(), f.p(), 1, None)
+    assert rep(_cache(csa2_lib, f, idxk_format=2)) == 1
+    assert rep(_cache(csa2_lib, f, idxk_format=-1)) == 1
+    assert L.csa2_kv_quant_append(B(_cache(csa2_lib, f, idxk_format=7)), f.p(), f.p(), f.p(), f.p(), 1, 1,
+                                  None) == 1
