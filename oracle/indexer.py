@@ -25,6 +25,12 @@ Readings taken where the pages are silent:
   wins a tie); fewer candidates than k -> all of them, padded with -1; the
   output set is listed in ascending position order;
 * Reindex ranks the tokens of the pool that the Full layer built.
+* block score: the pages do not give it.  Default ("mean"): the score of the
+  block key (mean-pooled keys) -- a real hierarchy that reads L/8 keys.
+  Alternative ("max"): the largest score of the block's present tokens.  It
+  reads every key, and it is lossless: a token of the flat top-k lies in a
+  block that fewer than pool_blocks blocks can beat (each of those holds a
+  token that beats it), so the pool's top-k equals the flat top-k.
 
 Keys are bf16 bit patterns [n, 64] or FP8 keys (oracle.idxk_fp8.Fp8Keys):
 an FP8 key's score is its scale times the score of its code values, and
@@ -125,15 +131,35 @@ def select_tokens(q_bits, key_bits, candidates: np.ndarray, w=None, k: int = TOP
     return out, s
 
 
+def block_max_scores(q_bits, key_bits, length: int, w=None, block: int = BLOCK) -> np.ndarray:
+    """Max-pooled block scores [ceil(L/block)]: the largest token score of each block."""
+    keys = key_bits if isinstance(key_bits, Fp8Keys) else np.asarray(key_bits)
+    ts = index_scores(q_bits, keys[:length], w)
+    nb = (length + block - 1) // block
+    out = np.full(nb, -np.inf, dtype=np.float32)
+    for t in range(block):                       # each block's present tokens
+        rows = np.arange(nb) * block + t
+        present = rows < length
+        out[present] = np.maximum(out[present], ts[rows[present]])
+    return out
+
+
 def full_indexer(q_bits, key_bits, length: int, w=None, hierarchical: bool = True,
-                 pool_blocks: int = POOL_BLOCKS, block: int = BLOCK, k: int = TOP_K):
+                 pool_blocks: int = POOL_BLOCKS, block: int = BLOCK, k: int = TOP_K,
+                 pooling: str = "mean"):
     """Full layer: returns (pool block ids [pool_blocks] ascending, -1 padded;
-    selected positions [k] ascending, -1 padded; info dict)."""
+    selected positions [k] ascending, -1 padded; info dict).  pooling: the
+    block score of the hierarchy, "mean" (block keys) or "max" (token scores)."""
     nb = (length + block - 1) // block
     info = {}
     if hierarchical and nb > pool_blocks:
-        kb = block_keys(key_bits, length, block)
-        bs = index_scores(q_bits, kb, w)
+        if pooling == "mean":
+            kb = block_keys(key_bits, length, block)
+            bs = index_scores(q_bits, kb, w)
+        elif pooling == "max":
+            bs = block_max_scores(q_bits, key_bits, length, w, block)
+        else:
+            raise ValueError(pooling)
         pool = top_k(bs, np.ones(nb, dtype=bool), pool_blocks)
         info["block_scores"] = bs
     else:

@@ -167,3 +167,52 @@ def test_reindex_with_full_query_reproduces_full_set():
     other, info = indexer.reindex_indexer(q2, k, L, pool)
     assert set(other.tolist()) <= set(info["candidates"].tolist())
     assert not np.array_equal(other, idx)
+
+
+def _keys_of(kind, rng, L):
+    if kind == "random":
+        return _bf16(rng.standard_normal((L, 64)))
+    if kind == "zero":
+        return np.zeros((L, 64), np.uint16)
+    base = _bf16(rng.standard_normal((5, 64)))          # few distinct keys: heavy ties
+    return base[rng.integers(0, 5, L)]
+
+
+@pytest.mark.parametrize("kind", ["random", "zero", "few"])
+@pytest.mark.parametrize("L", [20000, 16391, 40960])
+def test_max_pooled_hierarchy_is_lossless(kind, L):
+    """With max-pooled block scores the pool's top-512 equals the flat top-512
+    (the block-beating argument), ties included."""
+    rng = np.random.default_rng(L)
+    k = _keys_of(kind, rng, L)
+    q = _bf16(rng.standard_normal((4, 64)))
+    w = np.array([1.0, -0.5, 2.0, 0.25], np.float32)
+    pool, idx, info = indexer.full_indexer(q, k, L, w, pooling="max")
+    _, flat, _ = indexer.full_indexer(q, k, L, w, hierarchical=False)
+    np.testing.assert_array_equal(idx, flat)
+    assert pool[pool >= 0].size == 2048 and np.all(np.diff(pool[pool >= 0]) > 0)
+    # the pool is the top-2048 of the block maxima, computed here by brute force
+    ts = indexer.index_scores(q, k, w).astype(np.float64)
+    nb = (L + 7) // 8
+    bmax = np.array([ts[8 * b: min(8 * b + 8, L)].max() for b in range(nb)])
+    order = sorted(range(nb), key=lambda b: (-bmax[b], b))[:2048]
+    np.testing.assert_array_equal(pool[pool >= 0], np.sort(order))
+
+
+def test_max_pooled_hierarchy_brute_force_on_shrunken_sizes():
+    """Pools of 3 blocks of 4 tokens and k = 2: every pool and selection by loops."""
+    rng = np.random.default_rng(9)
+    for trial in range(40):
+        L = int(rng.integers(13, 40))
+        k = _bf16(rng.integers(-3, 4, (L, 64)).astype(np.float32))   # small integers: many ties
+        q = _bf16(rng.integers(-2, 3, (4, 64)).astype(np.float32))
+        pool, idx, _ = indexer.full_indexer(q, k, L, pool_blocks=3, block=4, k=2, pooling="max")
+        ts = [float(indexer.index_scores(q, k[i:i + 1])[0]) for i in range(L)]
+        blocks = [(-max(ts[4 * b: min(4 * b + 4, L)]), b) for b in range((L + 3) // 4)]
+        want_pool = sorted(b for _, b in sorted(blocks)[:3])
+        assert list(pool[pool >= 0]) == want_pool
+        cand = [t for b in want_pool for t in range(4 * b, min(4 * b + 4, L))]
+        want = sorted(sorted(cand, key=lambda t: (-ts[t], t))[:2])
+        assert list(idx[idx >= 0]) == want
+        flat = sorted(sorted(range(L), key=lambda t: (-ts[t], t))[:2])
+        assert want == flat
