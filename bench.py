@@ -369,6 +369,7 @@ def run_gpu(args):
         "clocks": clocks,
     }
     result["window_store"] = measure_window_store(w, cache, step, stream, flush, peaks, reuse_ms)
+    result["max_pooled_blocks"] = measure_max_pool(w, cache, step, stream, flush, peaks, idx_full_ms)
     result["fp8_indexer_keys"] = measure_fp8_keys(
         w, stream, flush, peaks, {"step": ms_per_step, "full": idx_full_ms, "reindex": idx_ri_ms})
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -460,6 +461,41 @@ def measure_window_store(w, cache, step, stream, flush, peaks, attn_global_ms):
         "note": "CUDA graphs of one call (replay) or 2 x 3 Reuse calls (attention), L2 flushed first; "
                 "bytes: bf16 rows read + FP4 rows (and keys) written",
     }
+
+
+def measure_max_pool(w, cache, step, stream, flush, peaks, mean_full_ms):
+    """The Full indexer with max-pooled block scores on the bench batch, outside the
+    timed region: it scores every key (the flat score kernel also writing each
+    block's maximum), then selects the pool and the tokens.  Also the recall of the
+    mean-pooled hierarchy: the share of the exact top-512 (= the max-pooled one)
+    that the step's mean-pooled Full layer selects."""
+    import torch
+
+    from fp4_kv_cache_decode_b200 import csa2
+    f_layer = w.layers.index("F")
+    iset = csa2.IndexSet(step.nq, row_cache=False)
+    ws = torch.empty(csa2.csa2_workspace_bytes(csa2.OP_INDEXER, step.nq, 0, step.max_visible, csa2.HIER_MAX),
+                     dtype=torch.uint8, device="cuda")
+
+    def full_max():
+        csa2.csa2_indexer_score_topk(cache, step.idxq[f_layer], step.q_seq, csa2.FULL, f_layer, iset, ws,
+                                     step.max_visible, hierarchical=csa2.HIER_MAX)
+    ms = _graph_ms(full_max, flush, stream)
+    mean_set = csa2.IndexSet(step.nq, row_cache=False)
+    csa2.csa2_indexer_score_topk(cache, step.idxq[f_layer], step.q_seq, csa2.FULL, f_layer, mean_set,
+                                 step.ws_idx, step.max_visible, hierarchical=csa2.HIER_MEAN)
+    full_max()
+    torch.cuda.synchronize()
+    assert csa2.csa2_check_device_error(cache) == 0
+    exact, approx = iset.idx.cpu().numpy(), mean_set.idx.cpu().numpy()
+    recall = float(np.mean([np.isin(a[a >= 0], e[e >= 0]).sum() / max(1, (e >= 0).sum())
+                            for e, a in zip(exact, approx)]))
+    key_bytes = sum(w.lengths[s] for s in step.seqs) * 128
+    gbs = key_bytes / (ms * 1e-3) / 1e9
+    return {"indexer_full_ms": ms, "indexer_full_ms_mean_pooled": mean_full_ms,
+            "key_bytes": key_bytes, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
+            "mean_pooled_recall_of_exact_top512": recall,
+            "note": "median of CUDA-graph replays, L2 flushed first; bytes = every visible bf16 key once"}
 
 
 def measure_fp8_keys(w, stream, flush, peaks, bf16_ms):

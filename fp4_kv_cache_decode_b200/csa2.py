@@ -23,6 +23,7 @@ PAGE_BYTES = ROW_BYTES * PAGE_TOKENS
 IDX_PAGE_BYTES = 64 * 128
 IDX8_PAGE_BYTES = 64 * 64 + 64 * 4   # FP8 indexer keys: codes, then fp32 scales
 IDXK_BF16, IDXK_FP8 = 0, 1
+HIER_FLAT, HIER_MEAN, HIER_MAX = 0, 1, 2   # indexer candidate sets (hierarchical argument)
 BK_PAGE_BYTES = 8 * 128
 TOP_K = 512
 POOL_BLOCKS = 2048
@@ -224,7 +225,7 @@ class IndexSet:
 
 def csa2_workspace_bytes(op: int, nq: int, heads: int = 0, max_visible: int = 0,
                          hierarchical: bool = True) -> int:
-    return int(lib().csa2_workspace_bytes(op, nq, heads, max_visible, int(bool(hierarchical))))
+    return int(lib().csa2_workspace_bytes(op, nq, heads, max_visible, int(hierarchical)))
 
 
 def csa2_kv_quant_append(cache: Cache, kv: torch.Tensor, idxk: torch.Tensor, entry_seq: torch.Tensor,
@@ -247,7 +248,7 @@ def csa2_indexer_score_topk(cache: Cache, idx_q: torch.Tensor, q_seq: torch.Tens
     st = lib().csa2_indexer_score_topk(
         cache.ref(), _ptr(idx_q, _BF16, "idx_q", nq * 256),
         _ptr(head_w, (torch.float32,), "head_w", nq * 4), _ptr(q_seq, _I32T, "q_seq"),
-        _ptr(q_visible, _I32T, "q_visible", nq), nq, int(max_visible), mode, int(bool(hierarchical)),
+        _ptr(q_visible, _I32T, "q_visible", nq), nq, int(max_visible), mode, int(hierarchical),
         layer, indexset.ref(), _ptr(workspace, (torch.uint8,), "workspace"),
         workspace.numel(), _stream(stream))
     _check(st, "csa2_indexer_score_topk")
@@ -268,7 +269,7 @@ def csa2_indexer_score_topk_noalloc(cache: Cache, idx_q: torch.Tensor, q_seq: to
     st = lib().csa2_indexer_score_topk_noalloc(
         cache.ref(), _ptr(idx_q, _BF16, "idx_q", nq * 256),
         _ptr(head_w, (torch.float32,), "head_w", nq * 4), _ptr(q_seq, _I32T, "q_seq"),
-        _ptr(q_visible, _I32T, "q_visible", nq), nq, int(max_visible), mode, int(bool(hierarchical)),
+        _ptr(q_visible, _I32T, "q_visible", nq), nq, int(max_visible), mode, int(hierarchical),
         layer, indexset.ref(), _stream(stream))
     _check(st, "csa2_indexer_score_topk_noalloc")
 

@@ -13,7 +13,8 @@ cudaError_t launch_append(const CacheView&, const uint16_t*, const uint16_t*, co
 cudaError_t launch_replay(const CacheView&, const uint16_t*, const uint16_t*, const uint8_t*,
                           int, cudaStream_t);
 cudaError_t launch_score(int, const CacheView&, const uint16_t*, const float*, const int32_t*,
-                         const int32_t*, const int32_t*, int, int64_t, int64_t, float*, cudaStream_t);
+                         const int32_t*, const int32_t*, int, int64_t, int64_t, float*, float*, int64_t,
+                         cudaStream_t);
 cudaError_t launch_topk(int, const CacheView&, const float*, int64_t, const int32_t*, const int32_t*,
                         const int32_t*, int, int, int32_t*, int64_t, cudaStream_t);
 cudaError_t indexer_set_attributes();
@@ -82,8 +83,15 @@ int from_cuda(cudaError_t e) { return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Score-buffer stride (floats per query) of an indexer call.
+// Per-query floats of the indexer workspace: token (or block-key) scores, then,
+// for a max-pooled Full call, the block maxima at offset nq * flat stride.
+int64_t max_pool_block_stride(int64_t max_visible) {
+  return ceil_div(ceil_div(max_visible, kBlock), kBlocksPerPage) * kBlocksPerPage;
+}
+
 int64_t indexer_stride(int64_t max_visible, int hierarchical) {
   const int64_t nb = ceil_div(max_visible, kBlock);
+  if (hierarchical == CSA2_HIER_MAX) return nb * kBlock;
   if (hierarchical) {
     const int64_t bk = ceil_div(nb, kBlocksPerPage) * kBlocksPerPage;
     const int64_t pool = (int64_t)kPoolBlocks * kBlock;
@@ -145,8 +153,11 @@ int csa2_indexer_score_topk(const csa2_cache* cache, const uint16_t* idx_q, cons
   if (nq < 0 || max_visible < 0 || max_visible > ((int64_t)1 << 31) - 1 || layer < 0)
     return CSA2_ERR_INVALID_ARG;
   if (!set || !set->idx) return CSA2_ERR_INVALID_ARG;
+  if (hierarchical < CSA2_HIER_FLAT || hierarchical > CSA2_HIER_MAX) return CSA2_ERR_INVALID_ARG;
   if (nq > set->rows || nq > kMaxQueries) return CSA2_ERR_SHAPE;
   const bool hier = hierarchical != 0 || mode == CSA2_REINDEX;
+  // the workspace layout this call uses (Reindex: pool scores)
+  const int ws_kind = mode == CSA2_REINDEX ? CSA2_HIER_MEAN : hierarchical;
   if (hier && !set->pool_blocks) return CSA2_ERR_INVALID_ARG;
   if (mode == CSA2_REINDEX) {
     // Reindex ranks the pool of the last hierarchical Full layer on this cache
@@ -158,34 +169,47 @@ int csa2_indexer_score_topk(const csa2_cache* cache, const uint16_t* idx_q, cons
   if (!aligned(idx_q, 16) || !aligned(head_w, 4) || !aligned(q_seq, 4) || !aligned(q_visible, 4) ||
       !aligned(set->idx, 4) || !aligned(set->pool_blocks, 4))
     return CSA2_ERR_ALIGNMENT;
-  const size_t need = csa2_workspace_bytes(CSA2_OP_INDEXER, nq, 0, max_visible, hier ? 1 : 0);
+  const size_t need = csa2_workspace_bytes(CSA2_OP_INDEXER, nq, 0, max_visible, ws_kind);
   if (nq > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16)))
     return CSA2_ERR_WORKSPACE;
   if (nq > 0) {
     if ((st = ensure_device_setup())) return st;
     cudaStream_t s = (cudaStream_t)stream;
     float* scores = static_cast<float*>(workspace);
-    const int64_t stride = indexer_stride(max_visible, hier ? 1 : 0);
+    const int64_t stride = indexer_stride(max_visible, ws_kind);
     const int64_t nb = ceil_div(max_visible, kBlock);
     cudaError_t e = cudaSuccess;
-    if (mode == CSA2_FULL && hier) {
+    if (mode == CSA2_FULL && hierarchical == CSA2_HIER_MAX) {
+      // every token scored once; the score kernel also writes each block's
+      // maximum; the pool is the 2,048 best maxima, the tokens the flat top-512
+      float* bmax = scores + (int64_t)nq * stride;
+      const int64_t bstride = max_pool_block_stride(max_visible);
+      e = launch_score(kSrcFlat, v, idx_q, head_w, q_seq, q_visible, nullptr, nq, nb, stride, scores,
+                       bmax, bstride, s);
+      if (e == cudaSuccess)
+        e = launch_topk(kSrcBlockKeys, v, bmax, bstride, q_seq, q_visible, nullptr, nq, kPoolBlocks,
+                        set->pool_blocks, kPoolBlocks, s);
+      if (e == cudaSuccess)
+        e = launch_topk(kSrcFlat, v, scores, stride, q_seq, q_visible, nullptr, nq, kTopK, set->idx,
+                        kTopK, s);
+    } else if (mode == CSA2_FULL && hier) {
       const int64_t bk_units = ceil_div(nb, kBlocksPerPage);
       e = launch_score(kSrcBlockKeys, v, idx_q, head_w, q_seq, q_visible, nullptr, nq, bk_units,
-                       stride, scores, s);
+                       stride, scores, nullptr, 0, s);
       if (e == cudaSuccess)
         e = launch_topk(kSrcBlockKeys, v, scores, stride, q_seq, q_visible, nullptr, nq,
                         kPoolBlocks, set->pool_blocks, kPoolBlocks, s);
     }
-    if (e == cudaSuccess && hier) {
+    if (e == cudaSuccess && hier && !(mode == CSA2_FULL && hierarchical == CSA2_HIER_MAX)) {
       e = launch_score(kSrcPool, v, idx_q, head_w, q_seq, q_visible, set->pool_blocks, nq,
-                       kPoolBlocks, stride, scores, s);
+                       kPoolBlocks, stride, scores, nullptr, 0, s);
       if (e == cudaSuccess)
         e = launch_topk(kSrcPool, v, scores, stride, q_seq, q_visible, set->pool_blocks, nq, kTopK,
                         set->idx, kTopK, s);
     }
     if (e == cudaSuccess && !hier) {
       e = launch_score(kSrcFlat, v, idx_q, head_w, q_seq, q_visible, nullptr, nq, nb, stride,
-                       scores, s);
+                       scores, nullptr, 0, s);
       if (e == cudaSuccess)
         e = launch_topk(kSrcFlat, v, scores, stride, q_seq, q_visible, nullptr, nq, kTopK, set->idx,
                         kTopK, s);
@@ -269,7 +293,10 @@ size_t csa2_workspace_bytes(int32_t op, int32_t nq, int32_t heads, int64_t max_v
   if (nq < 0) return 0;
   if (op == CSA2_OP_INDEXER) {
     if (max_visible < 0) return 0;
-    return (size_t)nq * (size_t)indexer_stride(max_visible, hierarchical ? 1 : 0) * sizeof(float) + 256;
+    if (hierarchical < CSA2_HIER_FLAT || hierarchical > CSA2_HIER_MAX) return 0;
+    int64_t per_query = indexer_stride(max_visible, hierarchical);
+    if (hierarchical == CSA2_HIER_MAX) per_query += max_pool_block_stride(max_visible);
+    return (size_t)nq * (size_t)per_query * sizeof(float) + 256;
   }
   if (op == CSA2_OP_ATTENTION) {
     if (heads != 16 && heads != 32 && heads != 48 && heads != 64) return 0;

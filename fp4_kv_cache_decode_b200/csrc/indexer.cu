@@ -84,7 +84,9 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView
                                                                        const int32_t* __restrict__ q_vis,
                                                                        const int32_t* __restrict__ pool,
                                                                        int64_t max_units, int64_t stride,
-                                                                       int upc, float* __restrict__ scores) {
+                                                                       int upc, float* __restrict__ scores,
+                                                                       float* __restrict__ block_max,
+                                                                       int64_t bstride) {
   extern __shared__ __align__(16) uint8_t stage[];
   static_assert(!F8 || SRC != SRC_BLOCKKEYS, "block keys are bf16");
   __shared__ const uint8_t* ubase[kUnitsPerCta];
@@ -250,8 +252,20 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView
       sc += __shfl_xor_sync(0xffffffffu, sc, 1);
       sc += __shfl_xor_sync(0xffffffffu, sc, 2);
       if (F8) sc *= srow;
-      if (j < nu && (lane & 3) == 0)
-        scores[(int64_t)r * stride + u * kBlock + row] = row < urows[j] ? sc : -INFINITY;
+      const float val = row < urows[j] ? sc : -INFINITY;
+      if (j < nu && (lane & 3) == 0) scores[(int64_t)r * stride + u * kBlock + row] = val;
+      if (SRC == SRC_FLAT && block_max != nullptr) {   // max-pooled block score of block u
+        float m = fmaxf(val, __shfl_xor_sync(0xffffffffu, val, 4));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+        float* brow = block_max + (int64_t)r * bstride;
+        if (j < nu && lane == 0) brow[u] = m;
+        // the last block's CTA pads the row to a whole 8-block unit with -inf
+        if (j < nu && u == nunits - 1 && lane < kBlocksPerPage) {
+          const int64_t pad = nunits + lane;
+          if (pad < (nunits + kBlocksPerPage - 1) / kBlocksPerPage * kBlocksPerPage) brow[pad] = -INFINITY;
+        }
+      }
     }
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
@@ -711,7 +725,8 @@ cudaError_t indexer_set_attributes() {
 // Scores of every query's units into `scores` (row stride `stride` floats).
 cudaError_t launch_score(int src, const CacheView& c, const uint16_t* idx_q, const float* head_w,
                          const int32_t* q_seq, const int32_t* q_vis, const int32_t* pool, int nq,
-                         int64_t max_units, int64_t stride, float* scores, cudaStream_t st) {
+                         int64_t max_units, int64_t stride, float* scores, float* block_max,
+                         int64_t bstride, cudaStream_t st) {
   // units per CTA: enough CTAs for two per SM over the whole batch, in whole
   // 32-unit stages, at most 256
   int sms = 148, dev = 0;
@@ -728,15 +743,15 @@ cudaError_t launch_score(int src, const CacheView& c, const uint16_t* idx_q, con
   dim3 grid((unsigned)((max_units + upc - 1) / upc), (unsigned)nq);
   if (grid.x == 0) return cudaSuccess;
   if (src == SRC_BLOCKKEYS)
-    score_units_kernel<SRC_BLOCKKEYS, false><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores);
+    score_units_kernel<SRC_BLOCKKEYS, false><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
   else if (src == SRC_FLAT && f8)
-    score_units_kernel<SRC_FLAT, true><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores);
+    score_units_kernel<SRC_FLAT, true><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
   else if (src == SRC_FLAT)
-    score_units_kernel<SRC_FLAT, false><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores);
+    score_units_kernel<SRC_FLAT, false><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
   else if (f8)
-    score_units_kernel<SRC_POOL, true><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores);
+    score_units_kernel<SRC_POOL, true><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
   else
-    score_units_kernel<SRC_POOL, false><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores);
+    score_units_kernel<SRC_POOL, false><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
   return cudaGetLastError();
 }
 

@@ -62,7 +62,7 @@ extern "C" int csa2_indexer_score_topk_noalloc(const csa2_cache* cache, const ui
                                                int32_t hierarchical, int32_t layer,
                                                csa2_indexset* set, csa2_stream_t stream) {
   if (nq < 0 || max_visible < 0) return CSA2_ERR_INVALID_ARG;
-  const int32_t hier = (hierarchical != 0 || mode == CSA2_REINDEX) ? 1 : 0;
+  const int32_t hier = mode == CSA2_REINDEX ? CSA2_HIER_MEAN : hierarchical;
   const size_t need = csa2_workspace_bytes(CSA2_OP_INDEXER, nq, 0, max_visible, hier);
   if (need > (size_t)CSA2_NOALLOC_SCRATCH_BYTES) return CSA2_ERR_WORKSPACE;
   void* scratch = nullptr;

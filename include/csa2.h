@@ -68,6 +68,9 @@ typedef struct CUstream_st* csa2_stream_t; /* == cudaStream_t */
 #define CSA2_TOP_K 512            /* indices selected per query                     */
 #define CSA2_WINDOW 128           /* sliding-window length                          */
 #define CSA2_REPLAY 128           /* tokens recomputed by bounded replay            */
+#define CSA2_HIER_FLAT 0          /* indexer: every visible entry is a candidate    */
+#define CSA2_HIER_MEAN 1          /* pool of 2,048 blocks by mean-pooled block keys  */
+#define CSA2_HIER_MAX 2           /* pool by the largest token score of each block   */
 #define CSA2_IDXK_BF16 0          /* indexer keys stored as bf16, 128 B per token   */
 #define CSA2_IDXK_FP8 1           /* 64 E4M3 codes + one fp32 scale, 68 B per token */
 
@@ -193,10 +196,16 @@ int csa2_kv_quant_append(const csa2_cache* cache, const uint16_t* kv, const uint
  * that sizes the grid and the workspace); nq <= 65535.
  * score(q, k) = sum_h w_h * max(0, q_h . k) in fp32; an FP8 key scores
  * s x score(q, code values).  Block keys are bf16 in both formats.
- *  - CSA2_FULL, hierarchical != 0 (decoder): if ceil(v/8) > 2048 the 2,048
- *    best block keys form the pool, else every block does; writes
- *    set->pool_blocks[r] and the 512 best pool tokens to set->idx[r].
- *  - CSA2_FULL, hierarchical == 0 (encoder): 512 best of positions [0, v).
+ *  - CSA2_FULL, hierarchical == CSA2_HIER_MEAN (decoder): if ceil(v/8) >
+ *    2048 the 2,048 best block keys form the pool, else every block does;
+ *    writes set->pool_blocks[r] and the 512 best pool tokens to set->idx[r].
+ *  - CSA2_FULL, hierarchical == CSA2_HIER_MAX: the block score is the
+ *    largest score of the block's present tokens (the pages do not fix the
+ *    block score; this reading reads every key and loses nothing: the pool's
+ *    512 best tokens are the 512 best of [0, v), which is how they are
+ *    computed).  Writes the pool and set->idx[r] like CSA2_HIER_MEAN.
+ *  - CSA2_FULL, hierarchical == CSA2_HIER_FLAT (encoder): 512 best of
+ *    positions [0, v); no pool.
  *  - CSA2_REINDEX: 512 best tokens of the pool written by the last
  *    hierarchical Full call on `set` (requires set->pool_layer < layer).
  * Ranking: score descending, then position ascending; output ascending, -1

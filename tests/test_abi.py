@@ -56,6 +56,10 @@ def test_workspace_sizes(csa2_lib):
     assert ws(2, 148, 64, 0, False) == 0
     assert ws(2, 32, 20, 0, False) == 0          # unsupported head count
     assert ws(7, 1, 64, 0, False) == 0
+    # max-pooled hierarchy: every token's score, then the 8,192 block maxima
+    assert ws(1, 32, 0, 65536, 2) == 32 * (65536 + 8192) * 4 + 256
+    assert ws(1, 3, 0, 100, 2) == 3 * (104 + 16) * 4 + 256
+    assert ws(1, 32, 0, 65536, 3) == 0
 
 
 class _Fake:
@@ -150,6 +154,10 @@ def test_mode_order_state_machine(csa2_lib):
     assert idx(FULL, 6, hier=0) == 0
     assert s.pool_layer == -1
     assert idx(REINDEX, 7) == 4
+    # a max-pooled Full call leaves a pool for Reindex; an unknown block score is refused
+    assert idx(FULL, 6, hier=2) == 0 and s.pool_layer == 6
+    assert idx(REINDEX, 7) == 0
+    assert idx(FULL, 8, hier=3) == 1
     # more queries than the set has rows
     assert idx(FULL, 8, nq=3) == 2
     # workspace too small
