@@ -16,6 +16,8 @@ from . import _build
 
 FULL, REINDEX, REUSE = 0, 1, 2
 OP_INDEXER, OP_ATTENTION = 1, 2
+OP_SHARD_INDEXER, OP_SHARD_MERGE, OP_SHARD_ATTENTION = 3, 4, 5
+SHARD_BLOCKS, SHARD_TOKENS = 0, 1
 LATENT_DIM = 512
 ROW_BYTES = 288
 PAGE_TOKENS = 64
@@ -89,6 +91,13 @@ SIGNATURES = {
     "csa2_indexer_score_topk_noalloc": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _I32, _I64, _I32, _I32,
                                                        _I32, _VP, _VP]),
     "csa2_swa_replay": (ctypes.c_int, [_VP, _VP, _VP, _VP, ctypes.c_int32, _VP]),
+    "csa2_shard_indexer_candidates": (ctypes.c_int, [_VP, _VP, _VP, _VP, _VP, _I32, _I64, _I32, _VP, _VP,
+                                                     _VP, _VP, _SZ, _VP]),
+    "csa2_shard_merge_topk": (ctypes.c_int, [_VP, _VP, _I32, _I32, _I32, _I64, _I64, _I32, _VP, _VP, _VP,
+                                             _SZ, _VP]),
+    "csa2_sparse_attn_shard": (ctypes.c_int, [_VP, _VP, _I32, _F32, _VP, _VP, _VP, _VP, _I32, _VP, _VP,
+                                              _VP, _SZ, _VP]),
+    "csa2_shard_combine": (ctypes.c_int, [_VP, _VP, _I32, _I32, _I32, _I64, _I64, _VP, _VP]),
     "csa2_workspace_bytes": (_SZ, [_I32, _I32, _I32, _I64, _I32]),
     "csa2_check_device_error": (ctypes.c_int, [_VP, _VP, ctypes.POINTER(ctypes.c_uint32)]),
     "csa2_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -295,6 +304,54 @@ def csa2_swa_replay(cache: Cache, kv_last: torch.Tensor, idxk_last: torch.Tensor
         _ptr(idxk_last, _BF16, "idxk_last", b * REPLAY * compress * 64),
         _ptr(miss, (torch.uint8, torch.bool), "miss", b), compress, _stream(stream))
     _check(st, "csa2_swa_replay")
+
+
+def csa2_shard_indexer_candidates(cache: Cache, idx_q: torch.Tensor, q_seq: torch.Tensor,
+                                  shard_offset: torch.Tensor, stage: int, cand_score: torch.Tensor,
+                                  cand_id: torch.Tensor, workspace: torch.Tensor, max_visible: int,
+                                  global_pool: torch.Tensor | None = None, head_w: torch.Tensor | None = None,
+                                  stream=None):
+    nq = q_seq.numel()
+    k = POOL_BLOCKS if stage == SHARD_BLOCKS else TOP_K
+    st = lib().csa2_shard_indexer_candidates(
+        cache.ref(), _ptr(idx_q, _BF16, "idx_q", nq * 4 * 64), _ptr(head_w, (torch.float32,), "head_w", nq * 4),
+        _ptr(q_seq, _I32T, "q_seq"), _ptr(shard_offset, _I32T, "shard_offset", nq), nq, int(max_visible),
+        stage, _ptr(global_pool, _I32T, "global_pool", nq * POOL_BLOCKS),
+        _ptr(cand_score, (torch.float32,), "cand_score", nq * k), _ptr(cand_id, _I32T, "cand_id", nq * k),
+        _ptr(workspace, (torch.uint8,), "workspace"), workspace.numel(), _stream(stream))
+    _check(st, "csa2_shard_indexer_candidates")
+
+
+def csa2_shard_merge_topk(cand_score: torch.Tensor, cand_id: torch.Tensor, nshard: int, nq: int, n: int,
+                          query_stride: int, shard_stride: int, k: int, out_id: torch.Tensor,
+                          workspace: torch.Tensor, out_score: torch.Tensor | None = None, stream=None):
+    st = lib().csa2_shard_merge_topk(
+        _ptr(cand_score, (torch.float32,), "cand_score"), _ptr(cand_id, _I32T, "cand_id"), nshard, nq, n,
+        query_stride, shard_stride, k, _ptr(out_id, _I32T, "out_id", nq * k),
+        _ptr(out_score, (torch.float32,), "out_score", nq * k), _ptr(workspace, (torch.uint8,), "workspace"),
+        workspace.numel(), _stream(stream))
+    _check(st, "csa2_shard_merge_topk")
+
+
+def csa2_sparse_attn_shard(cache: Cache, q: torch.Tensor, q_seq: torch.Tensor, shard_offset: torch.Tensor,
+                           global_idx: torch.Tensor, window_start: torch.Tensor, out: torch.Tensor,
+                           lse2: torch.Tensor, workspace: torch.Tensor, sm_scale: float = 1.0, stream=None):
+    nq, heads = q.shape[0], q.shape[1]
+    st = lib().csa2_sparse_attn_shard(
+        cache.ref(), _ptr(q, _BF16, "q", nq * heads * LATENT_DIM), heads, float(sm_scale),
+        _ptr(q_seq, _I32T, "q_seq", nq), _ptr(shard_offset, _I32T, "shard_offset", nq),
+        _ptr(global_idx, _I32T, "global_idx", nq * TOP_K), _ptr(window_start, _I32T, "window_start", nq), nq,
+        _ptr(out, _BF16, "out", nq * heads * LATENT_DIM), _ptr(lse2, (torch.float32,), "lse2", nq * heads),
+        _ptr(workspace, (torch.uint8,), "workspace"), workspace.numel(), _stream(stream))
+    _check(st, "csa2_sparse_attn_shard")
+
+
+def csa2_shard_combine(part: torch.Tensor, lse2: torch.Tensor, nshard: int, nq: int, heads: int,
+                       query_stride: int, shard_stride: int, out: torch.Tensor, stream=None):
+    st = lib().csa2_shard_combine(
+        _ptr(part, _BF16, "part"), _ptr(lse2, (torch.float32,), "lse2"), nshard, nq, heads, query_stride,
+        shard_stride, _ptr(out, _BF16, "out", nq * heads * LATENT_DIM), _stream(stream))
+    _check(st, "csa2_shard_combine")
 
 
 def csa2_check_device_error(cache: Cache, stream=None) -> int:

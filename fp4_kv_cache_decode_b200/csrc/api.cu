@@ -16,21 +16,28 @@ cudaError_t launch_score(int, const CacheView&, const uint16_t*, const float*, c
                          const int32_t*, const int32_t*, int, int64_t, int64_t, float*, float*, int64_t,
                          cudaStream_t);
 cudaError_t launch_topk(int, const CacheView&, const float*, int64_t, const int32_t*, const int32_t*,
-                        const int32_t*, int, int, int32_t*, int64_t, cudaStream_t);
+                        const int32_t*, int, int, int32_t*, int64_t, cudaStream_t, float* = nullptr,
+                        const int32_t* = nullptr, int = 0);
 cudaError_t indexer_set_attributes();
+cudaError_t launch_shard_localize(const CacheView&, const int32_t*, const int32_t*, const int32_t*, int, int,
+                                  int32_t*, const int32_t*, int32_t*, int, cudaStream_t);
+cudaError_t launch_shard_pack(const float*, const int32_t*, int, int, int64_t, int64_t, int, float*, int32_t*,
+                              cudaStream_t);
+cudaError_t launch_shard_combine(const uint16_t*, const float*, int, int, int, int64_t, int64_t, uint16_t*,
+                                 cudaStream_t);
 cudaError_t attention_set_attributes();
 size_t attn_workspace_bytes(int nq, int H);
 int attn_splits_for(int nq);
 cudaError_t launch_attention(const CacheView&, const uint16_t*, int, float, const int32_t*,
                              const int32_t*, const int32_t*, int, uint16_t*, void*, int32_t*, int, int,
-                             cudaStream_t);
+                             cudaStream_t, const int32_t* = nullptr, float* = nullptr);
 }  // namespace csa2
 
 using namespace csa2;
 
 namespace {
 
-constexpr int kSrcFlat = 0, kSrcBlockKeys = 1, kSrcPool = 2;
+constexpr int kSrcFlat = 0, kSrcBlockKeys = 1, kSrcPool = 2, kSrcCand = 3;
 constexpr int32_t kMaxQueries = 65535;   // queries map to gridDim.y
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -87,6 +94,10 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // for a max-pooled Full call, the block maxima at offset nq * flat stride.
 int64_t max_pool_block_stride(int64_t max_visible) {
   return ceil_div(ceil_div(max_visible, kBlock), kBlocksPerPage) * kBlocksPerPage;
+}
+
+size_t shard_attn_idx_offset(int nq, int heads) {
+  return (attn_workspace_bytes(nq, heads) + 255) / 256 * 256;
 }
 
 int64_t indexer_stride(int64_t max_visible, int hierarchical) {
@@ -302,7 +313,131 @@ size_t csa2_workspace_bytes(int32_t op, int32_t nq, int32_t heads, int64_t max_v
     if (heads != 16 && heads != 32 && heads != 48 && heads != 64) return 0;
     return attn_workspace_bytes(nq, heads);
   }
+  if (op == CSA2_OP_SHARD_INDEXER) {   // scores, then the local pool
+    if (max_visible < 0) return 0;
+    return (size_t)nq * (size_t)(indexer_stride(max_visible, CSA2_HIER_MEAN) + kPoolBlocks) * 4 + 256;
+  }
+  if (op == CSA2_OP_SHARD_MERGE) {     // heads = shards, max_visible = candidates per shard
+    if (heads < 1 || max_visible < 8 || max_visible % 8 != 0) return 0;
+    return (size_t)nq * (size_t)heads * (size_t)max_visible * 8 + 256;
+  }
+  if (op == CSA2_OP_SHARD_ATTENTION) {  // attention slices, then local indices and window starts
+    if (heads != 16 && heads != 32 && heads != 48 && heads != 64) return 0;
+    return shard_attn_idx_offset(nq, heads) + (size_t)nq * (kTopK + 1) * 4 + 256;
+  }
   return 0;
+}
+
+int csa2_shard_indexer_candidates(const csa2_cache* cache, const uint16_t* idx_q, const float* head_w,
+                                  const int32_t* q_seq, const int32_t* shard_offset, int32_t nq,
+                                  int64_t max_visible, int32_t stage, const int32_t* global_pool,
+                                  float* cand_score, int32_t* cand_id, void* workspace,
+                                  size_t workspace_bytes, csa2_stream_t stream) {
+  CacheView v;
+  int st = make_view(cache, &v);
+  if (st) return st;
+  if (stage != CSA2_SHARD_BLOCKS && stage != CSA2_SHARD_TOKENS) return CSA2_ERR_INVALID_ARG;
+  if (nq < 0 || max_visible < 0 || max_visible > ((int64_t)1 << 31) - 1) return CSA2_ERR_INVALID_ARG;
+  if (nq > kMaxQueries) return CSA2_ERR_SHAPE;
+  if (nq == 0) return CSA2_OK;
+  if (!idx_q || !q_seq || !shard_offset || !cand_score || !cand_id) return CSA2_ERR_INVALID_ARG;
+  if (stage == CSA2_SHARD_TOKENS && !global_pool) return CSA2_ERR_INVALID_ARG;
+  if (!aligned(idx_q, 16) || !aligned(head_w, 4) || !aligned(q_seq, 4) || !aligned(shard_offset, 4) ||
+      !aligned(global_pool, 4) || !aligned(cand_score, 4) || !aligned(cand_id, 4))
+    return CSA2_ERR_ALIGNMENT;
+  const size_t need = csa2_workspace_bytes(CSA2_OP_SHARD_INDEXER, nq, 0, max_visible, 0);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return CSA2_ERR_WORKSPACE;
+  if ((st = ensure_device_setup())) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  float* scores = static_cast<float*>(workspace);
+  const int64_t stride = indexer_stride(max_visible, CSA2_HIER_MEAN);
+  cudaError_t e;
+  if (stage == CSA2_SHARD_BLOCKS) {
+    const int64_t bk_units = ceil_div(ceil_div(max_visible, kBlock), kBlocksPerPage);
+    e = launch_score(kSrcBlockKeys, v, idx_q, head_w, q_seq, nullptr, nullptr, nq, bk_units, stride, scores,
+                     nullptr, 0, s);
+    if (e == cudaSuccess)
+      e = launch_topk(kSrcBlockKeys, v, scores, stride, q_seq, nullptr, nullptr, nq, kPoolBlocks, cand_id,
+                      kPoolBlocks, s, cand_score, shard_offset, 3);
+  } else {
+    int32_t* lpool = reinterpret_cast<int32_t*>(scores + (int64_t)nq * stride);
+    e = launch_shard_localize(v, q_seq, shard_offset, global_pool, kPoolBlocks, kBlock, lpool, nullptr, nullptr,
+                              nq, s);
+    if (e == cudaSuccess)
+      e = launch_score(kSrcPool, v, idx_q, head_w, q_seq, nullptr, lpool, nq, kPoolBlocks, stride, scores,
+                       nullptr, 0, s);
+    if (e == cudaSuccess)
+      e = launch_topk(kSrcPool, v, scores, stride, q_seq, nullptr, lpool, nq, kTopK, cand_id, kTopK, s,
+                      cand_score, shard_offset, 0);
+  }
+  return from_cuda(e);
+}
+
+int csa2_shard_merge_topk(const float* cand_score, const int32_t* cand_id, int32_t nshard, int32_t nq,
+                          int32_t n, int64_t query_stride, int64_t shard_stride, int32_t k,
+                          int32_t* out_id, float* out_score, void* workspace, size_t workspace_bytes,
+                          csa2_stream_t stream) {
+  if (nshard < 1 || nq < 0 || n < 8 || n % 8 != 0 || k < 1 || query_stride < 0 || shard_stride < 0)
+    return CSA2_ERR_INVALID_ARG;
+  if (nq > kMaxQueries || (int64_t)nshard * n > ((int64_t)1 << 30)) return CSA2_ERR_SHAPE;
+  if (nq == 0) return CSA2_OK;
+  if (!cand_score || !cand_id || !out_id) return CSA2_ERR_INVALID_ARG;
+  if (!aligned(cand_score, 4) || !aligned(cand_id, 4) || !aligned(out_id, 4) || !aligned(out_score, 4))
+    return CSA2_ERR_ALIGNMENT;
+  const size_t need = csa2_workspace_bytes(CSA2_OP_SHARD_MERGE, nq, nshard, n, 0);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return CSA2_ERR_WORKSPACE;
+  int st;
+  if ((st = ensure_device_setup())) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int64_t m = (int64_t)nshard * n;
+  float* pscore = static_cast<float*>(workspace);
+  int32_t* pid = reinterpret_cast<int32_t*>(pscore + (int64_t)nq * m);
+  cudaError_t e = launch_shard_pack(cand_score, cand_id, nshard, n, query_stride, shard_stride, nq, pscore, pid, s);
+  CacheView none{};
+  if (e == cudaSuccess)
+    e = launch_topk(kSrcCand, none, pscore, m, nullptr, nullptr, pid, nq, k, out_id, k, s, out_score, nullptr, 0);
+  return from_cuda(e);
+}
+
+int csa2_sparse_attn_shard(const csa2_cache* cache, const uint16_t* q, int32_t heads, float sm_scale,
+                           const int32_t* q_seq, const int32_t* shard_offset, const int32_t* global_idx,
+                           const int32_t* window_start, int32_t nq, uint16_t* out, float* lse2,
+                           void* workspace, size_t workspace_bytes, csa2_stream_t stream) {
+  CacheView v;
+  int st = make_view(cache, &v);
+  if (st) return st;
+  if (heads != 16 && heads != 32 && heads != 48 && heads != 64) return CSA2_ERR_SHAPE;
+  if (nq < 0) return CSA2_ERR_INVALID_ARG;
+  if (nq > kMaxQueries) return CSA2_ERR_SHAPE;
+  if (nq == 0) return CSA2_OK;
+  if (!q || !q_seq || !shard_offset || !global_idx || !window_start || !out || !lse2) return CSA2_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(q_seq, 4) || !aligned(shard_offset, 4) ||
+      !aligned(global_idx, 4) || !aligned(window_start, 4) || !aligned(lse2, 4))
+    return CSA2_ERR_ALIGNMENT;
+  const size_t need = csa2_workspace_bytes(CSA2_OP_SHARD_ATTENTION, nq, heads, 0, 0);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 16)) return CSA2_ERR_WORKSPACE;
+  if ((st = ensure_device_setup())) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  int32_t* lidx = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) + shard_attn_idx_offset(nq, heads));
+  int32_t* lwin = lidx + (int64_t)nq * kTopK;
+  cudaError_t e = launch_shard_localize(v, q_seq, shard_offset, global_idx, kTopK, 1, lidx, window_start, lwin,
+                                        nq, s);
+  if (e == cudaSuccess)
+    e = launch_attention(v, q, heads, sm_scale, q_seq, nullptr, lidx, nq, out, workspace, nullptr, 0,
+                         attn_splits_for(nq), s, lwin, lse2);
+  return from_cuda(e);
+}
+
+int csa2_shard_combine(const uint16_t* part, const float* lse2, int32_t nshard, int32_t nq, int32_t heads,
+                       int64_t query_stride, int64_t shard_stride, uint16_t* out, csa2_stream_t stream) {
+  if (nshard < 1 || nq < 0 || query_stride < 0 || shard_stride < 0) return CSA2_ERR_INVALID_ARG;
+  if (heads != 16 && heads != 32 && heads != 48 && heads != 64) return CSA2_ERR_SHAPE;
+  if (nq > kMaxQueries) return CSA2_ERR_SHAPE;
+  if (nq == 0) return CSA2_OK;
+  if (!part || !lse2 || !out) return CSA2_ERR_INVALID_ARG;
+  if (!aligned(part, 16) || !aligned(out, 16) || !aligned(lse2, 4)) return CSA2_ERR_ALIGNMENT;
+  return from_cuda(launch_shard_combine(part, lse2, nshard, nq, heads, query_stride, shard_stride, out,
+                                        (cudaStream_t)stream));
 }
 
 int csa2_check_device_error(const csa2_cache* cache, csa2_stream_t stream, uint32_t* bits) {

@@ -74,6 +74,14 @@ constexpr uint32_t kSwaRow = 0x80000000u;              // flag: id = slot of the
 constexpr int kRowCacheInts = CSA2_ATTN_ROWS_INTS;      // 640 row ids + 8 range counts per query
 static_assert(kRowCacheInts >= kMaxRows + 8, "row cache layout");
 constexpr float kSlack2 = 12.0f;                       // base-2 headroom before the max moves
+
+// Optional inputs/outputs of a position-sharded call: a per-query window start
+// (the window is [max(v - 128, wstart), v)) and the base-2 log-sum-exp of each
+// head's logits over the attended set (-inf when the set is empty).
+struct AttnShardIO {
+  const int32_t* wstart;
+  float* lse2;
+};
 static_assert(kPipeSmem <= 232448, "shared memory budget");
 
 // Instruction descriptors for tcgen05.mma kind::f16: D fp32 (bits 4-5 = 1),
@@ -407,7 +415,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
 attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_scale,
                  const int32_t* __restrict__ q_seq, const int32_t* __restrict__ q_vis,
                  const int32_t* __restrict__ idx, int nsplit, int range_slots, uint16_t* __restrict__ out,
-                 uint16_t* __restrict__ part, int32_t* __restrict__ rcache, int rmode) {
+                 uint16_t* __restrict__ part, int32_t* __restrict__ rcache, int rmode, AttnShardIO shard) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw_s = (uint32_t)__cvta_generic_to_shared(smem_raw);
   const uint32_t sb = (raw_s + 1023u) & ~1023u;            // 1024-B aligned base (swizzle atoms)
@@ -417,6 +425,7 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
   float* const fac = m_run + 64;
   float* const l_s = m_run + 128;
   float* const f_s = m_run + 192;                                 // output factor per head
+  float2* const lse_ml = reinterpret_cast<float2*>(sp + kOffRedM);  // epilogue: final (M, L) per head
   uint32_t* const rows_s = reinterpret_cast<uint32_t*>(sp + kOffRows);
   // [0] TMEM base, [1] last barrier the MMA thread committed to (0: none), [2] its parity,
   // [4 + w] used-slot count of warp w, [20 + w] largest |q| bits seen by warp w
@@ -476,7 +485,10 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
     if (s0 + 1 < hi && s0 + 1 < kTopK) e1 = idx_row[s0 + 1];
     const int seq = q_seq[r];
     const int64_t v = q_vis ? (int64_t)q_vis[r] : (int64_t)seq_len_of(c, seq);
-    const int64_t w0 = v > kWindow ? v - kWindow : 0;
+    // window [w0, v): the last 128 visible positions, or from a given start
+    // (at most 128 positions; a start at v leaves the window empty)
+    int64_t w0 = v > kWindow ? v - kWindow : 0;
+    if (shard.wstart) w0 = max(w0, min(v, (int64_t)max(0, shard.wstart[r])));
     auto slot_pos = [&](int sl, int32_t e) -> int64_t {   // attended position of a slot, -1 if unused
       if (sl >= hi) return -1;
       if (sl < kTopK) {
@@ -831,11 +843,21 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
       }
       const float2 self = ml[split * 64 + tid];
       f_s[tid] = (self.y > 0.0f && L > 0.0f) ? ex2(self.x - M) / L : 0.0f;
+      lse_ml[tid] = make_float2(M, L);
     }
   } else if (tid < 64) {
-    f_s[tid] = (all_ok && l_s[tid] > 0.0f) ? 1.0f / l_s[tid] : 0.0f;
+    const bool have = all_ok && l_s[tid] > 0.0f;
+    f_s[tid] = have ? 1.0f / l_s[tid] : 0.0f;
+    lse_ml[tid] = make_float2(have ? m_run[tid] : -INFINITY, have ? l_s[tid] : 0.0f);
   }
   __syncthreads();
+  // the idle MMA warp writes the log-sum-exp of a sharded call (one range per query)
+  if (warp == kMmaWarp && shard.lse2 != nullptr && split == 0) {
+    for (int h = lane; h < H; h += 32) {
+      const float2 ml = lse_ml[h];
+      shard.lse2[(int64_t)r * H + h] = ml.y > 0.0f ? ml.x + __log2f(ml.y) : -INFINITY;
+    }
+  }
   // f . O^T straight from TMEM to global [H][512]: the lanes of a warp hold 32
   // consecutive channels, so each 2-B store instruction writes one 64-B run.
   // Warps 0..11 share the work, three per TMEM sub-partition (warp % 4).
@@ -948,7 +970,8 @@ int attn_splits_for(int nq) { return attn_splits(nq); }
 
 cudaError_t launch_attention(const CacheView& c, const uint16_t* q, int H, float sm_scale,
                              const int32_t* q_seq, const int32_t* q_vis, const int32_t* idx, int nq,
-                             uint16_t* out, void* ws, int32_t* rcache, int rmode, int s, cudaStream_t st) {
+                             uint16_t* out, void* ws, int32_t* rcache, int rmode, int s, cudaStream_t st,
+                             const int32_t* wstart, float* lse2) {
   if (nq == 0) return cudaSuccess;
   if (H % 16 != 0 || H < 16 || H > kHeadsMma) return cudaErrorInvalidValue;
   if (s != 1 && s != 2 && s != 4 && s != 8) return cudaErrorInvalidValue;
@@ -966,8 +989,9 @@ cudaError_t launch_attention(const CacheView& c, const uint16_t* q, int H, float
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = s > 1 ? 1 : 0;
+  const AttnShardIO shard{wstart, lse2};
   return cudaLaunchKernelEx(&cfg, attn_pipe_kernel, c, q, H, sm_scale, q_seq, q_vis, idx, s, range, out,
-                            reinterpret_cast<uint16_t*>(ws), rcache, rmode);
+                            reinterpret_cast<uint16_t*>(ws), rcache, rmode, shard);
 }
 
 }  // namespace csa2

@@ -30,7 +30,26 @@
 
 namespace csa2 {
 
-enum UnitSource : int { SRC_FLAT = 0, SRC_BLOCKKEYS = 1, SRC_POOL = 2 };
+// SRC_CAND (top-k only): explicit candidates -- scores[r][i] with the id of
+// entry i in cand_ids[r][i], the entries of a row in ascending id order.
+enum UnitSource : int { SRC_FLAT = 0, SRC_BLOCKKEYS = 1, SRC_POOL = 2, SRC_CAND = 3 };
+
+// Where a top-k writes: ids [nq][stride] (-1 padded), optionally the selected
+// scores (same layout, -inf padded), and optionally a per-query offset added to
+// every selected id, id_offset[r] >> offset_shift (a shard's first global
+// position, or its first block with shift 3).
+struct TopkOut {
+  int32_t* ids;
+  int64_t stride;
+  float* scores;
+  const int32_t* id_offset;
+  int offset_shift;
+};
+
+// Inverse of score_key on non-zero keys (exact; -0 comes back as +0).
+__device__ __forceinline__ float key_score(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
 
 constexpr int kScoreThreads = 256;
 constexpr int kScoreWarps = kScoreThreads / 32;
@@ -358,6 +377,7 @@ __device__ __forceinline__ void find_bucket(TopkSmem* sm, int nbins, uint32_t k_
 template <int SRC>
 __device__ __forceinline__ int32_t map_out(int64_t i, const int32_t* pool_row) {
   if (SRC == SRC_POOL) return pool_row[i >> 3] * kBlock + (int32_t)(i & 7);
+  if (SRC == SRC_CAND) return pool_row[i];
   return (int32_t)i;
 }
 
@@ -385,7 +405,7 @@ static_assert(kKeysPerThread == 16, "a thread's positions span exactly two 8-tok
 template <int SRC>
 __device__ __forceinline__ void topk_registers(const float* __restrict__ srow, int64_t n, int k,
                                                const int32_t* pool_row, int32_t* __restrict__ orow,
-                                               TopkSmem* sm) {
+                                               float* __restrict__ oscore, int32_t id_off, TopkSmem* sm) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t lo = (int64_t)tid * kKeysPerThread;
   uint32_t key[kKeysPerThread];
@@ -550,12 +570,17 @@ __device__ __forceinline__ void topk_registers(const float* __restrict__ srow, i
     if (sel && slot < (uint32_t)k) {
       int32_t o;
       if (SRC == SRC_POOL) o = (j < 8 ? pb0 : pb1) * kBlock + (int32_t)((lo + j) & 7);
+      else if (SRC == SRC_CAND) o = pool_row[lo + j];
       else o = (int32_t)(lo + j);
-      orow[slot++] = o;
+      if (oscore) oscore[slot] = key_score(kj);
+      orow[slot++] = o + id_off;
     }
   }
   const uint32_t total = tot_gt + min(tot_eq, need_eq);
-  for (int64_t s = (int64_t)total + tid; s < k; s += kTopkThreads) orow[s] = -1;
+  for (int64_t s = (int64_t)total + tid; s < k; s += kTopkThreads) {
+    orow[s] = -1;
+    if (oscore) oscore[s] = -INFINITY;
+  }
 }
 
 // One CTA per query: select the k best entries of scores[r][0 .. n_r).
@@ -574,19 +599,23 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(CacheView c, const f
                                                             int64_t stride, const int32_t* __restrict__ q_seq,
                                                             const int32_t* __restrict__ q_vis,
                                                             const int32_t* __restrict__ pool, int k,
-                                                            int32_t* __restrict__ out, int64_t out_stride) {
+                                                            TopkOut out) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   TopkSmem* sm = reinterpret_cast<TopkSmem*>(smem_raw);
 
   const int r = blockIdx.x;
   const int tid = threadIdx.x;
-  const int64_t v = visible_of(c, q_seq, q_vis, r);
-  const int64_t n = min(units_of(SRC, v) * kBlock, stride);   // a multiple of 8
+  // candidates: every entry of the row (a multiple of 8), ids from `pool`
+  const int64_t n = SRC == SRC_CAND ? stride
+                                    : min(units_of(SRC, visible_of(c, q_seq, q_vis, r)) * kBlock, stride);
   const float* srow = scores + (int64_t)r * stride;
-  const int32_t* pool_row = pool ? pool + (int64_t)r * kPoolBlocks : nullptr;
-  int32_t* orow = out + (int64_t)r * out_stride;
+  const int32_t* pool_row =
+      pool ? pool + (int64_t)r * (SRC == SRC_CAND ? stride : (int64_t)kPoolBlocks) : nullptr;
+  int32_t* orow = out.ids + (int64_t)r * out.stride;
+  float* oscore = out.scores ? out.scores + (int64_t)r * out.stride : nullptr;
+  const int32_t id_off = out.id_offset ? (out.id_offset[r] >> out.offset_shift) : 0;
   if (n <= kTopkSmemKeys) {
-    topk_registers<SRC>(srow, n, k, pool_row, orow, sm);
+    topk_registers<SRC>(srow, n, k, pool_row, orow, oscore, id_off, sm);
     return;
   }
   auto key_at = [&](int64_t i) -> uint32_t { return score_key(srow[i]); };
@@ -690,12 +719,18 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(CacheView c, const f
         if (kk[j] == 0u || kk[j] < T) continue;
         bool sel = kk[j] > T;
         if (!sel) sel = eq_rank++ < need_eq;
-        if (sel && slot < (uint32_t)k) orow[slot++] = map_out<SRC>(i + j, pool_row);
+        if (sel && slot < (uint32_t)k) {
+          if (oscore) oscore[slot] = key_score(kk[j]);
+          orow[slot++] = map_out<SRC>(i + j, pool_row) + id_off;
+        }
       }
     }
   }
   const uint32_t total = tot_gt + min(tot_eq, need_eq);
-  for (int64_t s = (int64_t)total + tid; s < k; s += kTopkThreads) orow[s] = -1;
+  for (int64_t s = (int64_t)total + tid; s < k; s += kTopkThreads) {
+    orow[s] = -1;
+    if (oscore) oscore[s] = -INFINITY;
+  }
 }
 
 }  // namespace csa2
@@ -719,6 +754,8 @@ cudaError_t indexer_set_attributes() {
     e = cudaFuncSetAttribute(topk_kernel<SRC_BLOCKKEYS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(topk_kernel<SRC_POOL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(topk_kernel<SRC_CAND>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   return e;
 }
 
@@ -757,15 +794,19 @@ cudaError_t launch_score(int src, const CacheView& c, const uint16_t* idx_q, con
 
 cudaError_t launch_topk(int src, const CacheView& c, const float* scores, int64_t stride,
                         const int32_t* q_seq, const int32_t* q_vis, const int32_t* pool, int nq,
-                        int k, int32_t* out, int64_t out_stride, cudaStream_t st) {
+                        int k, int32_t* out, int64_t out_stride, cudaStream_t st, float* out_scores,
+                        const int32_t* id_offset, int offset_shift) {
   const size_t smem = topk_smem_bytes();
   if (nq == 0) return cudaSuccess;
+  const TopkOut o{out, out_stride, out_scores, id_offset, offset_shift};
   if (src == SRC_FLAT)
-    topk_kernel<SRC_FLAT><<<nq, kTopkThreads, smem, st>>>(c, scores, stride, q_seq, q_vis, pool, k, out, out_stride);
+    topk_kernel<SRC_FLAT><<<nq, kTopkThreads, smem, st>>>(c, scores, stride, q_seq, q_vis, pool, k, o);
   else if (src == SRC_BLOCKKEYS)
-    topk_kernel<SRC_BLOCKKEYS><<<nq, kTopkThreads, smem, st>>>(c, scores, stride, q_seq, q_vis, pool, k, out, out_stride);
+    topk_kernel<SRC_BLOCKKEYS><<<nq, kTopkThreads, smem, st>>>(c, scores, stride, q_seq, q_vis, pool, k, o);
+  else if (src == SRC_POOL)
+    topk_kernel<SRC_POOL><<<nq, kTopkThreads, smem, st>>>(c, scores, stride, q_seq, q_vis, pool, k, o);
   else
-    topk_kernel<SRC_POOL><<<nq, kTopkThreads, smem, st>>>(c, scores, stride, q_seq, q_vis, pool, k, out, out_stride);
+    topk_kernel<SRC_CAND><<<nq, kTopkThreads, smem, st>>>(c, scores, stride, q_seq, q_vis, pool, k, o);
   return cudaGetLastError();
 }
 

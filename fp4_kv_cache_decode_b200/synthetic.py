@@ -54,6 +54,25 @@ def fill_decode_cache(w: wl.Workload, cache: csa2.Cache, lengths=None, chunk: in
             csa2.csa2_kv_quant_append(cache, kvbuf[:n], kbuf[:n], eseq, epos, 1)
 
 
+def fill_sharded_cache(w: wl.Workload, cache: csa2.Cache, bounds, chunk: int = 65536):
+    """Shard caches of position-sharded sequences: sequence b * S + s of `cache`
+    holds positions [start, end) = bounds[b][s] of sequence b of the workload
+    as its entries 0 .. end - start - 1 (ratio 1)."""
+    col = torch.from_numpy(wl.kv_col_scale(w.seed)).cuda()
+    kvbuf = torch.empty((chunk, 512), dtype=torch.bfloat16, device="cuda")
+    kbuf = torch.empty((chunk, 64), dtype=torch.bfloat16, device="cuda")
+    for b, shards in enumerate(bounds):
+        for s, (lo, hi) in enumerate(shards):
+            seq = b * len(shards) + s
+            for p0 in range(lo, hi, chunk):
+                n = min(chunk, hi - p0)
+                wdev.kv_rows(w.seed, b, p0, n, out=kvbuf[:n], col_scale=col)
+                wdev.idxk_rows(w.seed, b, p0, n, out=kbuf[:n])
+                eseq = torch.full((n,), seq, dtype=torch.int32, device="cuda")
+                epos = torch.arange(p0 - lo, p0 - lo + n, dtype=torch.int32, device="cuda")
+                csa2.csa2_kv_quant_append(cache, kvbuf[:n], kbuf[:n], eseq, epos, 1)
+
+
 def fill_prefill_chunk(w: wl.Workload, cache: csa2.Cache, chunk_index: int, seq: int = 0):
     """Encode the raw tokens of one prefill chunk at compression ratio w.compress."""
     r0 = chunk_index * w.chunk

@@ -87,7 +87,14 @@ typedef enum {
 
 typedef enum { CSA2_FULL = 0, CSA2_REINDEX = 1, CSA2_REUSE = 2 } csa2_mode;
 
-typedef enum { CSA2_OP_INDEXER = 1, CSA2_OP_ATTENTION = 2 } csa2_op;
+typedef enum {
+  CSA2_OP_INDEXER = 1,
+  CSA2_OP_ATTENTION = 2,
+  CSA2_OP_SHARD_INDEXER = 3,    /* csa2_shard_indexer_candidates: nq, max_visible         */
+  CSA2_OP_SHARD_MERGE = 4,      /* csa2_shard_merge_topk: nq, heads = nshard,
+                                   max_visible = candidates per shard                     */
+  CSA2_OP_SHARD_ATTENTION = 5   /* csa2_sparse_attn_shard: nq, heads                      */
+} csa2_op;
 
 /* bits OR-ed into *error_word by kernels */
 #define CSA2_DEVERR_PAGE 1u  /* page id outside [0, n_pages) or page slot >= max_pages */
@@ -292,8 +299,87 @@ int csa2_indexer_score_topk_noalloc(const csa2_cache* cache, const uint16_t* idx
                                     int32_t mode, int32_t hierarchical, int32_t layer,
                                     csa2_indexset* set, csa2_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Position-sharded decode of long sequences (multi-GPU).
+ *
+ * A sequence is split into contiguous position ranges (shards), one per GPU;
+ * a shard's cache holds its positions as entries 0 .. n-1 of its own
+ * sequence, and shard_offset[r] (a multiple of 8) is the global position of
+ * entry 0 for query r.  Per layer every GPU calls, with the same queries:
+ *   1. csa2_shard_indexer_candidates(stage CSA2_SHARD_BLOCKS): its 2,048 best
+ *      blocks (score, global block id); all-gather; csa2_shard_merge_topk
+ *      (k = 2048) -> the global pool, identical on every GPU;
+ *   2. csa2_shard_indexer_candidates(stage CSA2_SHARD_TOKENS, the pool): its
+ *      512 best pool positions (score, global position); all-gather;
+ *      csa2_shard_merge_topk (k = 512) -> the global index set;
+ *   3. csa2_sparse_attn_shard: attention over the set's positions and the
+ *      window's positions that it holds -> normalised output + base-2
+ *      log-sum-exp; all-gather; csa2_shard_combine -> the layer's output.
+ * Each merge is exact: an element of a global top-k is in its own shard's
+ * top-k; candidate lists concatenated in shard order are in ascending global
+ * order, so ties go to the lowest position as in the unsharded call.  The
+ * result equals the unsharded hierarchical (mean-pooled) Full step up to the
+ * rounding of the partial outputs (the pool, the 2,048-block rule and the
+ * window are those of csa2_indexer_score_topk / csa2_sparse_attn; agentnet.co.il,
+ * section "CSA2: דחיסה לאורך ציר השכבות").  The exchanges are the caller's
+ * collectives (e.g. an NCCL all-gather); the merge and combine calls read the
+ * gathered rows through (query_stride, shard_stride) in rows: shard s of
+ * query q is row q * query_stride + s * shard_stride.
+ * ------------------------------------------------------------------------ */
+#define CSA2_SHARD_BLOCKS 0
+#define CSA2_SHARD_TOKENS 1
+
+/* Candidates of one shard for queries r < nq (sequence q_seq[r] of `cache`,
+ * all its entries visible, idx_q / head_w as in csa2_indexer_score_topk).
+ * stage CSA2_SHARD_BLOCKS: cand_score / cand_id [nq][2048] = the shard's
+ * 2,048 best block keys, ids = global block ids (shard_offset / 8 + local),
+ * ascending, (-inf, -1) padded.  stage CSA2_SHARD_TOKENS: global_pool
+ * [nq][2048] (global block ids, -1 padded) -> cand_score / cand_id
+ * [nq][512] = the 512 best positions of the pool blocks this shard holds,
+ * global positions, ascending, (-inf, -1) padded.  Workspace:
+ * csa2_workspace_bytes(CSA2_OP_SHARD_INDEXER, nq, 0, max_visible, 0).
+ * A non-empty shard whose shard_offset is negative or not a multiple of 8
+ * raises CSA2_DEVERR_POS. */
+int csa2_shard_indexer_candidates(const csa2_cache* cache, const uint16_t* idx_q, const float* head_w,
+                                  const int32_t* q_seq, const int32_t* shard_offset, int32_t nq,
+                                  int64_t max_visible, int32_t stage, const int32_t* global_pool,
+                                  float* cand_score, int32_t* cand_id, void* workspace,
+                                  size_t workspace_bytes, csa2_stream_t stream);
+
+/* Exact top-k of gathered candidate lists: for query q, the nshard rows of n
+ * candidates (score, id) at rows q * query_stride + s * shard_stride (n a
+ * multiple of 8; rows in shard order hold ascending ids, -1 entries with
+ * -inf scores are no candidates).  Writes out_id [nq][k] (ascending, -1
+ * padded) and, if out_score != NULL, their scores.  Workspace:
+ * csa2_workspace_bytes(CSA2_OP_SHARD_MERGE, nq, nshard, n, 0). */
+int csa2_shard_merge_topk(const float* cand_score, const int32_t* cand_id, int32_t nshard, int32_t nq,
+                          int32_t n, int64_t query_stride, int64_t shard_stride, int32_t k,
+                          int32_t* out_id, float* out_score, void* workspace, size_t workspace_bytes,
+                          csa2_stream_t stream);
+
+/* Attention of one shard: query r attends over the positions of global_idx[r]
+ * (global positions, [nq][512], -1 padded) that this shard holds, joined with
+ * the window positions [window_start[r], end) that it holds (window_start =
+ * the global window's first position, max(0, L - 128)).  out (bf16
+ * [nq][heads][512]) is normalised over that set; lse2 (float [nq][heads]) is
+ * its base-2 log-sum-exp of sm_scale q . k (-inf, with a zero output, when
+ * the shard holds none of the set).  Same numerics as csa2_sparse_attn.
+ * Workspace: csa2_workspace_bytes(CSA2_OP_SHARD_ATTENTION, nq, heads, 0, 0). */
+int csa2_sparse_attn_shard(const csa2_cache* cache, const uint16_t* q, int32_t heads, float sm_scale,
+                           const int32_t* q_seq, const int32_t* shard_offset, const int32_t* global_idx,
+                           const int32_t* window_start, int32_t nq, uint16_t* out, float* lse2,
+                           void* workspace, size_t workspace_bytes, csa2_stream_t stream);
+
+/* Merge of the shards' attention outputs: out[q] = sum_s w_s O_s / sum_s w_s,
+ * w_s = 2^(lse2_s - max_s lse2_s), over the shards with lse2 > -inf (zero if
+ * none), rounded to bf16.  part: bf16 rows of [heads][512] and lse2: rows of
+ * [heads], shard s of query q at row q * query_stride + s * shard_stride. */
+int csa2_shard_combine(const uint16_t* part, const float* lse2, int32_t nshard, int32_t nq, int32_t heads,
+                       int64_t query_stride, int64_t shard_stride, uint16_t* out, csa2_stream_t stream);
+
 /* Workspace bytes for an indexer call (op = CSA2_OP_INDEXER: nq, max_visible,
- * hierarchical) or an attention call (op = CSA2_OP_ATTENTION: nq, heads).
+ * hierarchical), an attention call (op = CSA2_OP_ATTENTION: nq, heads) or a
+ * sharded call (CSA2_OP_SHARD_*, arguments as listed with the ops).
  * Returns 0 for an invalid request or when none is needed. */
 size_t csa2_workspace_bytes(int32_t op, int32_t nq, int32_t heads, int64_t max_visible,
                             int32_t hierarchical);

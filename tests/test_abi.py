@@ -193,3 +193,33 @@ def test_indexer_key_format_is_checked(csa2_lib):
     assert rep(_cache(csa2_lib, f, idxk_format=-1)) == 1
     assert L.csa2_kv_quant_append(B(_cache(csa2_lib, f, idxk_format=7)), f.p(), f.p(), f.p(), f.p(), 1, 1,
                                   None) == 1
+
+
+def test_sharded_call_argument_checks(csa2_lib):
+    L = csa2_lib.lib()
+    f = _Fake()
+    c = _cache(csa2_lib, f)
+    B = ctypes.byref
+    ws = csa2_lib.csa2_workspace_bytes
+    assert ws(3, 4, 0, 40000, 0) == 4 * (16384 + 2048) * 4 + 256
+    assert ws(4, 4, 8, 2048, 0) == 4 * 8 * 2048 * 8 + 256
+    assert ws(4, 4, 8, 12, 0) == 0                      # candidates per shard: a multiple of 8
+    assert ws(5, 4, 20, 0, 0) == 0
+    cand = lambda stage, pool=None, wsz=1 << 30: L.csa2_shard_indexer_candidates(
+        B(c), f.p(), None, f.p(), f.p(), 2, 40000, stage, pool, f.p(), f.p(), f.p(), wsz, None)
+    assert cand(2) == 1                                 # unknown stage
+    assert cand(1) == 1                                 # the token stage needs the pool
+    assert cand(0, wsz=16) == 5
+    merge = lambda nshard, n, k, wsz=1 << 30: L.csa2_shard_merge_topk(
+        f.p(), f.p(), nshard, 2, n, 1, 2, k, f.p(), None, f.p(), wsz, None)
+    assert merge(0, 2048, 2048) == 1
+    assert merge(2, 12, 8) == 1
+    assert merge(2, 2048, 0) == 1
+    assert merge(2, 2048, 2048, wsz=100) == 5
+    attn = lambda heads, wsz=1 << 30: L.csa2_sparse_attn_shard(
+        B(c), f.p(), heads, ctypes.c_float(1.0), f.p(), f.p(), f.p(), f.p(), 2, f.p(), f.p(), f.p(), wsz, None)
+    assert attn(20) == 2
+    assert attn(64, wsz=0) == 5
+    assert L.csa2_shard_combine(f.p(), f.p(), 0, 2, 64, 1, 2, f.p(), None) == 1
+    assert L.csa2_shard_combine(f.p(), f.p(), 2, 2, 24, 1, 2, f.p(), None) == 2
+    assert L.csa2_shard_combine(f.p(8), f.p(), 2, 2, 64, 1, 2, f.p(), None) == 3
