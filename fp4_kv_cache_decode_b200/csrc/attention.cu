@@ -36,6 +36,7 @@
 // (tcgen05.commit for tensor-core completion); every wait is bounded and
 // reports CSA2_DEVERR_TIMEOUT instead of hanging.
 #include "common.cuh"
+#include "tc.cuh"
 
 #include <cuda_fp16.h>
 
@@ -93,58 +94,7 @@ constexpr uint32_t kIdescPV = (1u << 4) | (1u << 15) | (1u << 16) | ((uint32_t)(
 constexpr uint32_t kIdescL = (1u << 4) | (1u << 16) | ((uint32_t)(kHeadsMma >> 3) << 17) | ((uint32_t)(64 >> 4) << 24);
 
 
-constexpr uint32_t kWaitLimit = 1u << 22;    // try_wait rounds before a wait gives up
 constexpr uint32_t kPollLimit = 1u << 26;    // idle polls of the MMA thread before it gives up
-
-// Shared-memory matrix descriptor: start address, leading and stride byte
-// offsets (16-B units), descriptor version 1, 128-byte swizzle.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
-}
-
-__device__ __forceinline__ void mma_commit(uint32_t mbar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
-               : "memory");
-}
-
-// Non-blocking check of an mbarrier phase.
-__device__ __forceinline__ bool mbar_test(uint32_t mbar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(mbar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(mbar), "r"(parity)
-        : "memory");
-    if (ok) return true;
-  }
-  return false;
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // 32 consecutive fp32 TMEM columns of this thread's lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
@@ -192,14 +142,6 @@ __device__ __forceinline__ uint4 decode8_f16(uint32_t codes, uint32_t scale2) {
   asm("mul.rn.f16x2 %0, %0, %1;" : "+r"(d2) : "r"(scale2));
   asm("mul.rn.f16x2 %0, %0, %1;" : "+r"(d3) : "r"(scale2));
   return make_uint4(d0, d1, d2, d3);
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}\n" ::"r"(bar) : "memory");
 }
 
 __device__ __forceinline__ void smx_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kSmxThreads) : "memory"); }

@@ -27,12 +27,9 @@
 // lowest-position entries equal to T, so the tie-break is "lowest position
 // wins" and the output comes out in ascending position order.
 #include "common.cuh"
+#include "indexer.cuh"
 
 namespace csa2 {
-
-// SRC_CAND (top-k only): explicit candidates -- scores[r][i] with the id of
-// entry i in cand_ids[r][i], the entries of a row in ascending id order.
-enum UnitSource : int { SRC_FLAT = 0, SRC_BLOCKKEYS = 1, SRC_POOL = 2, SRC_CAND = 3 };
 
 // Where a top-k writes: ids [nq][stride] (-1 padded), optionally the selected
 // scores (same layout, -inf padded), and optionally a per-query offset added to
@@ -69,19 +66,6 @@ struct ScoreGeom {
 };
 constexpr uint32_t kScoreSmemMax = ScoreGeom<false>::kSmem;   // 98,304 B
 static_assert(ScoreGeom<true>::kSmem <= kScoreSmemMax, "stage sizes");
-
-__device__ __forceinline__ int64_t visible_of(const CacheView& c, const int32_t* q_seq,
-                                              const int32_t* q_vis, int r) {
-  return q_vis ? (int64_t)q_vis[r] : (int64_t)seq_len_of(c, q_seq[r]);
-}
-
-// Number of units of query r for a source.
-__device__ __forceinline__ int64_t units_of(int src, int64_t v) {
-  const int64_t nb = (v + kBlock - 1) / kBlock;
-  if (src == SRC_FLAT) return nb;
-  if (src == SRC_BLOCKKEYS) return (nb + kBlocksPerPage - 1) / kBlocksPerPage;
-  return kPoolBlocks;
-}
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -740,6 +724,12 @@ namespace csa2 {
 
 size_t topk_smem_bytes() { return sizeof(TopkSmem); }
 
+cudaError_t score_mma_set_attributes();
+cudaError_t launch_score_mma(int src, const CacheView& c, const uint16_t* idx_q, const float* head_w,
+                             const int32_t* q_seq, const int32_t* q_vis, const int32_t* pool, int nq,
+                             int64_t max_units, int64_t stride, float* scores, float* block_max, int64_t bstride,
+                             cudaStream_t st);
+
 // Opt the top-k kernels in to their shared-memory size (once per device).
 cudaError_t indexer_set_attributes() {
   const int smem = (int)topk_smem_bytes();
@@ -750,6 +740,7 @@ cudaError_t indexer_set_attributes() {
       (const void*)score_units_kernel<SRC_POOL, true>};
   for (const void* k : score_kernels)
     if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmemMax);
+  if (e == cudaSuccess) e = score_mma_set_attributes();
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(topk_kernel<SRC_BLOCKKEYS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess)
@@ -766,12 +757,16 @@ cudaError_t launch_score(int src, const CacheView& c, const uint16_t* idx_q, con
                          int64_t bstride, cudaStream_t st) {
   // units per CTA: enough CTAs for two per SM over the whole batch, in whole
   // 32-unit stages, at most 256
+  const bool f8 = c.idxk_fp8 && src != SRC_BLOCKKEYS;
+  // bf16 keys: tensor-core scoring (score_mma.cu); FP8 keys: the FFMA kernel below
+  if (!f8)
+    return launch_score_mma(src, c, idx_q, head_w, q_seq, q_vis, pool, nq, max_units, stride, scores, block_max,
+                            bstride, st);
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   int64_t per_query = nq > 0 ? ((int64_t)2 * sms) / nq : 1;   // CTAs per query that fit in one wave
   if (per_query < 1) per_query = 1;
   int64_t upc = (max_units + per_query - 1) / per_query;
-  const bool f8 = c.idxk_fp8 && src != SRC_BLOCKKEYS;
   const int stage_units = f8 ? ScoreGeom<true>::kUnits : ScoreGeom<false>::kUnits;
   const uint32_t smem = f8 ? ScoreGeom<true>::kSmem : ScoreGeom<false>::kSmem;
   upc = (upc + stage_units - 1) / stage_units * stage_units;
