@@ -358,6 +358,8 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
                  const int32_t* __restrict__ q_seq, const int32_t* __restrict__ q_vis,
                  const int32_t* __restrict__ idx, int nsplit, int range_slots, uint16_t* __restrict__ out,
                  uint16_t* __restrict__ part, int32_t* __restrict__ rcache, int rmode, AttnShardIO shard) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw_s = (uint32_t)__cvta_generic_to_shared(smem_raw);
   const uint32_t sb = (raw_s + 1023u) & ~1023u;            // 1024-B aligned base (swizzle atoms)
@@ -924,13 +926,15 @@ cudaError_t launch_attention(const CacheView& c, const uint16_t* q, int H, float
   cfg.blockDim = dim3(kPipeThreads);
   cfg.dynamicSmemBytes = kPipeSmem;
   cfg.stream = st;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = (unsigned)s;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see launch_pdl
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[1].id = cudaLaunchAttributeClusterDimension;
+  at[1].val.clusterDim.x = (unsigned)s;
+  at[1].val.clusterDim.y = 1;
+  at[1].val.clusterDim.z = 1;
   cfg.attrs = at;
-  cfg.numAttrs = s > 1 ? 1 : 0;
+  cfg.numAttrs = s > 1 ? 2 : 1;
   const AttnShardIO shard{wstart, lse2};
   return cudaLaunchKernelEx(&cfg, attn_pipe_kernel, c, q, H, sm_scale, q_seq, q_vis, idx, s, range, out,
                             reinterpret_cast<uint16_t*>(ws), rcache, rmode, shard);

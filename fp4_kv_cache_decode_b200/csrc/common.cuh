@@ -125,4 +125,28 @@ __device__ __forceinline__ uint32_t score_key(float s) {
   return k <= 0x007FFFFFu ? 0u : k;
 }
 
+// Programmatic dependent launch.  Kernels are launched with launch_pdl, so a
+// kernel's CTAs may be scheduled while the previous kernel of the stream drains;
+// every kernel calls pdl_wait() before it reads anything (an earlier kernel may
+// have written it) and then pdl_trigger() so that the next launch can begin.
+// Both are no-ops for a launch without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 }  // namespace csa2

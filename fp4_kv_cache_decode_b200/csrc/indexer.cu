@@ -90,6 +90,8 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_units_kernel(CacheView
                                                                        int upc, float* __restrict__ scores,
                                                                        float* __restrict__ block_max,
                                                                        int64_t bstride) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) uint8_t stage[];
   static_assert(!F8 || SRC != SRC_BLOCKKEYS, "block keys are bf16");
   __shared__ const uint8_t* ubase[kUnitsPerCta];
@@ -584,6 +586,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(CacheView c, const f
                                                             const int32_t* __restrict__ q_vis,
                                                             const int32_t* __restrict__ pool, int k,
                                                             TopkOut out) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   TopkSmem* sm = reinterpret_cast<TopkSmem*>(smem_raw);
 
@@ -775,15 +779,15 @@ cudaError_t launch_score(int src, const CacheView& c, const uint16_t* idx_q, con
   dim3 grid((unsigned)((max_units + upc - 1) / upc), (unsigned)nq);
   if (grid.x == 0) return cudaSuccess;
   if (src == SRC_BLOCKKEYS)
-    score_units_kernel<SRC_BLOCKKEYS, false><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
+    launch_pdl(score_units_kernel<SRC_BLOCKKEYS, false>, grid, kScoreThreads, smem, st, c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
   else if (src == SRC_FLAT && f8)
-    score_units_kernel<SRC_FLAT, true><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
+    launch_pdl(score_units_kernel<SRC_FLAT, true>, grid, kScoreThreads, smem, st, c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
   else if (src == SRC_FLAT)
-    score_units_kernel<SRC_FLAT, false><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
+    launch_pdl(score_units_kernel<SRC_FLAT, false>, grid, kScoreThreads, smem, st, c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
   else if (f8)
-    score_units_kernel<SRC_POOL, true><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
+    launch_pdl(score_units_kernel<SRC_POOL, true>, grid, kScoreThreads, smem, st, c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
   else
-    score_units_kernel<SRC_POOL, false><<<grid, kScoreThreads, smem, st>>>(c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
+    launch_pdl(score_units_kernel<SRC_POOL, false>, grid, kScoreThreads, smem, st, c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
   return cudaGetLastError();
 }
 
@@ -795,13 +799,13 @@ cudaError_t launch_topk(int src, const CacheView& c, const float* scores, int64_
   if (nq == 0) return cudaSuccess;
   const TopkOut o{out, out_stride, out_scores, id_offset, offset_shift};
   if (src == SRC_FLAT)
-    topk_kernel<SRC_FLAT><<<nq, kTopkThreads, smem, st>>>(c, scores, stride, q_seq, q_vis, pool, k, o);
+    launch_pdl(topk_kernel<SRC_FLAT>, nq, kTopkThreads, smem, st, c, scores, stride, q_seq, q_vis, pool, k, o);
   else if (src == SRC_BLOCKKEYS)
-    topk_kernel<SRC_BLOCKKEYS><<<nq, kTopkThreads, smem, st>>>(c, scores, stride, q_seq, q_vis, pool, k, o);
+    launch_pdl(topk_kernel<SRC_BLOCKKEYS>, nq, kTopkThreads, smem, st, c, scores, stride, q_seq, q_vis, pool, k, o);
   else if (src == SRC_POOL)
-    topk_kernel<SRC_POOL><<<nq, kTopkThreads, smem, st>>>(c, scores, stride, q_seq, q_vis, pool, k, o);
+    launch_pdl(topk_kernel<SRC_POOL>, nq, kTopkThreads, smem, st, c, scores, stride, q_seq, q_vis, pool, k, o);
   else
-    topk_kernel<SRC_CAND><<<nq, kTopkThreads, smem, st>>>(c, scores, stride, q_seq, q_vis, pool, k, o);
+    launch_pdl(topk_kernel<SRC_CAND>, nq, kTopkThreads, smem, st, c, scores, stride, q_seq, q_vis, pool, k, o);
   return cudaGetLastError();
 }
 

@@ -207,6 +207,8 @@ __global__ void __launch_bounds__(256) append_rows_kernel(CacheView c, const uin
                                                           const int32_t* __restrict__ eseq,
                                                           const int32_t* __restrict__ epos, int n,
                                                           int compress) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int i = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
   if (i >= n) return;
@@ -232,6 +234,8 @@ __global__ void __launch_bounds__(256) append_block_keys_kernel(CacheView c,
                                                                 const int32_t* __restrict__ eseq,
                                                                 const int32_t* __restrict__ epos,
                                                                 int n) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int i = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
   if (i >= n) return;
@@ -252,6 +256,8 @@ __global__ void __launch_bounds__(256) append_block_keys_kernel(CacheView c,
 __global__ void __launch_bounds__(256) replay_rows_kernel(CacheView c, const uint16_t* __restrict__ kv_last,
                                                           const uint16_t* __restrict__ idxk_last,
                                                           const uint8_t* __restrict__ miss, int compress) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int b = blockIdx.y;
   const int r = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
@@ -272,6 +278,8 @@ __global__ void __launch_bounds__(256) replay_rows_kernel(CacheView c, const uin
 
 // Replay block keys: warp (b, j) recomputes the j-th block touched in seq b.
 __global__ void __launch_bounds__(256) replay_block_keys_kernel(CacheView c, const uint8_t* __restrict__ miss) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int b = blockIdx.y;
   const int j = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
@@ -292,19 +300,19 @@ cudaError_t launch_append(const CacheView& c, const uint16_t* kv, const uint16_t
                           const int32_t* eseq, const int32_t* epos, int n, int compress,
                           cudaStream_t st) {
   const int grid = (n + kWarpsPerCta - 1) / kWarpsPerCta;
-  append_rows_kernel<<<grid, 256, 0, st>>>(c, kv, idxk, eseq, epos, n, compress);
-  append_block_keys_kernel<<<grid, 256, 0, st>>>(c, eseq, epos, n);
+  launch_pdl(append_rows_kernel, grid, 256, 0, st, c, kv, idxk, eseq, epos, n, compress);
+  launch_pdl(append_block_keys_kernel, grid, 256, 0, st, c, eseq, epos, n);
   return cudaGetLastError();
 }
 
 cudaError_t launch_replay(const CacheView& c, const uint16_t* kv_last, const uint16_t* idxk_last,
                           const uint8_t* miss, int compress, cudaStream_t st) {
   dim3 g1(kReplay / kWarpsPerCta, c.batch);
-  replay_rows_kernel<<<g1, 256, 0, st>>>(c, kv_last, idxk_last, miss, compress);
+  launch_pdl(replay_rows_kernel, g1, 256, 0, st, c, kv_last, idxk_last, miss, compress);
   if (c.swa) return cudaGetLastError();   // the global cache's keys are untouched
   // a 128-token window touches at most 17 blocks of 8
   dim3 g2((kReplay / kBlock + 1 + kWarpsPerCta - 1) / kWarpsPerCta, c.batch);
-  replay_block_keys_kernel<<<g2, 256, 0, st>>>(c, miss);
+  launch_pdl(replay_block_keys_kernel, g2, 256, 0, st, c, miss);
   return cudaGetLastError();
 }
 

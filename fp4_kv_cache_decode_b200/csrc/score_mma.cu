@@ -59,6 +59,8 @@ __global__ void __launch_bounds__(kSmThreads) score_mma_kernel(const __grid_cons
                                                                const int32_t* __restrict__ pool, int64_t max_units,
                                                                int64_t stride, int upc, float* __restrict__ scores,
                                                                float* __restrict__ block_max, int64_t bstride) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   const uint32_t raw = (uint32_t)__cvta_generic_to_shared(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;   // 1024-B aligned: the swizzle atoms of A and B
@@ -323,15 +325,15 @@ cudaError_t launch_score_mma(int src, const CacheView& c, const uint16_t* idx_q,
   dim3 grid((unsigned)((max_units + upc - 1) / upc), (unsigned)nq);
   if (grid.x == 0 || nq == 0) return cudaSuccess;
   if (src == SRC_FLAT)
-    score_mma_kernel<SRC_FLAT><<<grid, kSmThreads, kScoreMmaSmem, st>>>(m, c, idx_q, head_w, q_seq, q_vis, pool,
+    launch_pdl(score_mma_kernel<SRC_FLAT>, grid, kSmThreads, kScoreMmaSmem, st, m, c, idx_q, head_w, q_seq, q_vis, pool,
                                                                         max_units, stride, (int)upc, scores,
                                                                         block_max, bstride);
   else if (src == SRC_BLOCKKEYS)
-    score_mma_kernel<SRC_BLOCKKEYS><<<grid, kSmThreads, kScoreMmaSmem, st>>>(m, c, idx_q, head_w, q_seq, q_vis,
+    launch_pdl(score_mma_kernel<SRC_BLOCKKEYS>, grid, kSmThreads, kScoreMmaSmem, st, m, c, idx_q, head_w, q_seq, q_vis,
                                                                              pool, max_units, stride, (int)upc,
                                                                              scores, nullptr, 0);
   else
-    score_mma_kernel<SRC_POOL><<<grid, kSmThreads, kScoreMmaSmem, st>>>(m, c, idx_q, head_w, q_seq, q_vis, pool,
+    launch_pdl(score_mma_kernel<SRC_POOL>, grid, kSmThreads, kScoreMmaSmem, st, m, c, idx_q, head_w, q_seq, q_vis, pool,
                                                                         max_units, stride, (int)upc, scores,
                                                                         nullptr, 0);
   return cudaGetLastError();

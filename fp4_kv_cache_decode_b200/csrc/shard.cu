@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(256) shard_localize_kernel(CacheView c, const 
                                                              int32_t* __restrict__ lout,
                                                              const int32_t* __restrict__ wstart_g,
                                                              int32_t* __restrict__ wstart_l) {
+  pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   const int64_t off = shard_offset[r];
   const int64_t len = seq_len_of(c, q_seq[r]);
@@ -49,6 +51,8 @@ __global__ void __launch_bounds__(256) shard_localize_kernel(CacheView c, const 
 __global__ void shard_pack_kernel(const float* __restrict__ score, const int32_t* __restrict__ id, int nshard,
                                   int n, int64_t qs, int64_t ss, float* __restrict__ pscore,
                                   int32_t* __restrict__ pid) {
+  pdl_wait();
+  pdl_trigger();
   const int q = blockIdx.y;
   const int64_t m = (int64_t)nshard * n;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < m; i += (int64_t)gridDim.x * blockDim.x) {
@@ -66,6 +70,8 @@ __global__ void shard_pack_kernel(const float* __restrict__ score, const int32_t
 __global__ void __launch_bounds__(128) shard_combine_kernel(const uint16_t* __restrict__ part,
                                                             const float* __restrict__ lse2, int nshard, int H,
                                                             int64_t qs, int64_t ss, uint16_t* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   const int q = blockIdx.x, h = blockIdx.y;
   float M = -INFINITY;
   for (int s = 0; s < nshard; ++s) M = fmaxf(M, lse2[((int64_t)q * qs + s * ss) * H + h]);
@@ -97,7 +103,7 @@ cudaError_t launch_shard_localize(const CacheView& c, const int32_t* q_seq, cons
                                   const int32_t* gin, int n, int unit, int32_t* lout, const int32_t* wstart_g,
                                   int32_t* wstart_l, int nq, cudaStream_t st) {
   if (nq == 0) return cudaSuccess;
-  shard_localize_kernel<<<nq, 256, 0, st>>>(c, q_seq, shard_offset, gin, n, unit, lout, wstart_g, wstart_l);
+  launch_pdl(shard_localize_kernel, nq, 256, 0, st, c, q_seq, shard_offset, gin, n, unit, lout, wstart_g, wstart_l);
   return cudaGetLastError();
 }
 
@@ -106,14 +112,14 @@ cudaError_t launch_shard_pack(const float* score, const int32_t* id, int nshard,
   if (nq == 0) return cudaSuccess;
   const int64_t m = (int64_t)nshard * n;
   const int bx = (int)((m + 255) / 256 < 64 ? (m + 255) / 256 : 64);
-  shard_pack_kernel<<<dim3(bx, nq), 256, 0, st>>>(score, id, nshard, n, qs, ss, pscore, pid);
+  launch_pdl(shard_pack_kernel, dim3(bx, nq), 256, 0, st, score, id, nshard, n, qs, ss, pscore, pid);
   return cudaGetLastError();
 }
 
 cudaError_t launch_shard_combine(const uint16_t* part, const float* lse2, int nshard, int nq, int H, int64_t qs,
                                  int64_t ss, uint16_t* out, cudaStream_t st) {
   if (nq == 0) return cudaSuccess;
-  shard_combine_kernel<<<dim3(nq, H), kD / 4, 0, st>>>(part, lse2, nshard, H, qs, ss, out);
+  launch_pdl(shard_combine_kernel, dim3(nq, H), kD / 4, 0, st, part, lse2, nshard, H, qs, ss, out);
   return cudaGetLastError();
 }
 
