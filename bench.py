@@ -35,8 +35,8 @@ METRIC = "CSA2 decode layer-steps/s at 64K ctx; achieved HBM GB/s vs B200 peak"
 UNIT = "layer-steps/s"
 CONFIG_ID = 1
 # dram__bytes_read.sum + dram__bytes_write.sum of one attn_pipe_kernel launch on this
-# workload (ncu, three launches: 9.820, 9.815, 9.797 MB read, 0 written)
-ATTN_DRAM_BYTES_PER_LAUNCH = 9.81e6
+# workload (ncu, three launches: 9.709, 9.703, 9.800 MB read, 0 written)
+ATTN_DRAM_BYTES_PER_LAUNCH = 9.74e6
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -368,10 +368,12 @@ def run_gpu(args):
         "gpu_launches": args.steps * launches_per_step(w),
         "clocks": clocks,
     }
-    result["window_store"] = measure_window_store(w, cache, step, stream, flush, peaks, reuse_ms)
-    result["max_pooled_blocks"] = measure_max_pool(w, cache, step, stream, flush, peaks, idx_full_ms)
-    result["fp8_indexer_keys"] = measure_fp8_keys(
-        w, stream, flush, peaks, {"step": ms_per_step, "full": idx_full_ms, "reindex": idx_ri_ms})
+    if not args.no_extra_legs:   # diagnostics outside the timed region
+        result["window_store"] = measure_window_store(w, cache, step, stream, flush, peaks, reuse_ms)
+        result["max_pooled_blocks"] = measure_max_pool(w, cache, step, stream, flush, peaks, idx_full_ms)
+        result["fp8_indexer_keys"] = measure_fp8_keys(
+            w, stream, flush, peaks, {"step": ms_per_step, "full": idx_full_ms, "reindex": idx_ri_ms})
+        result["workloads"] = measure_workloads(stream, flush, rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args, seqs=tuple(range(w.batch)))
     finish_ranks(world)
@@ -496,6 +498,71 @@ def measure_max_pool(w, cache, step, stream, flush, peaks, mean_full_ms):
             "key_bytes": key_bytes, "gbs": gbs, "frac_of_hbm": gbs / peaks["hbm_gbs"],
             "mean_pooled_recall_of_exact_top512": recall,
             "note": "median of CUDA-graph replays, L2 flushed first; bytes = every visible bf16 key once"}
+
+
+def measure_workloads(stream, flush, seed_rank: int = 0):
+    """Throughput of the other seeded workloads on this GPU, outside the timed
+    region: each step captured once as a CUDA graph and replayed (median of 5, L2
+    flushed first); inputs generated before the graph.  A decode layer-step is
+    one layer over the whole batch; a prefill chunk is the chunk's append, its
+    flat indexer over 8,192 queries and its Full + 5 Reuse attention layers."""
+    import torch
+
+    import workload as wl
+    from workload import device as wdev
+    from fp4_kv_cache_decode_b200 import csa2, synthetic
+    out = {}
+    for cid in (0, 2, 4):
+        w = wl.workload(cid)
+        w.seed = rank_seed(w.seed, seed_rank)
+        cache = synthetic.new_cache(w)
+        synthetic.fill_decode_cache(w, cache)
+        if cid == 4:
+            step = synthetic.RaggedStep(w, cache)
+            step.setup()
+            layers = 1
+        else:
+            step = synthetic.DecodeStep(w, cache)
+            layers = len(w.layers)
+        step.run()
+        torch.cuda.synchronize()
+        assert csa2.csa2_check_device_error(cache) == 0
+        ms = _graph_ms(step.run, flush, stream)
+        out[f"config{cid}"] = {"workload": w.name, "step_ms": ms, "layer_steps_per_s": layers / (ms * 1e-3),
+                               "tokens_per_s": w.batch / (ms * 1e-3)}
+        del step, cache
+        torch.cuda.empty_cache()
+    # encoder chunked prefill: the last chunk (the longest visible prefix)
+    w = wl.workload(3)
+    w.seed = rank_seed(w.seed, seed_rank)
+    cache = synthetic.new_cache(w)
+    nchunk = w.raw_tokens // w.chunk
+    for ci in range(nchunk):
+        synthetic.fill_prefill_chunk(w, cache, ci)
+    ch = synthetic.PrefillChunk(w, cache, nchunk - 1)
+    r0 = (nchunk - 1) * w.chunk
+    col = torch.from_numpy(wl.kv_col_scale(w.seed)).cuda()
+    kv = wdev.kv_rows(w.seed, 0, r0, w.chunk, col_scale=col)
+    k = wdev.idxk_rows(w.seed, 0, r0, w.chunk)
+    n_e = w.chunk // w.compress
+    eseq = torch.zeros(n_e, dtype=torch.int32, device="cuda")
+    epos = torch.arange(r0 // w.compress, r0 // w.compress + n_e, dtype=torch.int32, device="cuda")
+    q = ch.queries(0).clone()
+
+    def chunk_step():
+        csa2.csa2_kv_quant_append(cache, kv, k, eseq, epos, w.compress)
+        ch.indexer()
+        for layer in range(len(w.layers)):
+            ch.attention(layer, q=q)
+    chunk_step()
+    torch.cuda.synchronize()
+    assert csa2.csa2_check_device_error(cache) == 0
+    ms = _graph_ms(chunk_step, flush, stream)
+    out["config3"] = {"workload": w.name, "step_ms": ms, "layer_steps_per_s": len(w.layers) / (ms * 1e-3),
+                      "tokens_per_s": w.chunk / (ms * 1e-3), "step": "one 8,192-token chunk"}
+    del ch, cache
+    torch.cuda.empty_cache()
+    return out
 
 
 def measure_fp8_keys(w, stream, flush, peaks, bf16_ms):
@@ -695,6 +762,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--pool-pages", action="store_true",
                     help="profiling case: size the paged pool to the batch (not a bench number)")
+    ap.add_argument("--no-extra-legs", action="store_true",
+                    help="skip the diagnostic legs after the timed step (window store, max-pooled blocks, "
+                         "FP8 keys, other workloads): profiling runs keep a few GB on the device")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
