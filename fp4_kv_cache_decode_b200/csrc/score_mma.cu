@@ -257,6 +257,232 @@ __global__ void __launch_bounds__(kSmThreads) score_mma_kernel(const __grid_cons
   }
 }
 
+// ---- flat scoring of query groups ----
+//
+// Many queries of one sequence (an encoder prefill chunk: consecutive positions,
+// visible lengths within a few entries of each other) share their keys: a CTA
+// takes 16 consecutive queries, and D[128 keys x 64] = K . Q^T with the 16
+// queries' 4 heads as the 64 columns, so each key tile is loaded once for all 16
+// and the tensor core does 16x the work per copy.  Each query masks the keys at
+// or beyond its own visible length.  A group whose queries are not all of one
+// sequence is scored one query per pass (same Q^T, that query's 4 columns).
+constexpr int kGrp = 16;                                 // queries per CTA
+constexpr int kGrpN = kGrp * kIdxHeads;                  // 64 = MMA N
+constexpr uint32_t kGrpTmemCols = kSmStages * kGrpN;     // 256
+constexpr uint32_t kGrOffA = 0;                          // [stages][16 KiB]
+constexpr uint32_t kGrOffB = kSmStages * kTileBytesS;    // Q^T [64 x 64] bf16, 8 KiB
+constexpr uint32_t kGrOffRow = kGrOffB + 8192;
+constexpr uint32_t kGrOffNr = kGrOffRow + 4 * kSmUnitsPerCta;
+constexpr uint32_t kGrOffQv = kGrOffNr + 4 * kSmUnitsPerCta;   // int64 visible length per query
+constexpr uint32_t kGrOffW = kGrOffQv + 8 * kGrp;              // float head weights [16][4]
+constexpr uint32_t kGrOffBar = kGrOffW + 4 * kGrpN;
+constexpr uint32_t kGrOffMisc = kGrOffBar + 8 * 3 * kSmStages;  // TMEM base, abort flag, one-sequence flag
+// two CTAs per SM hold 2 x 256 TMEM columns; the shared-memory request keeps a third off the SM
+constexpr uint32_t kGrpSmem = 232448 / 2 - 1024;
+static_assert(kGrOffMisc + 16 + 1024 <= kGrpSmem, "group layout");
+static_assert(2 * (kGrpSmem + 1024) <= 233472 && 3 * (kGrpSmem + 1024) > 233472, "two CTAs per SM");
+constexpr uint32_t kIdescGrp = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kGrpN >> 3) << 17) | ((128u >> 4) << 24);
+
+__global__ void __launch_bounds__(kSmThreads, 1) score_mma_group_kernel(
+    const __grid_constant__ CUtensorMap tmap, CacheView c, const uint16_t* __restrict__ idx_q,
+    const float* __restrict__ head_w, const int32_t* __restrict__ q_seq, const int32_t* __restrict__ q_vis, int nq,
+    int64_t max_units, int64_t stride, int upc, float* __restrict__ scores) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const uint32_t raw = (uint32_t)__cvta_generic_to_shared(smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t* const sp = smem_raw + (sb - raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int r0 = blockIdx.y * kGrp;
+  const int ng = nq - r0 < kGrp ? nq - r0 : kGrp;
+  int32_t* const urow = reinterpret_cast<int32_t*>(sp + kGrOffRow);
+  int32_t* const unr = reinterpret_cast<int32_t*>(sp + kGrOffNr);
+  int64_t* const qv = reinterpret_cast<int64_t*>(sp + kGrOffQv);
+  float* const wq = reinterpret_cast<float*>(sp + kGrOffW);
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(sp + kGrOffMisc + 4);
+  volatile int* const one_seq = reinterpret_cast<volatile int*>(sp + kGrOffMisc + 8);
+  auto full = [&](int s) { return sb + kGrOffBar + 8u * s; };
+  auto done = [&](int s) { return sb + kGrOffBar + 8u * (kSmStages + s); };
+  auto freed = [&](int s) { return sb + kGrOffBar + 8u * (2 * kSmStages + s); };
+
+  if (tid < kGrp) qv[tid] = tid < ng ? visible_of(c, q_seq, q_vis, r0 + tid) : -1;
+  if (tid < kGrpN)
+    wq[tid] = (head_w != nullptr && (tid >> 2) < ng) ? __ldg(head_w + (int64_t)(r0 + (tid >> 2)) * kIdxHeads + (tid & 3))
+                                                     : 1.0f;
+  if (warp == 0) {
+    const int32_t s0 = q_seq[r0];
+    const bool same = __all_sync(0xffffffffu, lane >= ng || q_seq[r0 + lane] == s0);
+    if (lane == 0) *one_seq = same ? 1 : 0;
+  }
+  // Q^T: row 4 q + h = head h of query q (zero rows past the group), 128-B swizzled K-major
+  for (int i = tid; i < kGrpN * 8; i += kSmThreads) {
+    const int n = i >> 3, ch = i & 7, q = n >> 2, h = n & 3;
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (q < ng) val = __ldg(reinterpret_cast<const uint4*>(idx_q + ((int64_t)(r0 + q) * kIdxHeads + h) * kIdxDim) + ch);
+    *reinterpret_cast<uint4*>(sp + kGrOffB + n * 128 + ((ch ^ (n & 7)) << 4)) = val;
+  }
+  fence_async_smem();
+  if (tid == 0) {
+    for (int s = 0; s < kSmStages; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(done(s), 1);
+      mbar_init(freed(s), 4);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 5) tmem_alloc_warp(sb + kGrOffMisc, kGrpTmemCols);
+  if (warp == 4 && lane == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap)) : "memory");
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sp + kGrOffMisc);
+  const bool uniform = *one_seq != 0;
+  const int npass = uniform ? 1 : ng;
+  const int64_t u0 = (int64_t)blockIdx.x * upc;
+  int tbase = 0;          // tiles of earlier passes: the stage / phase count runs on across passes
+  int issued = 0, mmas = 0;   // tiles copied / multiplied (for the drains)
+
+#pragma unroll 1
+  for (int pass = 0; pass < npass; ++pass) {
+    if (*abort_flag) break;   // read after a barrier: the same value in every thread
+    const int rq = uniform ? r0 : r0 + pass;
+    const int seq = q_seq[rq];
+    int64_t v = 0;
+    if (uniform) {
+      for (int q = 0; q < ng; ++q) v = qv[q] > v ? qv[q] : v;
+    } else {
+      v = qv[pass];
+    }
+    int64_t nunits = units_of(SRC_FLAT, v);
+    if (nunits > max_units) {
+      if (blockIdx.x == 0 && tid == 0) raise_error(c.err, CSA2_DEVERR_POS);
+      nunits = max_units;
+    }
+    const int nu = u0 < nunits ? (int)(nunits - u0 < upc ? nunits - u0 : upc) : 0;
+    const int ntiles = (nu + kTileUnits - 1) / kTileUnits;
+    for (int j = tid; j < kSmUnitsPerCta; j += kSmThreads) {
+      int32_t row = -1, nr = 0;
+      if (j < nu) {
+        const int64_t u = u0 + j;
+        const int64_t pg = page_of(c, seq, u * kBlock);
+        if (pg >= 0) {
+          row = (int32_t)(pg * kPageTokens + (u & (kBlocksPerPage - 1)) * kBlock);
+          nr = (int)(v - u * kBlock < kBlock ? v - u * kBlock : kBlock);
+        }
+      }
+      urow[j] = row;
+      unr[j] = nr;
+    }
+    __syncthreads();
+
+    if (warp == 4) {
+      // ---- producer warp: one 64-key box (a whole page) per lane 0 / 1 of each tile ----
+      for (int t = 0; t < ntiles; ++t) {
+        if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+        const int tg = tbase + t, s = tg % kSmStages, n = tg / kSmStages;
+        bool ok = true;
+        if (n > 0) ok = __all_sync(0xffffffffu, lane != 0 || mbar_wait(freed(s), (n - 1) & 1));
+        if (!ok) {
+          if (lane == 0) {
+            *abort_flag = 1;
+            raise_error(c.err, CSA2_DEVERR_TIMEOUT);
+          }
+          break;
+        }
+        const int uj = t * kTileUnits + lane * kBlocksPerPage;
+        const int32_t row = (lane < kTileUnits / kBlocksPerPage && uj < nu) ? urow[uj] : -1;
+        const uint32_t mask = __ballot_sync(0xffffffffu, row >= 0);
+        if (lane == 0) mbar_arrive_expect_tx(full(s), (uint32_t)__popc(mask) * 1024u * kBlocksPerPage);
+        __syncwarp();
+        if (row >= 0)
+          tma_load_2d(sb + kGrOffA + (uint32_t)s * kTileBytesS + (uint32_t)(lane * kBlocksPerPage) * 1024u, &tmap, 0,
+                      row, full(s));
+        __syncwarp();
+        ++issued;
+      }
+    } else if (warp == 5) {
+      // ---- MMA issue ----
+      if (lane == 0) {
+        const uint64_t bdesc = smem_desc(sb + kGrOffB, 16, 1024);
+        for (int t = 0; t < ntiles; ++t) {
+          if (*abort_flag) break;
+          const int tg = tbase + t, s = tg % kSmStages, n = tg / kSmStages;
+          bool ok = mbar_wait(full(s), n & 1);
+          if (ok && n > 0) ok = mbar_wait(freed(s), (n - 1) & 1);
+          if (!ok) {
+            *abort_flag = 1;
+            raise_error(c.err, CSA2_DEVERR_TIMEOUT);
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc(sb + kGrOffA + (uint32_t)s * kTileBytesS, 16, 1024);
+#pragma unroll
+          for (int k = 0; k < kIdxDim / 16; ++k)
+            mma_f16(tmem + (uint32_t)s * kGrpN, adesc + 2u * k, bdesc + 2u * k, kIdescGrp, k > 0 ? 1u : 0u);
+          mma_commit(done(s));
+          ++mmas;
+        }
+      }
+    } else {
+      // ---- epilogue: warps 0..3 own TMEM lanes 32 warp .. 32 warp + 31 ----
+      const int row = 32 * warp + lane;
+      for (int t = 0; t < ntiles; ++t) {
+        if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+        const int tg = tbase + t, s = tg % kSmStages, n = tg / kSmStages;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(done(s), n & 1));
+        if (!ok) {
+          if (lane == 0) {
+            *abort_flag = 1;
+            raise_error(c.err, CSA2_DEVERR_TIMEOUT);
+          }
+          break;
+        }
+        tc_fence_after();
+        const int j = t * kTileUnits + (row >> 3);
+        const bool in = j < nu;
+        const int64_t pos = (u0 + j) * kBlock + (row & 7);
+        const bool key_ok = in && (row & 7) < unr[in ? j : 0];
+        const uint32_t tbase_addr = tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)s * kGrpN;
+        const int q_lo = uniform ? 0 : pass, q_hi = uniform ? ng : pass + 1;
+#pragma unroll 1
+        for (int q4 = q_lo & ~3; q4 < q_hi; q4 += 4) {   // 4 queries (16 columns) per load
+          float d[16];
+          tmem_ld16(tbase_addr + 4u * q4, d);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int q = q4 + k;
+            if (q < q_lo || q >= q_hi) continue;
+            const float* w = wq + 4 * q;
+            float sc = __fmul_rn(w[0], fmaxf(d[4 * k], 0.0f));
+            sc = __fadd_rn(sc, __fmul_rn(w[1], fmaxf(d[4 * k + 1], 0.0f)));
+            sc = __fadd_rn(sc, __fmul_rn(w[2], fmaxf(d[4 * k + 2], 0.0f)));
+            sc = __fadd_rn(sc, __fmul_rn(w[3], fmaxf(d[4 * k + 3], 0.0f)));
+            if (in) scores[(int64_t)(r0 + q) * stride + pos] = (key_ok && pos < qv[q]) ? sc : -INFINITY;
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(freed(s));
+      }
+    }
+    tbase += ntiles;
+    __syncthreads();   // the next pass rewrites the unit lists
+  }
+  // drains: every issued copy has landed and every MMA has finished before the exit
+  if (warp == 4 && lane == 0)
+    for (int k = (issued > kSmStages ? issued - kSmStages : 0); k < issued; ++k)
+      mbar_wait(full(k % kSmStages), (k / kSmStages) & 1);
+  if (warp == 5 && lane == 0 && mmas > 0) mbar_wait(done((mmas - 1) % kSmStages), ((mmas - 1) / kSmStages) & 1);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc_warp(tmem, kGrpTmemCols);
+  }
+}
+
 // ---- host side ----
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
@@ -300,6 +526,8 @@ cudaError_t score_mma_set_attributes() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(score_mma_kernel<SRC_POOL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kScoreMmaSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(score_mma_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGrpSmem);
   return e;
 }
 
@@ -316,6 +544,21 @@ cudaError_t launch_score_mma(int src, const CacheView& c, const uint16_t* idx_q,
   if (!ok) return cudaErrorInvalidValue;
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (src == SRC_FLAT && block_max == nullptr && nq >= 2 * kGrp) {
+    // groups of 16 queries (two CTAs per SM)
+    const int ngroups = (nq + kGrp - 1) / kGrp;
+    int64_t per_group = ((int64_t)2 * sms) / ngroups;
+    if (per_group < 1) per_group = 1;
+    int64_t gupc = (max_units + per_group - 1) / per_group;
+    gupc = (gupc + kTileUnits - 1) / kTileUnits * kTileUnits;
+    if (gupc > kSmUnitsPerCta) gupc = kSmUnitsPerCta;
+    if (gupc < kTileUnits) gupc = kTileUnits;
+    const dim3 ggrid((unsigned)((max_units + gupc - 1) / gupc), (unsigned)ngroups);
+    if (ggrid.x == 0) return cudaSuccess;
+    launch_pdl(score_mma_group_kernel, ggrid, kSmThreads, kGrpSmem, st, m, c, idx_q, head_w, q_seq, q_vis, nq,
+               max_units, stride, (int)gupc, scores);
+    return cudaGetLastError();
+  }
   int64_t per_query = nq > 0 ? ((int64_t)3 * sms) / nq : 1;
   if (per_query < 1) per_query = 1;
   int64_t upc = (max_units + per_query - 1) / per_query;

@@ -99,3 +99,40 @@ def test_topk_on_ties_equal_and_signed_scores(crafted):
         _, idx, _ = oidx.full_indexer(iq[b], keys[b], L, w=hw[b], hierarchical=False)
         parity.check_index_set(gflat[b], idx, lambda x: oidx.index_scores(iq[b], keys[b][np.asarray(x)], hw[b]),
                                f"flat {CASES[b]} L={L}")
+
+
+def test_flat_query_groups_uniform_and_mixed(csa2_lib):
+    """Flat (encoder) selection with 48 queries, scored in groups of 16 that share
+    their keys when a group's queries are of one sequence: a group on one sequence
+    with staggered visible lengths, a group interleaving five sequences (scored
+    query by query), and a ragged last group crossing into another sequence."""
+    import workload
+    workload.build_cuda()
+    from fp4_kv_cache_decode_b200 import synthetic as syn
+    from workload import device as wdev
+    csa2 = csa2_lib
+    lens = [20000, 3000, 16400, 9000, 700]
+    w = small_workload(lens, seed=29, heads=16)
+    cache = syn.new_cache(w)
+    syn.fill_decode_cache(w, cache)
+    seqs = [0] * 16 + [r % 5 for r in range(16)] + [3] * 10 + [4] * 6
+    vis = ([19000 + 7 * r for r in range(16)] + [lens[s] for s in seqs[16:32]] +
+           [9000 - 13 * r for r in range(10)] + [700, 1, 0, 8, 9, 511])
+    nq = len(seqs)
+    q_seq = torch.tensor(seqs, dtype=torch.int32, device="cuda")
+    q_vis = torch.tensor(vis, dtype=torch.int32, device="cuda")
+    idxq = torch.cat([wdev.idxq_batch(w.seed, 9, r, 1) for r in range(nq)])
+    iset = csa2.IndexSet(nq)
+    ws = torch.empty(csa2.csa2_workspace_bytes(csa2.OP_INDEXER, nq, 0, max(vis), 0), dtype=torch.uint8,
+                     device="cuda")
+    csa2.csa2_indexer_score_topk(cache, idxq, q_seq, csa2.FULL, 0, iset, ws, max(vis), q_visible=q_vis,
+                                 hierarchical=False)
+    assert csa2.csa2_check_device_error(cache) == 0
+    gidx = iset.idx.cpu().numpy()
+    keys = {s: parity.OracleSeq(w, s, lens[s]).keys for s in set(seqs)}
+    for r in range(nq):
+        iq = wl.idxq_rows(w.seed, 9, r)
+        k = keys[seqs[r]]
+        _, idx, _ = oidx.full_indexer(iq, k, vis[r], hierarchical=False)
+        parity.check_index_set(gidx[r], idx, lambda x: oidx.index_scores(iq, k[np.asarray(x)]),
+                               f"query {r} seq {seqs[r]} v={vis[r]}")
