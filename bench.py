@@ -364,7 +364,9 @@ def run_gpu(args):
         "ms_graph": {"attention_launch": reuse_ms, "indexer_full": idx_full_ms, "indexer_reindex": idx_ri_ms},
         "roofline": dom,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
-                "d2h_bytes_per_step": e2e["d2h"]},
+                "d2h_bytes_per_step": e2e["d2h"],
+                "note": "copies of step k+1 (up) and k-1 (down) on two copy streams overlap step k's compute; "
+                        "L2 flushed before every step inside the timed region"},
         "gpu_launches": args.steps * launches_per_step(w),
         "clocks": clocks,
     }
@@ -620,40 +622,67 @@ def launches_per_step(w) -> int:
 
 
 def run_e2e(args, w, step, stream, flush):
-    """Same step through the C ABI, inputs copied from pinned host memory and the
-    outputs read back every step, all inside the timed region."""
+    """Same step through the C ABI as a serving loop runs it: every step copies its
+    inputs from pinned host memory and reads its outputs back, inside the timed
+    region, with the copies pipelined against the compute -- step k+1's inputs go
+    up (one copy stream) and step k-1's outputs come down (another) while step k
+    computes, two sets of device buffers alternating.  The L2 flush before each
+    step's compute stays in the timed region (the bench repeats identical steps)."""
     import torch
-    host_in = {"new_kv": step.new_kv, "new_k": step.new_k}
-    for i, q in enumerate(step.q):
-        host_in[f"q{i}"] = q
-    for i, q in step.idxq.items():
-        host_in[f"iq{i}"] = q
-    pinned = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in host_in.items()}
-    for k, v in host_in.items():
+
+    from fp4_kv_cache_decode_b200 import synthetic
+    sets = [step, synthetic.DecodeStep(w, step.cache)]
+
+    def inputs(st):
+        d = {"new_kv": st.new_kv, "new_k": st.new_k}
+        for i, q in enumerate(st.q):
+            d[f"q{i}"] = q
+        for i, q in st.idxq.items():
+            d[f"iq{i}"] = q
+        return d
+    pinned = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in inputs(step).items()}
+    for k, v in inputs(step).items():
         pinned[k].copy_(v)
-    outs = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in step.out]
+    outs = [[torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in st.out] for st in sets]
     h2d = sum(v.numel() * v.element_size() for v in pinned.values())
-    d2h = sum(o.numel() * o.element_size() for o in outs)
-    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    d2h = sum(o.numel() * o.element_size() for o in outs[0])
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
 
-    def one():
-        for k, v in host_in.items():
-            v.copy_(pinned[k], non_blocking=True)
-        step.run()
-        for o, h in zip(step.out, outs):
-            h.copy_(o, non_blocking=True)
+    def pipeline(n: int):
+        ev = lambda: torch.cuda.Event()
+        ready, done, back = [ev() for _ in range(n)], [ev() for _ in range(n)], [ev() for _ in range(n)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(up)
+        stream.wait_event(t0)
+        down.wait_event(t0)
+        for k in range(n):
+            st = sets[k % 2]
+            with torch.cuda.stream(up):   # inputs of step k (its buffer set was last used by step k-2)
+                if k >= 2:
+                    up.wait_event(done[k - 2])
+                for name, t in inputs(st).items():
+                    t.copy_(pinned[name], non_blocking=True)
+                ready[k].record(up)
+            stream.wait_event(ready[k])
+            if k >= 2:
+                stream.wait_event(back[k - 2])   # step k-2's outputs (same set) are read back
+            flush.fill_(k & 0xFF)
+            st.run()
+            done[k].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(done[k])
+                for o, h in zip(st.out, outs[k % 2]):
+                    h.copy_(o, non_blocking=True)
+                back[k].record(down)
+        down.wait_event(done[n - 1])
+        t1.record(down)
+        return t0, t1
 
-    for _ in range(max(1, args.warmup)):
-        one()
+    pipeline(max(3, args.warmup))
     torch.cuda.synchronize()
-    for k in range(args.steps):
-        flush.fill_(k & 0xFF)
-        ev0[k].record(stream)
-        one()
-        ev1[k].record(stream)
+    t0, t1 = pipeline(args.steps)
     torch.cuda.synchronize()
-    ms = sum(ev0[k].elapsed_time(ev1[k]) for k in range(args.steps))
+    ms = t0.elapsed_time(t1)
     return {"ms": ms, "h2d": h2d, "d2h": d2h}
 
 
