@@ -14,11 +14,11 @@
 // tokens' 512 code bytes plus their 32 scale bytes, and a key scores
 // s x score(q, code values) -- s >= 0 commutes with the ReLU.
 //
-// Scoring is HBM-bound (4 heads x 64 dims = 4 FLOP per key byte): each warp
-// streams whole units with 16-B non-allocating loads, several units in flight
-// per lane; lane l holds 16 dims of row l/4, so a row's four partial dot
-// products meet in two shuffles.  Scores go to the caller's workspace (4 B
-// per 128-B key) and a second kernel selects the top k.
+// Scoring of bf16 keys runs on the tensor cores (score_mma.cu).  The kernel
+// here scores FP8 keys on the FMA pipes: each warp streams whole units through
+// a cp.async ring, lane l holds 16 dims of row l/4 (E4M3 pairs converted to
+// fp32), so a row's four partial dot products meet in two shuffles.  Scores go
+// to the caller's workspace (4 B per key) and a second kernel selects the top k.
 //
 // Top-k: one CTA per query.  Keys are the order-preserving uint32 image of
 // the scores (-inf, the "not a candidate" marker, maps to 0).  A 12/12/8-bit
@@ -738,10 +738,8 @@ cudaError_t launch_score_mma(int src, const CacheView& c, const uint16_t* idx_q,
 cudaError_t indexer_set_attributes() {
   const int smem = (int)topk_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(topk_kernel<SRC_FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  const void* score_kernels[] = {
-      (const void*)score_units_kernel<SRC_FLAT, false>, (const void*)score_units_kernel<SRC_FLAT, true>,
-      (const void*)score_units_kernel<SRC_BLOCKKEYS, false>, (const void*)score_units_kernel<SRC_POOL, false>,
-      (const void*)score_units_kernel<SRC_POOL, true>};
+  const void* score_kernels[] = {(const void*)score_units_kernel<SRC_FLAT, true>,
+                                 (const void*)score_units_kernel<SRC_POOL, true>};
   for (const void* k : score_kernels)
     if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmemMax);
   if (e == cudaSuccess) e = score_mma_set_attributes();
@@ -759,35 +757,31 @@ cudaError_t launch_score(int src, const CacheView& c, const uint16_t* idx_q, con
                          const int32_t* q_seq, const int32_t* q_vis, const int32_t* pool, int nq,
                          int64_t max_units, int64_t stride, float* scores, float* block_max,
                          int64_t bstride, cudaStream_t st) {
-  // units per CTA: enough CTAs for two per SM over the whole batch, in whole
-  // 32-unit stages, at most 256
-  const bool f8 = c.idxk_fp8 && src != SRC_BLOCKKEYS;
-  // bf16 keys: tensor-core scoring (score_mma.cu); FP8 keys: the FFMA kernel below
-  if (!f8)
+  // bf16 keys (and block keys, always bf16): tensor-core scoring (score_mma.cu);
+  // FP8 keys: the FFMA kernel below
+  if (!c.idxk_fp8 || src == SRC_BLOCKKEYS)
     return launch_score_mma(src, c, idx_q, head_w, q_seq, q_vis, pool, nq, max_units, stride, scores, block_max,
                             bstride, st);
+  // units per CTA: enough CTAs for two per SM over the whole batch, in whole
+  // 32-unit stages, at most 256
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   int64_t per_query = nq > 0 ? ((int64_t)2 * sms) / nq : 1;   // CTAs per query that fit in one wave
   if (per_query < 1) per_query = 1;
   int64_t upc = (max_units + per_query - 1) / per_query;
-  const int stage_units = f8 ? ScoreGeom<true>::kUnits : ScoreGeom<false>::kUnits;
-  const uint32_t smem = f8 ? ScoreGeom<true>::kSmem : ScoreGeom<false>::kSmem;
+  const int stage_units = ScoreGeom<true>::kUnits;
+  const uint32_t smem = ScoreGeom<true>::kSmem;
   upc = (upc + stage_units - 1) / stage_units * stage_units;
   if (upc > kUnitsPerCta) upc = kUnitsPerCta;
   if (upc < stage_units) upc = stage_units;
   dim3 grid((unsigned)((max_units + upc - 1) / upc), (unsigned)nq);
   if (grid.x == 0) return cudaSuccess;
-  if (src == SRC_BLOCKKEYS)
-    launch_pdl(score_units_kernel<SRC_BLOCKKEYS, false>, grid, kScoreThreads, smem, st, c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
-  else if (src == SRC_FLAT && f8)
-    launch_pdl(score_units_kernel<SRC_FLAT, true>, grid, kScoreThreads, smem, st, c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
-  else if (src == SRC_FLAT)
-    launch_pdl(score_units_kernel<SRC_FLAT, false>, grid, kScoreThreads, smem, st, c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
-  else if (f8)
-    launch_pdl(score_units_kernel<SRC_POOL, true>, grid, kScoreThreads, smem, st, c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
+  if (src == SRC_FLAT)
+    launch_pdl(score_units_kernel<SRC_FLAT, true>, grid, kScoreThreads, smem, st, c, idx_q, head_w, q_seq, q_vis,
+               pool, max_units, stride, (int)upc, scores, block_max, bstride);
   else
-    launch_pdl(score_units_kernel<SRC_POOL, false>, grid, kScoreThreads, smem, st, c, idx_q, head_w, q_seq, q_vis, pool, max_units, stride, (int)upc, scores, block_max, bstride);
+    launch_pdl(score_units_kernel<SRC_POOL, true>, grid, kScoreThreads, smem, st, c, idx_q, head_w, q_seq, q_vis,
+               pool, max_units, stride, (int)upc, scores, block_max, bstride);
   return cudaGetLastError();
 }
 
