@@ -1,6 +1,7 @@
 // C ABI of the CSA2 library: host-side validation, mode-order checks and
 // kernel launches.  No allocation, no host synchronisation (except in
 // csa2_check_device_error); every launch goes to the caller's stream.
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -17,7 +18,7 @@ cudaError_t launch_score(int, const CacheView&, const uint16_t*, const float*, c
                          cudaStream_t);
 cudaError_t launch_topk(int, const CacheView&, const float*, int64_t, const int32_t*, const int32_t*,
                         const int32_t*, int, int, int32_t*, int64_t, cudaStream_t, float* = nullptr,
-                        const int32_t* = nullptr, int = 0);
+                        const int32_t* = nullptr, int = 0, int = 1);
 cudaError_t indexer_set_attributes();
 cudaError_t launch_shard_localize(const CacheView&, const int32_t*, const int32_t*, const int32_t*, int, int,
                                   int32_t*, const int32_t*, int32_t*, int, cudaStream_t);
@@ -90,6 +91,49 @@ int from_cuda(cudaError_t e) { return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Score-buffer stride (floats per query) of an indexer call.
+// Long rows (more entries than one top-k CTA holds in registers) are selected
+// in segments of kSegLen entries, one CTA each, whose nseg x k candidates
+// (score, id) are merged by one more top-k -- exact, and ties still go to the
+// lowest position since the segments' lists concatenate in ascending order.
+// Used when the candidates fit one CTA and the rows alone would leave most SMs
+// idle (fewer than kSegMaxRows queries: 4 x 1M decode rows go from 4 CTAs to 32);
+// otherwise the streaming top-k runs (an 8,192-query prefill chunk already fills
+// the GPU with one CTA per row, and segmenting it was measured slower).
+constexpr int64_t kSegLen = 16384;
+constexpr int kSegMaxRows = 256;
+
+int seg_count(int64_t n_max, int k, int nq) {
+  if (n_max <= kSegLen || nq >= kSegMaxRows) return 0;
+  const int64_t nseg = (n_max + kSegLen - 1) / kSegLen;
+  return nseg * k <= kSegLen ? (int)nseg : 0;
+}
+
+size_t seg_bytes(int nq, int64_t n_max, int k) {
+  const int nseg = seg_count(n_max, k, nq);
+  return nseg ? (size_t)nq * nseg * k * 8 : 0;
+}
+
+// Top-k of rows of up to n_max entries, segmented when seg_count() says so;
+// cand: workspace for the segments' candidates (seg_bytes()).
+cudaError_t select_topk(int src, const CacheView& v, const float* scores, int64_t stride, const int32_t* q_seq,
+                        const int32_t* q_vis, const int32_t* pool, int nq, int k, int32_t* out,
+                        int64_t out_stride, cudaStream_t s, int64_t n_max, void* cand,
+                        float* out_scores = nullptr, const int32_t* id_offset = nullptr, int shift = 0) {
+  const int nseg = seg_count(n_max, k, nq);
+  if (nseg == 0)
+    return launch_topk(src, v, scores, stride, q_seq, q_vis, pool, nq, k, out, out_stride, s, out_scores,
+                       id_offset, shift);
+  float* cs = static_cast<float*>(cand);
+  int32_t* ci = reinterpret_cast<int32_t*>(cs + (int64_t)nq * nseg * k);
+  cudaError_t e = launch_topk(src, v, scores, stride, q_seq, q_vis, pool, nq, k, ci, k, s, cs, id_offset, shift,
+                              nseg);
+  CacheView none{};
+  if (e == cudaSuccess)
+    e = launch_topk(kSrcCand, none, cs, (int64_t)nseg * k, nullptr, nullptr, ci, nq, k, out, out_stride, s,
+                    out_scores);
+  return e;
+}
+
 // Per-query floats of the indexer workspace: token (or block-key) scores, then,
 // for a max-pooled Full call, the block maxima at offset nq * flat stride.
 int64_t max_pool_block_stride(int64_t max_visible) {
@@ -98,6 +142,18 @@ int64_t max_pool_block_stride(int64_t max_visible) {
 
 size_t shard_attn_idx_offset(int nq, int heads) {
   return (attn_workspace_bytes(nq, heads) + 255) / 256 * 256;
+}
+
+int64_t indexer_stride(int64_t max_visible, int hierarchical);
+
+// Segment candidates of an indexer call (the largest of its selections).
+size_t indexer_seg_bytes(int nq, int64_t max_visible, int hierarchical) {
+  const int64_t flat_n = ceil_div(max_visible, kBlock) * kBlock;
+  const int64_t blocks_n = max_pool_block_stride(max_visible);
+  size_t b = 0;
+  if (hierarchical != CSA2_HIER_MEAN) b = seg_bytes(nq, flat_n, kTopK);                  // flat token top-k
+  if (hierarchical != CSA2_HIER_FLAT) b = std::max(b, seg_bytes(nq, blocks_n, kPoolBlocks));  // block top-k
+  return b;
 }
 
 int64_t indexer_stride(int64_t max_visible, int hierarchical) {
@@ -195,21 +251,22 @@ int csa2_indexer_score_topk(const csa2_cache* cache, const uint16_t* idx_q, cons
       // maximum; the pool is the 2,048 best maxima, the tokens the flat top-512
       float* bmax = scores + (int64_t)nq * stride;
       const int64_t bstride = max_pool_block_stride(max_visible);
+      void* cand = bmax + (int64_t)nq * bstride;
       e = launch_score(kSrcFlat, v, idx_q, head_w, q_seq, q_visible, nullptr, nq, nb, stride, scores,
                        bmax, bstride, s);
       if (e == cudaSuccess)
-        e = launch_topk(kSrcBlockKeys, v, bmax, bstride, q_seq, q_visible, nullptr, nq, kPoolBlocks,
-                        set->pool_blocks, kPoolBlocks, s);
+        e = select_topk(kSrcBlockKeys, v, bmax, bstride, q_seq, q_visible, nullptr, nq, kPoolBlocks,
+                        set->pool_blocks, kPoolBlocks, s, bstride, cand);
       if (e == cudaSuccess)
-        e = launch_topk(kSrcFlat, v, scores, stride, q_seq, q_visible, nullptr, nq, kTopK, set->idx,
-                        kTopK, s);
+        e = select_topk(kSrcFlat, v, scores, stride, q_seq, q_visible, nullptr, nq, kTopK, set->idx, kTopK, s,
+                        nb * kBlock, cand);
     } else if (mode == CSA2_FULL && hier) {
       const int64_t bk_units = ceil_div(nb, kBlocksPerPage);
       e = launch_score(kSrcBlockKeys, v, idx_q, head_w, q_seq, q_visible, nullptr, nq, bk_units,
                        stride, scores, nullptr, 0, s);
       if (e == cudaSuccess)
-        e = launch_topk(kSrcBlockKeys, v, scores, stride, q_seq, q_visible, nullptr, nq,
-                        kPoolBlocks, set->pool_blocks, kPoolBlocks, s);
+        e = select_topk(kSrcBlockKeys, v, scores, stride, q_seq, q_visible, nullptr, nq, kPoolBlocks,
+                        set->pool_blocks, kPoolBlocks, s, bk_units * kBlocksPerPage, scores + (int64_t)nq * stride);
     }
     if (e == cudaSuccess && hier && !(mode == CSA2_FULL && hierarchical == CSA2_HIER_MAX)) {
       e = launch_score(kSrcPool, v, idx_q, head_w, q_seq, q_visible, set->pool_blocks, nq,
@@ -222,8 +279,8 @@ int csa2_indexer_score_topk(const csa2_cache* cache, const uint16_t* idx_q, cons
       e = launch_score(kSrcFlat, v, idx_q, head_w, q_seq, q_visible, nullptr, nq, nb, stride,
                        scores, nullptr, 0, s);
       if (e == cudaSuccess)
-        e = launch_topk(kSrcFlat, v, scores, stride, q_seq, q_visible, nullptr, nq, kTopK, set->idx,
-                        kTopK, s);
+        e = select_topk(kSrcFlat, v, scores, stride, q_seq, q_visible, nullptr, nq, kTopK, set->idx, kTopK, s,
+                        nb * kBlock, scores + (int64_t)nq * stride);
     }
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
   }
@@ -307,15 +364,16 @@ size_t csa2_workspace_bytes(int32_t op, int32_t nq, int32_t heads, int64_t max_v
     if (hierarchical < CSA2_HIER_FLAT || hierarchical > CSA2_HIER_MAX) return 0;
     int64_t per_query = indexer_stride(max_visible, hierarchical);
     if (hierarchical == CSA2_HIER_MAX) per_query += max_pool_block_stride(max_visible);
-    return (size_t)nq * (size_t)per_query * sizeof(float) + 256;
+    return (size_t)nq * (size_t)per_query * sizeof(float) + indexer_seg_bytes(nq, max_visible, hierarchical) + 256;
   }
   if (op == CSA2_OP_ATTENTION) {
     if (heads != 16 && heads != 32 && heads != 48 && heads != 64) return 0;
     return attn_workspace_bytes(nq, heads);
   }
-  if (op == CSA2_OP_SHARD_INDEXER) {   // scores, then the local pool
+  if (op == CSA2_OP_SHARD_INDEXER) {   // scores, the local pool, segment candidates
     if (max_visible < 0) return 0;
-    return (size_t)nq * (size_t)(indexer_stride(max_visible, CSA2_HIER_MEAN) + kPoolBlocks) * 4 + 256;
+    return (size_t)nq * (size_t)(indexer_stride(max_visible, CSA2_HIER_MEAN) + kPoolBlocks) * 4 +
+           seg_bytes(nq, max_pool_block_stride(max_visible), kPoolBlocks) + 256;
   }
   if (op == CSA2_OP_SHARD_MERGE) {     // heads = shards, max_visible = candidates per shard
     if (heads < 1 || max_visible < 8 || max_visible % 8 != 0) return 0;
@@ -357,8 +415,9 @@ int csa2_shard_indexer_candidates(const csa2_cache* cache, const uint16_t* idx_q
     e = launch_score(kSrcBlockKeys, v, idx_q, head_w, q_seq, nullptr, nullptr, nq, bk_units, stride, scores,
                      nullptr, 0, s);
     if (e == cudaSuccess)
-      e = launch_topk(kSrcBlockKeys, v, scores, stride, q_seq, nullptr, nullptr, nq, kPoolBlocks, cand_id,
-                      kPoolBlocks, s, cand_score, shard_offset, 3);
+      e = select_topk(kSrcBlockKeys, v, scores, stride, q_seq, nullptr, nullptr, nq, kPoolBlocks, cand_id,
+                      kPoolBlocks, s, bk_units * kBlocksPerPage,
+                      scores + (int64_t)nq * (stride + kPoolBlocks), cand_score, shard_offset, 3);
   } else {
     int32_t* lpool = reinterpret_cast<int32_t*>(scores + (int64_t)nq * stride);
     e = launch_shard_localize(v, q_seq, shard_offset, global_pool, kPoolBlocks, kBlock, lpool, nullptr, nullptr,

@@ -41,6 +41,9 @@ struct TopkOut {
   float* scores;
   const int32_t* id_offset;
   int offset_shift;
+  int nseg;   // > 1: CTA b takes segment b % nseg (seg_len entries) of row b / nseg and
+              // writes its own output row b (ids offset by the segment's start)
+  int seg_len;
 };
 
 // Inverse of score_key on non-zero keys (exact; -0 comes back as +0).
@@ -591,17 +594,20 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(CacheView c, const f
   extern __shared__ __align__(16) uint8_t smem_raw[];
   TopkSmem* sm = reinterpret_cast<TopkSmem*>(smem_raw);
 
-  const int r = blockIdx.x;
+  const int r = out.nseg > 1 ? (int)(blockIdx.x / out.nseg) : (int)blockIdx.x;
+  const int64_t seg0 = out.nseg > 1 ? (int64_t)(blockIdx.x % out.nseg) * out.seg_len : 0;
   const int tid = threadIdx.x;
-  // candidates: every entry of the row (a multiple of 8), ids from `pool`
-  const int64_t n = SRC == SRC_CAND ? stride
-                                    : min(units_of(SRC, visible_of(c, q_seq, q_vis, r)) * kBlock, stride);
-  const float* srow = scores + (int64_t)r * stride;
+  // candidates: every entry of the row (a multiple of 8), ids from `pool`; a
+  // segment: entries [seg0, seg0 + seg_len) of it
+  int64_t n = SRC == SRC_CAND ? stride
+                              : min(units_of(SRC, visible_of(c, q_seq, q_vis, r)) * kBlock, stride);
+  if (out.nseg > 1) n = n - seg0 < 0 ? 0 : (n - seg0 < out.seg_len ? n - seg0 : out.seg_len);
+  const float* srow = scores + (int64_t)r * stride + seg0;
   const int32_t* pool_row =
       pool ? pool + (int64_t)r * (SRC == SRC_CAND ? stride : (int64_t)kPoolBlocks) : nullptr;
-  int32_t* orow = out.ids + (int64_t)r * out.stride;
-  float* oscore = out.scores ? out.scores + (int64_t)r * out.stride : nullptr;
-  const int32_t id_off = out.id_offset ? (out.id_offset[r] >> out.offset_shift) : 0;
+  int32_t* orow = out.ids + (int64_t)blockIdx.x * out.stride;
+  float* oscore = out.scores ? out.scores + (int64_t)blockIdx.x * out.stride : nullptr;
+  const int32_t id_off = (out.id_offset ? (out.id_offset[r] >> out.offset_shift) : 0) + (int32_t)seg0;
   if (n <= kTopkSmemKeys) {
     topk_registers<SRC>(srow, n, k, pool_row, orow, oscore, id_off, sm);
     return;
@@ -788,10 +794,12 @@ cudaError_t launch_score(int src, const CacheView& c, const uint16_t* idx_q, con
 cudaError_t launch_topk(int src, const CacheView& c, const float* scores, int64_t stride,
                         const int32_t* q_seq, const int32_t* q_vis, const int32_t* pool, int nq,
                         int k, int32_t* out, int64_t out_stride, cudaStream_t st, float* out_scores,
-                        const int32_t* id_offset, int offset_shift) {
+                        const int32_t* id_offset, int offset_shift, int nseg) {
   const size_t smem = topk_smem_bytes();
   if (nq == 0) return cudaSuccess;
-  const TopkOut o{out, out_stride, out_scores, id_offset, offset_shift};
+  // nseg > 1: one CTA per segment of kTopkSmemKeys entries; output rows nq x nseg
+  const TopkOut o{out, out_stride, out_scores, id_offset, offset_shift, nseg > 1 ? nseg : 1, kTopkSmemKeys};
+  if (nseg > 1) nq *= nseg;
   if (src == SRC_FLAT)
     launch_pdl(topk_kernel<SRC_FLAT>, nq, kTopkThreads, smem, st, c, scores, stride, q_seq, q_vis, pool, k, o);
   else if (src == SRC_BLOCKKEYS)

@@ -45,10 +45,13 @@ def test_workspace_sizes(csa2_lib):
     ws = csa2_lib.csa2_workspace_bytes
     # hierarchical decode at 64K: max(8192 block scores, 16384 pool scores) per query
     assert ws(1, 32, 0, 65536, True) == 32 * 16384 * 4 + 256
-    # 1M: 131072 block scores per query dominate
-    assert ws(1, 4, 0, 1048576, True) == 4 * 131072 * 4 + 256
-    # flat encoder chunk: 8192 queries x 65536 entries
+    # 1M: 131072 block scores per query dominate; the block top-2048 runs in 8
+    # segments of 16384 whose candidates (8 x 2048 x 8 B per query) follow the scores
+    assert ws(1, 4, 0, 1048576, True) == 4 * 131072 * 4 + 4 * 8 * 2048 * 8 + 256
+    # flat encoder chunk: 8192 queries x 65536 entries (enough rows to fill the GPU:
+    # one streaming top-k per row, no segments); 32 queries: 4 segments each
     assert ws(1, 8192, 0, 65536, False) == 8192 * 65536 * 4 + 256
+    assert ws(1, 32, 0, 65536, False) == 32 * 65536 * 4 + 32 * 4 * 512 * 8 + 256
     # attention: 32 queries split 4 ways (4 x 32 <= 148 SMs) exchange f16 partials
     # [4][64][512]; 148 queries are not split
     assert ws(2, 32, 64, 0, False) == 32 * 4 * 64 * 512 * 2 + 256
@@ -57,7 +60,7 @@ def test_workspace_sizes(csa2_lib):
     assert ws(2, 32, 20, 0, False) == 0          # unsupported head count
     assert ws(7, 1, 64, 0, False) == 0
     # max-pooled hierarchy: every token's score, then the 8,192 block maxima
-    assert ws(1, 32, 0, 65536, 2) == 32 * (65536 + 8192) * 4 + 256
+    assert ws(1, 32, 0, 65536, 2) == 32 * (65536 + 8192) * 4 + 32 * 4 * 512 * 8 + 256
     assert ws(1, 3, 0, 100, 2) == 3 * (104 + 16) * 4 + 256
     assert ws(1, 32, 0, 65536, 3) == 0
 

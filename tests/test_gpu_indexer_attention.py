@@ -76,7 +76,7 @@ def test_full_and_reindex_sets(ragged):
     print(f"allowed boundary swaps: {swaps}")
 
 
-@pytest.mark.parametrize("heads", [64, 16])
+@pytest.mark.parametrize("heads", [64, 48, 32, 16])
 def test_attention_on_oracle_sets(ragged, heads):
     """Attention alone: the oracle's index sets are loaded into the GPU set, so any
     difference is the attention kernel's."""
