@@ -633,19 +633,17 @@ def run_e2e(args, w, step, stream, flush):
     from fp4_kv_cache_decode_b200 import synthetic
     sets = [step, synthetic.DecodeStep(w, step.cache)]
 
-    def inputs(st):
-        d = {"new_kv": st.new_kv, "new_k": st.new_k}
-        for i, q in enumerate(st.q):
-            d[f"q{i}"] = q
+    def inputs(st):   # the layers' queries travel as one tensor
+        d = {"new_kv": st.new_kv, "new_k": st.new_k, "q": st.q_all}
         for i, q in st.idxq.items():
             d[f"iq{i}"] = q
         return d
     pinned = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in inputs(step).items()}
     for k, v in inputs(step).items():
         pinned[k].copy_(v)
-    outs = [[torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in st.out] for st in sets]
+    outs = [torch.empty(st.out_all.shape, dtype=st.out_all.dtype, pin_memory=True) for st in sets]
     h2d = sum(v.numel() * v.element_size() for v in pinned.values())
-    d2h = sum(o.numel() * o.element_size() for o in outs[0])
+    d2h = outs[0].numel() * outs[0].element_size()
     up, down = torch.cuda.Stream(), torch.cuda.Stream()
 
     def pipeline(n: int):
@@ -671,8 +669,7 @@ def run_e2e(args, w, step, stream, flush):
             done[k].record(stream)
             with torch.cuda.stream(down):
                 down.wait_event(done[k])
-                for o, h in zip(st.out, outs[k % 2]):
-                    h.copy_(o, non_blocking=True)
+                outs[k % 2].copy_(st.out_all, non_blocking=True)
                 back[k].record(down)
         down.wait_event(done[n - 1])
         t1.record(down)

@@ -110,16 +110,19 @@ class DecodeStep:
                                                             w.hierarchical), dtype=torch.uint8, device=dev)
         self.ws_attn = torch.empty(csa2.csa2_workspace_bytes(csa2.OP_ATTENTION, self.nq, self.heads),
                                    dtype=torch.uint8, device=dev)
-        # per-layer inputs: attention queries and (Full/Reindex) indexer queries
-        self.q = []
+        # per-layer inputs: attention queries and (Full/Reindex) indexer queries; the
+        # layers' queries and outputs are views of one tensor each (one copy per step)
+        nl = len(self.layers)
+        self.q_all = torch.empty((nl, self.nq, self.heads, 512), dtype=torch.bfloat16, device=dev)
+        self.out_all = torch.empty((nl, self.nq, self.heads, 512), dtype=torch.bfloat16, device=dev)
+        self.q = [self.q_all[i] for i in range(nl)]
+        self.out = [self.out_all[i] for i in range(nl)]
         self.idxq = {}
         for i, mode in enumerate(self.layers):
             l = layer0 + i
-            self.q.append(_gather_rows(lambda s, n: wdev.q_batch(w.seed, l, s, n, self.heads), seqs))
+            self.q[i].copy_(_gather_rows(lambda s, n: wdev.q_batch(w.seed, l, s, n, self.heads), seqs))
             if mode in ("F", "RI"):
                 self.idxq[i] = _gather_rows(lambda s, n: wdev.idxq_batch(w.seed, l, s, n), seqs)
-        self.out = [torch.empty((self.nq, self.heads, 512), dtype=torch.bfloat16, device=dev)
-                    for _ in self.layers]
         # the step's new token: position L-1 of each sequence (its seeded value)
         col = torch.from_numpy(wl.kv_col_scale(w.seed)).cuda()
         self.new_kv = torch.empty((self.nq, 512), dtype=torch.bfloat16, device=dev)
