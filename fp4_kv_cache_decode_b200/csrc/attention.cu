@@ -418,11 +418,13 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
   bool u0 = false, u1 = false;   // slot used
   uint32_t id0 = kNoRow, id1 = kNoRow;
   if (rmode == 2) {   // the rows a Full / Reindex call resolved for this set and range
+    // the ids load together with the count (slots past it hold stale ids, dropped below)
+    const int32_t c0 = s0 < hi ? rc_row[s0] : -1, c1 = s0 + 1 < hi ? rc_row[s0 + 1] : -1;
     const int nrow_c = rc_row[kMaxRows + split];
     u0 = s0 < hi && s0 - lo < nrow_c;
     u1 = s0 + 1 < hi && s0 + 1 - lo < nrow_c;
-    if (u0) id0 = (uint32_t)rc_row[s0];
-    if (u1) id1 = (uint32_t)rc_row[s0 + 1];
+    if (u0) id0 = (uint32_t)c0;
+    if (u1) id1 = (uint32_t)c1;
   } else {
     int32_t e0 = -1, e1 = -1;
     if (s0 < hi && s0 < kTopK) e0 = idx_row[s0];
