@@ -30,9 +30,11 @@
 //     score exceeds it by more than kSlack2 (then O^T and l are rescaled in
 //     place), so the weights 2^(s - m) stay below 2^kSlack2 and the final
 //     O / l is exact up to rounding.
-// With S = 1 the CTA writes the normalised bf16 output; otherwise it writes
-// (m, l, O) and a combine kernel merges the S ranges (log-sum-exp).  Results
-// leave through shared memory with one bulk copy.  Hand-offs use mbarriers
+// With S = 1 the CTA writes the normalised bf16 output; otherwise every CTA
+// of the query's cluster writes its normalised output as an f16 slice to L2
+// and its (m, l) per head to the cluster's shared tables, and after one
+// cluster barrier each combines 1/S of the channels (log-sum-exp weights).
+// Hand-offs use mbarriers
 // (tcgen05.commit for tensor-core completion); every wait is bounded and
 // reports CSA2_DEVERR_TIMEOUT instead of hanging.
 #include "common.cuh"
@@ -306,13 +308,16 @@ __device__ __forceinline__ void raw_decode(const RawTile& R, uint8_t* sp, uint32
   }
 }
 
-// Rank `split` of a query's cluster sums channels [split C, (split + 1) C),
-// C = 512 / S, of the S f16 slices [S][H][512] in `part` and writes them as
-// bf16.  Task = (head, 8 channels); a thread's tasks are tid + 416 t, and all
-// of their loads (at most 16 x 16 B) are in flight before any sum is formed.
+// Rank `split` of a query's cluster combines channels [split C, (split + 1) C),
+// C = 512 / S, of the S normalised f16 slices [S][H][512] in `part`: slice j
+// enters with weight 2^(m_j - M) l_j / L (M the largest m_j of the ranks that
+// attended something, L the sum of 2^(m_j - M) l_j), read from the cluster's
+// (m, l) table `ml` [S][64].  Output bf16.  Task = (head, 8 channels); a
+// thread's tasks are tid + 416 t, and all of their loads (at most 16 x 16 B)
+// are in flight before the weights are formed.
 template <int S>
 __device__ __forceinline__ void reduce_slices(const uint16_t* __restrict__ part, uint16_t* __restrict__ out,
-                                              int r, int split, int H, int tid) {
+                                              const float2* ml, int r, int split, int H, int tid) {
   constexpr int nch = kD / S, c8n = nch / 8;
   constexpr int kTasks = (kHeadsMma * c8n + kPipeThreads - 1) / kPipeThreads;   // per thread at H = 64
   const int ntask = H * c8n;
@@ -331,18 +336,32 @@ __device__ __forceinline__ void reduce_slices(const uint16_t* __restrict__ part,
   for (int t = 0; t < kTasks; ++t) {
     const int task = tid + t * kPipeThreads;
     if (task < ntask) {
+      const int h = task / c8n, ch0 = split * nch + 8 * (task % c8n);
+      float wj[S], M = -INFINITY, L = 0.0f;
+#pragma unroll
+      for (int j = 0; j < S; ++j) {
+        const float2 x = ml[j * 64 + h];
+        if (x.y > 0.0f) M = fmaxf(M, x.x);
+      }
+#pragma unroll
+      for (int j = 0; j < S; ++j) {
+        const float2 x = ml[j * 64 + h];
+        wj[j] = x.y > 0.0f ? ex2(x.x - M) * x.y : 0.0f;
+        L += wj[j];
+      }
+      const float inv = L > 0.0f ? 1.0f / L : 0.0f;
       float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
       for (int j = 0; j < S; ++j) {
+        const float g = wj[j] * inv;
         const uint32_t w[4] = {xs[t][j].x, xs[t][j].y, xs[t][j].z, xs[t][j].w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
-          acc[2 * k] += f2.x;
-          acc[2 * k + 1] += f2.y;
+          acc[2 * k] = fmaf(g, f2.x, acc[2 * k]);
+          acc[2 * k + 1] = fmaf(g, f2.y, acc[2 * k + 1]);
         }
       }
-      const int h = task / c8n, ch0 = split * nch + 8 * (task % c8n);
       uint4 o;
       o.x = pack_bf16x2(acc[0], acc[1]);
       o.y = pack_bf16x2(acc[2], acc[3]);
@@ -759,46 +778,29 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
   }
 
   // ---- output ----
-  // One range per query (nsplit == 1): out = O / l in bf16.  Otherwise every
-  // rank of the query's cluster scales its O^T by 2^(m_j - M) / L (M, L over
-  // the cluster), writes it as f16 [H][512] to its slice of `part` (shared
-  // memory is too slow a path between SMs for 100+ KiB), and after a cluster
-  // barrier rank j sums channels [j C, (j + 1) C), C = 512 / nsplit, over
-  // the nsplit slices.  f16 keeps each term to 2^-11 relative, below the
+  // Every rank writes its normalised O / l: bf16 to `out` with one range per
+  // query (nsplit == 1), else f16 to its slice of `part` (shared memory is too
+  // slow a path between SMs for 100+ KiB) while its (m, l) per head goes to
+  // every rank's table; one cluster barrier later rank j combines channels
+  // [j C, (j + 1) C), C = 512 / nsplit, of the nsplit slices by their
+  // log-sum-exp weights.  f16 keeps each slice to 2^-11 relative, below the
   // final bf16 rounding.
   if (nsplit > 1) {
-    cluster_wait();
-    // publish this rank's (m, l) per head in every rank's table (l = 0: nothing to add)
-    if (tid < 64) {
+    cluster_wait();   // every rank of the cluster runs
+    if (tid < 64) {   // (m, l) of this rank per head (l = 0: nothing to add)
       const float mj = all_ok ? m_run[tid] : -INFINITY, lj = all_ok ? l_s[tid] : 0.0f;
       const uint32_t slot = sb + kOffMl + 8u * (uint32_t)(split * 64 + tid);
       for (int j = 0; j < nsplit; ++j) st_cluster_v2(map_shared(slot, (uint32_t)j), mj, lj);
     }
-    cluster_sync_all();   // every rank's tiles are done and its (m, l) have arrived
-    if (tid < 64) {
-      const float2* ml = reinterpret_cast<const float2*>(sp + kOffMl);
-      float M = -INFINITY;
-      for (int j = 0; j < nsplit; ++j) {
-        const float2 x = ml[j * 64 + tid];
-        if (x.y > 0.0f) M = fmaxf(M, x.x);
-      }
-      float L = 0.0f;
-      for (int j = 0; j < nsplit; ++j) {
-        const float2 x = ml[j * 64 + tid];
-        if (x.y > 0.0f) L += ex2(x.x - M) * x.y;
-      }
-      const float2 self = ml[split * 64 + tid];
-      f_s[tid] = (self.y > 0.0f && L > 0.0f) ? ex2(self.x - M) / L : 0.0f;
-      lse_ml[tid] = make_float2(M, L);
-    }
-  } else if (tid < 64) {
+  }
+  if (tid < 64) {
     const bool have = all_ok && l_s[tid] > 0.0f;
     f_s[tid] = have ? 1.0f / l_s[tid] : 0.0f;
     lse_ml[tid] = make_float2(have ? m_run[tid] : -INFINITY, have ? l_s[tid] : 0.0f);
   }
   __syncthreads();
-  // the idle MMA warp writes the log-sum-exp of a sharded call (one range per query)
-  if (warp == kMmaWarp && shard.lse2 != nullptr && split == 0) {
+  // the idle MMA warp writes the log-sum-exp of a sharded call with one range per query
+  if (warp == kMmaWarp && shard.lse2 != nullptr && nsplit == 1) {
     for (int h = lane; h < H; h += 32) {
       const float2 ml = lse_ml[h];
       shard.lse2[(int64_t)r * H + h] = ml.y > 0.0f ? ml.x + __log2f(ml.y) : -INFINITY;
@@ -838,10 +840,21 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
     }
   }
   if (nsplit > 1) {
-    cluster_sync_all();   // every rank's slice is in global memory
-    if (nsplit == 2) reduce_slices<2>(part, out, r, split, H, tid);
-    else if (nsplit == 4) reduce_slices<4>(part, out, r, split, H, tid);
-    else reduce_slices<8>(part, out, r, split, H, tid);
+    cluster_sync_all();   // every rank's slice is in global memory and its (m, l) in every table
+    const float2* ml = reinterpret_cast<const float2*>(sp + kOffMl);
+    if (shard.lse2 != nullptr && split == 0 && tid < H) {   // log-sum-exp over the cluster
+      float M = -INFINITY, L = 0.0f;
+      for (int j = 0; j < nsplit; ++j)
+        if (ml[j * 64 + tid].y > 0.0f) M = fmaxf(M, ml[j * 64 + tid].x);
+      for (int j = 0; j < nsplit; ++j) {
+        const float2 x = ml[j * 64 + tid];
+        if (x.y > 0.0f) L += ex2(x.x - M) * x.y;
+      }
+      shard.lse2[(int64_t)r * H + tid] = L > 0.0f ? M + __log2f(L) : -INFINITY;
+    }
+    if (nsplit == 2) reduce_slices<2>(part, out, ml, r, split, H, tid);
+    else if (nsplit == 4) reduce_slices<4>(part, out, ml, r, split, H, tid);
+    else reduce_slices<8>(part, out, ml, r, split, H, tid);
   }
 
   // teardown
