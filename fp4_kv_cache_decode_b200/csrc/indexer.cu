@@ -583,7 +583,9 @@ __device__ __forceinline__ void topk_registers(const float* __restrict__ srow, i
 //  3. each thread takes a contiguous segment of positions, counts its keys
 //     above T and equal to T, one CTA scan gives its output offset, and it
 //     writes its selected positions in order (ascending overall).
-template <int SRC>
+// kRegOnly: the launch guarantees n <= 16,384 for every row, so only the
+// register path is compiled (far less code for each launch to fetch).
+template <int SRC, bool kRegOnly>
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(CacheView c, const float* __restrict__ scores,
                                                             int64_t stride, const int32_t* __restrict__ q_seq,
                                                             const int32_t* __restrict__ q_vis,
@@ -608,7 +610,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(CacheView c, const f
   int32_t* orow = out.ids + (int64_t)blockIdx.x * out.stride;
   float* oscore = out.scores ? out.scores + (int64_t)blockIdx.x * out.stride : nullptr;
   const int32_t id_off = (out.id_offset ? (out.id_offset[r] >> out.offset_shift) : 0) + (int32_t)seg0;
-  if (n <= kTopkSmemKeys) {
+  if (kRegOnly || n <= kTopkSmemKeys) {
     topk_registers<SRC>(srow, n, k, pool_row, orow, oscore, id_off, sm);
     return;
   }
@@ -743,18 +745,19 @@ cudaError_t launch_score_mma(int src, const CacheView& c, const uint16_t* idx_q,
 // Opt the top-k kernels in to their shared-memory size (once per device).
 cudaError_t indexer_set_attributes() {
   const int smem = (int)topk_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(topk_kernel<SRC_FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const void* topk_kernels[] = {
+      (const void*)topk_kernel<SRC_FLAT, false>,      (const void*)topk_kernel<SRC_FLAT, true>,
+      (const void*)topk_kernel<SRC_BLOCKKEYS, false>, (const void*)topk_kernel<SRC_BLOCKKEYS, true>,
+      (const void*)topk_kernel<SRC_POOL, true>,       (const void*)topk_kernel<SRC_CAND, false>,
+      (const void*)topk_kernel<SRC_CAND, true>};
+  cudaError_t e = cudaSuccess;
+  for (const void* k : topk_kernels)
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   const void* score_kernels[] = {(const void*)score_units_kernel<SRC_FLAT, true>,
                                  (const void*)score_units_kernel<SRC_POOL, true>};
   for (const void* k : score_kernels)
     if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmemMax);
   if (e == cudaSuccess) e = score_mma_set_attributes();
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(topk_kernel<SRC_BLOCKKEYS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(topk_kernel<SRC_POOL>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(topk_kernel<SRC_CAND>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   return e;
 }
 
@@ -800,14 +803,25 @@ cudaError_t launch_topk(int src, const CacheView& c, const float* scores, int64_
   // nseg > 1: one CTA per segment of kTopkSmemKeys entries; output rows nq x nseg
   const TopkOut o{out, out_stride, out_scores, id_offset, offset_shift, nseg > 1 ? nseg : 1, kTopkSmemKeys};
   if (nseg > 1) nq *= nseg;
-  if (src == SRC_FLAT)
-    launch_pdl(topk_kernel<SRC_FLAT>, nq, kTopkThreads, smem, st, c, scores, stride, q_seq, q_vis, pool, k, o);
-  else if (src == SRC_BLOCKKEYS)
-    launch_pdl(topk_kernel<SRC_BLOCKKEYS>, nq, kTopkThreads, smem, st, c, scores, stride, q_seq, q_vis, pool, k, o);
-  else if (src == SRC_POOL)
-    launch_pdl(topk_kernel<SRC_POOL>, nq, kTopkThreads, smem, st, c, scores, stride, q_seq, q_vis, pool, k, o);
-  else
-    launch_pdl(topk_kernel<SRC_CAND>, nq, kTopkThreads, smem, st, c, scores, stride, q_seq, q_vis, pool, k, o);
+  // every row fits the register path when a row holds at most 16,384 entries:
+  // n <= stride always, n <= the segment length when segmented, and a pool row
+  // is 2,048 blocks x 8 tokens
+  const bool reg = nseg > 1 || src == SRC_POOL || stride <= kTopkSmemKeys;
+#define CSA2_TOPK_LAUNCH(S, R) \
+  launch_pdl(topk_kernel<S, R>, nq, kTopkThreads, smem, st, c, scores, stride, q_seq, q_vis, pool, k, o)
+  if (src == SRC_FLAT) {
+    if (reg) CSA2_TOPK_LAUNCH(SRC_FLAT, true);
+    else CSA2_TOPK_LAUNCH(SRC_FLAT, false);
+  } else if (src == SRC_BLOCKKEYS) {
+    if (reg) CSA2_TOPK_LAUNCH(SRC_BLOCKKEYS, true);
+    else CSA2_TOPK_LAUNCH(SRC_BLOCKKEYS, false);
+  } else if (src == SRC_POOL) {
+    CSA2_TOPK_LAUNCH(SRC_POOL, true);
+  } else {
+    if (reg) CSA2_TOPK_LAUNCH(SRC_CAND, true);
+    else CSA2_TOPK_LAUNCH(SRC_CAND, false);
+  }
+#undef CSA2_TOPK_LAUNCH
   return cudaGetLastError();
 }
 
