@@ -45,7 +45,6 @@
 namespace csa2 {
 
 constexpr int kRowTile = 64;                           // attended rows per pipeline step
-constexpr int kMaxSplits = kMaxRows / kRowTile;        // 10
 constexpr int kHeadsMma = 64;                          // MMA N: heads, padded
 constexpr int kSoftmaxWarps = 4;                       // warps 0..3 (TMEM sub-partitions 0..3)
 constexpr int kProducerWarps = 8;                      // warps 4..11
