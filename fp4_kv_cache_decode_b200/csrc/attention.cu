@@ -34,9 +34,8 @@
 // of the query's cluster writes its normalised output as an f16 slice to L2
 // and its (m, l) per head to the cluster's shared tables, and after one
 // cluster barrier each combines 1/S of the channels (log-sum-exp weights).
-// Hand-offs use mbarriers
-// (tcgen05.commit for tensor-core completion); every wait is bounded and
-// reports CSA2_DEVERR_TIMEOUT instead of hanging.
+// Hand-offs use mbarriers (tcgen05.commit for tensor-core completion); every
+// wait is bounded and reports CSA2_DEVERR_TIMEOUT instead of hanging.
 #include "common.cuh"
 #include "tc.cuh"
 
