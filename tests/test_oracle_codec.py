@@ -154,3 +154,20 @@ def test_decoded_values_exact_in_bf16():
     v = (formats.E2M1_VALUES[:, None] * codec.E4M3_GRID[None, :]).reshape(-1)
     b = formats.f32_to_bf16(v.astype(np.float32))
     np.testing.assert_array_equal(formats.bf16_to_f64(b), v)
+
+
+def test_compress_pairs_hand_values():
+    """2:1 compression is the mean of adjacent rows: hand-computed pairs, and on
+    random bf16 pairs in the normal range the fp32 result equals the exact mean
+    (fp64) rounded to fp32 (halving is exact, so fl32(a + b) / 2 = fl32((a + b) / 2))."""
+    def bits(vals):
+        return formats.f32_to_bf16(np.asarray(vals, dtype=np.float32)).reshape(len(vals), 1)
+    got = codec.compress_pairs_f32(bits([1.0, 2.0, -3.0, 3.0, 0.5, 0.25, -0.0, 0.0]))
+    np.testing.assert_array_equal(got[:, 0], np.array([1.5, 0.0, 0.375, 0.0], dtype=np.float32))
+    rng = np.random.default_rng(11)
+    x = formats.f32_to_bf16((rng.standard_normal((4096, 8)) * np.exp2(rng.integers(-20, 20, (4096, 8))))
+                            .astype(np.float32))
+    got = codec.compress_pairs_f32(x)
+    xf = formats.bf16_to_f64(x)
+    want = ((xf[0::2] + xf[1::2]) / 2.0).astype(np.float32)
+    np.testing.assert_array_equal(got, want)

@@ -216,3 +216,57 @@ def test_max_pooled_hierarchy_brute_force_on_shrunken_sizes():
         assert list(idx[idx >= 0]) == want
         flat = sorted(sorted(range(L), key=lambda t: (-ts[t], t))[:2])
         assert want == flat
+
+
+def test_pool_tokens_expansion_and_clipping():
+    """Pool blocks expand to their 8 positions each, ascending in pool order,
+    -1 entries dropped, positions at or past the context length removed."""
+    got = indexer.pool_tokens(np.array([0, 3, 5, -1, -1]), length=44)
+    want = list(range(0, 8)) + list(range(24, 32)) + list(range(40, 44))
+    np.testing.assert_array_equal(got, want)
+    assert indexer.pool_tokens(np.array([-1, -1]), length=100).size == 0
+    # a block wholly past the end contributes nothing
+    np.testing.assert_array_equal(indexer.pool_tokens(np.array([1, 9]), length=16), np.arange(8, 16))
+
+
+def test_select_tokens_brute_force():
+    """select_tokens = the k best candidates by (score desc, position asc), as
+    positions in ascending order, padded with -1; scores returned per candidate."""
+    rng = np.random.default_rng(7)
+    k = _bf16(rng.standard_normal((200, 64)))
+    q = _bf16(rng.standard_normal((4, 64)))
+    # ties: copy a few keys so that equal scores occur at different positions
+    k[50] = k[10]
+    k[120] = k[10]
+    cand = np.array(sorted(rng.choice(200, size=60, replace=False).tolist() + [10, 50, 120]))
+    cand = np.unique(cand)
+    for kk in (5, 17, len(cand), len(cand) + 9):
+        sel, s = indexer.select_tokens(q, k, cand, k=kk)
+        kf = formats.bf16_to_f32(k)
+        qf = formats.bf16_to_f32(q)
+        scores = {}
+        for p in cand:                               # brute force, same fp32 order as the oracle
+            tot = np.float32(0)
+            for h in range(4):
+                dot = np.float32(0)
+                for d in range(64):
+                    dot = np.float32(dot + np.float32(qf[h, d] * kf[p, d]))
+                tot = np.float32(tot + max(dot, np.float32(0)))
+            scores[int(p)] = tot
+        np.testing.assert_array_equal(s, np.array([scores[int(p)] for p in cand], dtype=np.float32))
+        best = sorted(scores, key=lambda p: (-scores[p], p))[:kk]
+        want = sorted(best) + [-1] * (kk - len(best))
+        np.testing.assert_array_equal(sel, want)
+
+
+def test_block_max_scores_brute_force():
+    """Each block's max-pooled score is the largest score among its present
+    tokens; a ragged last block uses only the tokens below the length."""
+    rng = np.random.default_rng(8)
+    k = _bf16(rng.standard_normal((77, 64)))
+    q = _bf16(rng.standard_normal((4, 64)))
+    for L in (1, 8, 9, 77):
+        ts = indexer.index_scores(q, k[:L])
+        got = indexer.block_max_scores(q, k, L)
+        want = [max(ts[8 * b: min(8 * b + 8, L)]) for b in range((L + 7) // 8)]
+        np.testing.assert_array_equal(got, np.array(want, dtype=np.float32))
