@@ -153,3 +153,22 @@ def test_window_store_holds_the_last_128_entries():
             assert len(set(slot.tolist())) == pos.size and slot.min() >= 0 and slot.max() < 128
             probe = np.arange(L)
             np.testing.assert_array_equal(modes.from_window_store(probe, L), np.isin(probe, list(fifo)))
+
+
+def test_window_store_is_a_ring_filled_from_slot_zero():
+    """Appending moves nothing: an entry keeps its slot for as long as it is in
+    the window, and the one appended takes the slot its evicted predecessor
+    left.  An empty store fills its first slots first.  Together these fix the
+    layout (by induction, slot of position p = p mod 128)."""
+    slot_of = {}
+    for L in range(1, 600):
+        pos, slot = modes.window_store_slots(L)
+        cur = dict(zip(pos.tolist(), slot.tolist()))
+        for p_, s_ in cur.items():
+            if p_ in slot_of:
+                assert slot_of[p_] == s_, (L, p_)            # no entry moves
+        if L <= 128:
+            assert cur[L - 1] == L - 1                       # filled from slot 0 in order
+        else:
+            assert cur[L - 1] == slot_of[L - 1 - 128]        # takes the evicted entry's slot
+        slot_of.update(cur)

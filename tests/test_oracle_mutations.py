@@ -204,3 +204,88 @@ def _compress_first_of_pair(bits):
 def test_codec_slips_are_caught(monkeypatch, name, fn):
     monkeypatch.setattr(codec, name, fn)
     assert _caught(CODEC_PINS)
+
+
+# ---- FP8 indexer keys ----
+
+from oracle import idxk_fp8, modes                     # noqa: E402
+from tests import test_oracle_idxk_fp8 as pin_fp8       # noqa: E402
+from tests import test_oracle_modes as pin_modes        # noqa: E402
+
+FP8_PINS = [pin_fp8.test_every_e4m3_value_encodes_to_itself,
+            pin_fp8.test_rounding_against_brute_force_on_all_bf16_magnitudes,
+            pin_fp8.test_midpoints_round_to_even_and_match_torch, pin_fp8.test_saturation,
+            pin_fp8.test_quantised_key_error_bound_and_degenerate_keys,
+            pin_fp8.test_exactly_representable_keys_round_trip_and_score_like_bf16,
+            pin_fp8.test_scores_against_fp64_on_the_dequantised_key]
+
+
+def _e4m3_ties_away(t):
+    t = np.asarray(t, dtype=np.float32)
+    mag = np.abs(t.astype(np.float64))
+    code = np.sum(idxk_fp8.E4M3_MIDS <= mag[..., None], axis=-1)   # slip: ties round up, not to even
+    return (code | (np.signbit(t).astype(np.int64) << 7)).astype(np.uint8)
+
+
+def _e4m3_sign_dropped(t):
+    t = np.asarray(t, dtype=np.float32)
+    mag = np.abs(t.astype(np.float64))
+    below = np.sum(idxk_fp8.E4M3_MIDS < mag[..., None], axis=-1)
+    tie = np.any(idxk_fp8.E4M3_MIDS == mag[..., None], axis=-1)
+    return (below + (tie & (below % 2 == 1))).astype(np.uint8)     # slip: the sign bit lost
+
+
+def _quantize_scale_240(key_bits):
+    k = bf16_to_f32(np.asarray(key_bits, dtype=np.uint16))
+    amax = np.max(np.abs(k), axis=-1).astype(np.float32)
+    s = (amax / np.float32(240.0)).astype(np.float32)                # slip: the E4M3 maximum taken as 240
+    codes = np.zeros(k.shape, dtype=np.uint8)
+    nz = s != 0
+    codes[nz] = idxk_fp8.e4m3_code((k[nz] / s[nz, None]).astype(np.float32))
+    return codes, s
+
+
+@pytest.mark.parametrize("name,fn", [("e4m3_code", _e4m3_ties_away), ("e4m3_code", _e4m3_sign_dropped),
+                                     ("quantize", _quantize_scale_240)])
+def test_fp8_key_slips_are_caught(monkeypatch, name, fn):
+    monkeypatch.setattr(idxk_fp8, name, fn)
+    assert _caught(FP8_PINS)
+
+
+# ---- replay and the sliding-window store ----
+
+MODES_PINS = [pin_modes.test_replay_positions, pin_modes.test_replay_idempotent_and_restores_poisoned_rows,
+              pin_modes.test_ratio2_replay_of_duplicated_rows_equals_ratio1,
+              pin_modes.test_window_store_holds_the_last_128_entries,
+              pin_modes.test_window_store_is_a_ring_filled_from_slot_zero,
+              lambda: pin_modes.test_ratio2_replay_of_an_intact_sequence_reproduces_its_entries(300)]
+
+
+def _replay_one_short(length, miss, window=modes.REPLAY):
+    if length <= 0:
+        return np.zeros(0, np.int64), np.zeros(0, np.int64)
+    if miss:
+        n = min(window - 1, length)                                  # slip: 127 entries replayed
+        return np.arange(length - n, length), np.arange(window - n, window)
+    return np.array([length - 1]), np.array([window - 1])
+
+
+def _replay_wrong_rows(length, miss, window=modes.REPLAY):
+    if length <= 0:
+        return np.zeros(0, np.int64), np.zeros(0, np.int64)
+    if miss:
+        n = min(window, length)
+        return np.arange(length - n, length), np.arange(0, n)        # slip: the block's first rows, not its last
+    return np.array([length - 1]), np.array([window - 1])
+
+
+def _store_slots_shifted(length, window=modes.REPLAY):
+    pos = np.arange(max(0, length - window), length, dtype=np.int64)
+    return pos, (pos + 1) % window                                   # slip: slots shifted by one
+
+
+@pytest.mark.parametrize("name,fn", [("replay_positions", _replay_one_short), ("replay_positions", _replay_wrong_rows),
+                                     ("window_store_slots", _store_slots_shifted)])
+def test_replay_slips_are_caught(monkeypatch, name, fn):
+    monkeypatch.setattr(modes, name, fn)
+    assert _caught(MODES_PINS)
