@@ -289,3 +289,35 @@ def _store_slots_shifted(length, window=modes.REPLAY):
 def test_replay_slips_are_caught(monkeypatch, name, fn):
     monkeypatch.setattr(modes, name, fn)
     assert _caught(MODES_PINS)
+
+
+# ---- the layer schedule ----
+
+def _run_layers_with(slip):
+    """run_layers with one schedule slip: "ri_own_pool" (a Reindex layer builds
+    its own pool), "reuse_recomputes" (a Reuse layer selects with its own query),
+    "ri_reuses" (a Reindex layer keeps the previous set)."""
+    def run(layers, length, key_bits, idxq_fn, q_fn, rows_fn, sm_scale=1.0, hierarchical=True, w=None):
+        results, pool, latest = [], None, None
+        for layer, mode in enumerate(layers):
+            if mode == "F" or (mode == "RI" and slip == "ri_own_pool") or (mode == "R" and slip == "reuse_recomputes"):
+                pool, latest, _ = indexer.full_indexer(idxq_fn(layer), key_bits, length, w, hierarchical)
+            elif mode == "RI" and slip != "ri_reuses":
+                latest, _ = indexer.reindex_indexer(idxq_fn(layer), key_bits, length, pool, w)
+            pos = attention.attended_positions(latest, length)
+            out = attention.attend(q_fn(layer), rows_fn(pos), sm_scale)
+            results.append({"mode": mode, "idx": latest.copy(), "pool": None if pool is None else pool.copy(),
+                            "out": out})
+        return results
+    return run
+
+
+@pytest.mark.parametrize("slip", ["ri_own_pool", "reuse_recomputes", "ri_reuses"])
+def test_schedule_slips_are_caught(monkeypatch, slip):
+    monkeypatch.setattr(modes, "run_layers", _run_layers_with(slip))
+    assert _caught([lambda: pin_modes.test_reuse_and_reindex_invariants(20000)])
+
+
+def test_schedule_reimplementation_without_slip_passes(monkeypatch):
+    monkeypatch.setattr(modes, "run_layers", _run_layers_with(None))
+    assert _some_pin_fails([lambda: pin_modes.test_reuse_and_reindex_invariants(20000)]) == []
