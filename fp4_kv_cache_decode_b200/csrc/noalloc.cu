@@ -21,7 +21,9 @@
 //    selection kernel later reads;
 //  * the first call on a device looks up the array's device address with that
 //    device current (a one-time set-up); make that first call before any
-//    stream capture.
+//    stream capture.  The address is kept until the process exits: a
+//    cudaDeviceReset() on that device invalidates it, and the call is not
+//    supported after one.
 // Nothing here allocates: no cudaMalloc, no cudaFree, no allocating library
 // routine.
 #include <mutex>
@@ -64,7 +66,13 @@ extern "C" int csa2_indexer_score_topk_noalloc(const csa2_cache* cache, const ui
   if (nq < 0 || max_visible < 0) return CSA2_ERR_INVALID_ARG;
   const int32_t hier = mode == CSA2_REINDEX ? CSA2_HIER_MEAN : hierarchical;
   const size_t need = csa2_workspace_bytes(CSA2_OP_INDEXER, nq, 0, max_visible, hier);
-  if (need > (size_t)CSA2_NOALLOC_SCRATCH_BYTES) return CSA2_ERR_WORKSPACE;
+  // an oversize request still gets the argument and mode-order checks first:
+  // with no workspace the regular call reports those, else CSA2_ERR_WORKSPACE,
+  // and launches nothing either way
+  // (a size of 0 means csa2_workspace_bytes found the arguments invalid)
+  if (need == 0 || need > (size_t)CSA2_NOALLOC_SCRATCH_BYTES)
+    return csa2_indexer_score_topk(cache, idx_q, head_w, q_seq, q_visible, nq, max_visible, mode, hierarchical,
+                                   layer, set, nullptr, 0, stream);
   void* scratch = nullptr;
   if (nq > 0) {
     const int st = scratch_address(&scratch);

@@ -15,7 +15,9 @@
  * --------------------------
  * - All tensor arguments are DEVICE pointers owned by the caller; the library
  *   allocates no memory.  Scratch space comes from a caller workspace sized by
- *   csa2_workspace_bytes().
+ *   csa2_workspace_bytes(), except in csa2_indexer_score_topk_noalloc, whose
+ *   scratch is one static device array of CSA2_NOALLOC_SCRATCH_BYTES that the
+ *   library holds on every GPU that loads it.
  * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *   default stream) and performs no host synchronisation and no allocation;
  *   csa2_check_device_error() is the only call that synchronises.  The calls
@@ -284,13 +286,16 @@ int csa2_swa_replay(const csa2_cache* cache, const uint16_t* kv_last, const uint
  * Same arguments and results as csa2_indexer_score_topk minus the workspace:
  * the score buffer is a library-owned static device array of
  * CSA2_NOALLOC_SCRATCH_BYTES, present on every GPU that loads the library
- * until the process exits.  Requests whose workspace (csa2_workspace_bytes)
- * exceeds that size return CSA2_ERR_WORKSPACE without launching anything.
+ * until the process exits.  Argument and mode-order errors are reported as by
+ * csa2_indexer_score_topk; a valid request whose workspace
+ * (csa2_workspace_bytes) exceeds that size returns CSA2_ERR_WORKSPACE without
+ * launching anything.
  * All calls share the one array: calls that overlap on the GPU race, so keep
  * them on one stream.  The array keeps the last call's contents; nothing in
  * it needs to start at zero.  The first call on a device looks up the
  * array's device address (a one-time set-up); make it before any stream
- * capture.  Allocates nothing.
+ * capture.  The address is kept for the life of the process, so the call is
+ * not supported after cudaDeviceReset() on that device.  Allocates nothing.
  */
 #define CSA2_NOALLOC_SCRATCH_BYTES (16u << 20)   /* 16 MiB */
 int csa2_indexer_score_topk_noalloc(const csa2_cache* cache, const uint16_t* idx_q,

@@ -170,6 +170,28 @@ def test_mode_order_state_machine(csa2_lib):
                                      f.p(), 1 << 30, None) == 3
 
 
+def test_noalloc_checks_arguments_before_size(csa2_lib):
+    """The entry point without a workspace reports argument and mode-order errors
+    like the regular call, and refuses a valid request larger than its static
+    array with CSA2_ERR_WORKSPACE; none of these launches anything."""
+    L = csa2_lib.lib()
+    f = _Fake()
+    c = _cache(csa2_lib, f)
+    s = _iset(csa2_lib, f, rows=64)
+    B = ctypes.byref
+    FULL, REINDEX = 0, 1
+    big = 1 << 20                                  # 64 queries at 1M: far above 16 MiB
+    assert csa2_lib.csa2_workspace_bytes(1, 64, 0, big, True) > csa2_lib.NOALLOC_SCRATCH_BYTES
+    na = lambda mode, hier=1, cache=c, q=f.p(): L.csa2_indexer_score_topk_noalloc(
+        B(cache), q, None, f.p(), None, 64, big, mode, hier, 3, B(s), None)
+    assert na(REINDEX) == 4                        # no Full pool yet: mode order first
+    assert na(FULL, hier=3) == 1                   # unknown block score
+    assert na(FULL, q=f.p(8)) == 3                 # misaligned query
+    assert na(FULL, cache=_cache(csa2_lib, f, batch=0)) == 2
+    assert na(FULL) == 5                           # valid, but larger than the array
+    assert s.layer == -1                           # nothing was recorded
+
+
 def test_replay_and_cache_argument_checks(csa2_lib):
     L = csa2_lib.lib()
     f = _Fake()
