@@ -11,6 +11,10 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "lib", "libcsa2.so")
+# The same library with test hooks (short wait limits, a stall that makes a
+# bounded wait run out): loaded only by tests/test_gpu_timeout.py.
+TEST_LIB = os.path.join(PKG, "lib", "libcsa2_test.so")
+TEST_HOOK_SOURCES = ("attention.cu", "score_mma.cu")
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",
@@ -30,9 +34,9 @@ def _inputs() -> list[str]:
 
 
 def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+    if not os.path.exists(LIB) or not os.path.exists(TEST_LIB):
         return False
-    t = os.path.getmtime(LIB)
+    t = min(os.path.getmtime(LIB), os.path.getmtime(TEST_LIB))
     return all(os.path.getmtime(p) <= t for p in _inputs())
 
 
@@ -43,23 +47,30 @@ def build(force: bool = False, verbose: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     os.makedirs(os.path.dirname(LIB), exist_ok=True)
 
-    def compile_one(src: str) -> tuple[str, str]:
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
-        cmd = ["nvcc", *NVCC_FLAGS, "-c", src, "-o", obj]
+    def compile_one(job: tuple[str, bool]) -> tuple[str, str]:
+        src, hooks = job
+        obj = os.path.join(BUILD, os.path.basename(src) + (".test.o" if hooks else ".o"))
+        cmd = ["nvcc", *NVCC_FLAGS, *(["-DCSA2_TEST_HOOKS"] if hooks else []), "-c", src, "-o", obj]
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:
             raise RuntimeError(f"nvcc failed for {src}:\n{res.stderr}")
         return obj, res.stderr
 
+    srcs = sources()
+    jobs = [(src, False) for src in srcs] + [(src, True) for src in srcs
+                                             if os.path.basename(src) in TEST_HOOK_SOURCES]
     with ThreadPoolExecutor(max_workers=max(1, min(8, os.cpu_count() or 1))) as ex:
-        results = list(ex.map(compile_one, sources()))
-    log = "".join(r[1] for r in results)
+        results = list(ex.map(compile_one, jobs))
+    log = "".join(r[1] for r, (_, hooks) in zip(results, jobs) if not hooks)
     with open(os.path.join(BUILD, "ptxas.log"), "w") as f:
         f.write(log)
     if verbose:
         print(log)
-    tmp = LIB + f".tmp{os.getpid()}"
-    subprocess.check_call(["nvcc", "-shared", "-gencode", "arch=compute_100a,code=sm_100a",
-                           *[r[0] for r in results], "-o", tmp])
-    os.replace(tmp, LIB)
+    product = [r[0] for r, (_, hooks) in zip(results, jobs) if not hooks]
+    hooked = {os.path.basename(src): r[0] for r, (src, hooks) in zip(results, jobs) if hooks}
+    test_objs = [hooked.get(os.path.basename(src), obj) for src, obj in zip(srcs, product)]
+    for objs, lib in ((product, LIB), (test_objs, TEST_LIB)):
+        tmp = lib + f".tmp{os.getpid()}"
+        subprocess.check_call(["nvcc", "-shared", "-gencode", "arch=compute_100a,code=sm_100a", *objs, "-o", tmp])
+        os.replace(tmp, lib)
     return LIB

@@ -94,7 +94,11 @@ constexpr uint32_t kIdescPV = (1u << 4) | (1u << 15) | (1u << 16) | ((uint32_t)(
 constexpr uint32_t kIdescL = (1u << 4) | (1u << 16) | ((uint32_t)(kHeadsMma >> 3) << 17) | ((uint32_t)(64 >> 4) << 24);
 
 
+#ifdef CSA2_TEST_HOOKS
+constexpr uint32_t kPollLimit = 1u << 20;    // test build: the MMA thread gives up sooner
+#else
 constexpr uint32_t kPollLimit = 1u << 26;    // idle polls of the MMA thread before it gives up
+#endif
 
 // 32 consecutive fp32 TMEM columns of this thread's lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
@@ -512,6 +516,9 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
       mbar_init(pfull(b), kSmxThreads);
     }
     mbar_init(qready, kPipeThreads);
+#ifdef CSA2_TEST_HOOKS
+    mbar_init(bar0 + 72u, 1);   // completed by nothing: the test stall waits on it
+#endif
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     misc[1] = 0;
     misc[2] = 0;
@@ -604,6 +611,9 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
     store_q();
     if (lane == 0) {
       ok = mbar_wait(qready, 0);
+#ifdef CSA2_TEST_HOOKS
+      const bool stall = test_stall(c.err);
+#endif
       int nqk = 0, npv = 0;
       uint32_t idle = 0;
       while (ok && npv < nt) {
@@ -649,6 +659,10 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
           misc[2] = (t >> 1) & 1;
           ++nqk;
           progressed = true;
+#ifdef CSA2_TEST_HOOKS
+          // test stall after the first QK: a wait that runs out with an MMA committed
+          if (stall && nqk == 1 && !test_stall_wait(bar0 + 72u)) ok = false;
+#endif
         }
         if (progressed) idle = 0;
         else if (++idle > kPollLimit) ok = false;

@@ -52,6 +52,17 @@ struct CacheView {
 
 __device__ __forceinline__ void raise_error(uint32_t* err, uint32_t bits) { atomicOr(err, bits); }
 
+#ifdef CSA2_TEST_HOOKS
+// Test build only (lib/libcsa2_test.so): while a caller has set this bit of the
+// cache's error word, the attention and tensor-core scorer kernels wait on an
+// mbarrier that nothing completes, so that a bounded wait runs out and the
+// timeout path (error bit, drain, TMEM release) runs on the GPU.
+constexpr uint32_t kTestStallBit = 0x80000000u;
+__device__ __forceinline__ bool test_stall(const uint32_t* err) {
+  return (*reinterpret_cast<const volatile uint32_t*>(err) & kTestStallBit) != 0;
+}
+#endif
+
 // Page id holding token `tok` of sequence `seq`, or -1 (with an error bit
 // raised) when the sequence, the page slot or the page id is out of range.
 __device__ __forceinline__ int64_t page_of(const CacheView& c, int seq, int64_t tok) {

@@ -136,6 +136,9 @@ __global__ void __launch_bounds__(kSmThreads) score_mma_kernel(const __grid_cons
       mbar_init(freed(s), 4);
     }
     *abort_flag = 0;
+#ifdef CSA2_TEST_HOOKS
+    mbar_init(sb + kSmOffMisc + 8, 1);   // completed by nothing: the test stall waits on it
+#endif
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 5) tmem_alloc_warp(sb + kSmOffMisc, kSmTmemCols);
@@ -184,6 +187,13 @@ __global__ void __launch_bounds__(kSmThreads) score_mma_kernel(const __grid_cons
     if (lane == 0) {
       const uint64_t bdesc = smem_desc(sb + kSmOffB, 16, 1024);
       int t = 0;
+#ifdef CSA2_TEST_HOOKS
+      // test stall before the first MMA: the wait runs out, the CTA aborts
+      if (test_stall(c.err) && !test_stall_wait(sb + kSmOffMisc + 8)) {
+        *abort_flag = 1;
+        raise_error(c.err, CSA2_DEVERR_TIMEOUT);
+      }
+#endif
       for (; t < ntiles; ++t) {
         if (*abort_flag) break;
         const int s = t % kSmStages, n = t / kSmStages;

@@ -6,7 +6,11 @@
 
 namespace csa2 {
 
+#ifdef CSA2_TEST_HOOKS
+constexpr uint32_t kWaitLimit = 1u << 16;    // test build: waits give up sooner
+#else
 constexpr uint32_t kWaitLimit = 1u << 22;    // try_wait rounds before a wait gives up
+#endif
 // Shared-memory matrix descriptor: start address, leading and stride byte
 // offsets (16-B units), descriptor version 1, 128-byte swizzle.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
@@ -52,6 +56,18 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
   }
   return false;
 }
+
+#ifdef CSA2_TEST_HOOKS
+// Test build: the stall wait on an mbarrier nothing completes -- polls for about
+// two milliseconds, then gives up like any bounded wait.
+__device__ __forceinline__ bool test_stall_wait(uint32_t mbar) {
+  for (int i = 0; i < 2000; ++i) {
+    if (mbar_test(mbar, 0)) return true;
+    __nanosleep(1000);
+  }
+  return false;
+}
+#endif
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
