@@ -95,3 +95,51 @@ def test_sharded_full_layer_equals_unsharded(csa2_lib, unsharded, plan):
     # a shard holding none of the set reports -inf and adds nothing
     l2 = lse2.view(B, S, HEADS).cpu().numpy()
     assert np.all(np.isfinite(l2) | (l2 == -np.inf))
+
+
+def test_emulated_decoder_layers_equal_unsharded(csa2_lib):
+    """Full, Reuse, Reindex, Reuse through the emulated sharded decoder (the
+    bench's 1M leg): index sets equal the unsharded calls', outputs within the
+    parity bound of the unsharded outputs."""
+    import workload
+    workload.build_cuda()
+    from fp4_kv_cache_decode_b200 import synthetic as syn
+    from fp4_kv_cache_decode_b200.sharded import EmulatedDecoder, shard_bounds
+    from workload import device as wdev
+    csa2 = csa2_lib
+    layers = ["F", "R", "RI", "R"]
+    w = small_workload(LENGTHS, seed=67, heads=HEADS, spare_pages=64)
+    w.layers = list(layers)
+    cache = syn.new_cache(w)
+    syn.fill_decode_cache(w, cache)
+    full = syn.DecodeStep(w, cache, layers=["F"])
+    full.run(append=False)
+    step = syn.DecodeStep(w, cache)
+    step.run(append=False)
+    S = 3
+    bounds = [shard_bounds(L, S) for L in LENGTHS]
+    lens = [hi - lo for sh in bounds for lo, hi in sh]
+    cs = syn.new_cache(small_workload(lens, seed=w.seed, heads=HEADS, spare_pages=64), lengths=lens)
+    syn.fill_sharded_cache(w, cs, bounds)
+    B = len(LENGTHS)
+    off = torch.tensor([lo for sh in bounds for lo, _ in sh], dtype=torch.int32, device="cuda")
+    wstart = torch.tensor([max(0, L - 128) for L in LENGTHS], dtype=torch.int32, device="cuda")
+    dec = EmulatedDecoder(cs, S, off, wstart, HEADS, max(lens))
+    for l, m in enumerate(layers):
+        q = wdev.q_batch(w.seed, l, 0, B, HEADS)
+        if m == "F":
+            o = dec.full(wdev.idxq_batch(w.seed, l, 0, B), q)
+            np.testing.assert_array_equal(dec.buf.pool.cpu().numpy(), full.iset.pool_blocks.cpu().numpy())
+            np.testing.assert_array_equal(dec.buf.idx.cpu().numpy(), full.iset.idx.cpu().numpy())
+        elif m == "RI":
+            o = dec.reindex(wdev.idxq_batch(w.seed, l, 0, B), q)
+            np.testing.assert_array_equal(dec.buf.idx.cpu().numpy(), step.iset.idx.cpu().numpy())
+        else:
+            o = dec.reuse(q)
+        got, want = bits(o), bits(step.out[l])
+        for b in range(B):
+            ref = bf16_to_f64(want[b])
+            bound = 1e-2 * float(np.abs(ref).max()) + 1e-3
+            assert float(np.max(np.abs(bf16_to_f64(got[b]) - ref))) <= bound, f"layer {l} seq {b}"
+    torch.cuda.synchronize()
+    assert csa2.csa2_check_device_error(cs) == 0 and csa2.csa2_check_device_error(cache) == 0
