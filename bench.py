@@ -248,6 +248,15 @@ def run_gpu(args):
     clocks = sampler.stop()
     step_ms = np.array([events[k][0].elapsed_time(events[k][1]) for k in range(args.steps)])
     total_ms = float(step_ms.sum())
+    # diagnostic outside the timed region: the same replays without the L2 flush
+    # (inputs and kernel code left in L2 by the previous step)
+    warm = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for k in range(args.steps):
+        warm[k][0].record(stream)
+        graph.replay()
+        warm[k][1].record(stream)
+    torch.cuda.synchronize()
+    warm_ms = float(np.median([e[0].elapsed_time(e[1]) for e in warm]))
 
     # diagnostics outside the timed region: (1) a per-call breakdown from eager steps
     # with an event between calls (each event adds a little to its call); (2) the
@@ -362,6 +371,8 @@ def run_gpu(args):
         "ms_per_call": {c: float(m) for c, m in zip(calls, mean_call)},
         "ms_per_call_note": "diagnostic: eager steps outside the timed region, one event between calls",
         "ms_graph": {"attention_launch": reuse_ms, "indexer_full": idx_full_ms, "indexer_reindex": idx_ri_ms},
+        "ms_per_step_warm_l2": warm_ms,
+        "ms_per_step_warm_l2_note": "median of graph replays back to back with no L2 flush (diagnostic)",
         "roofline": dom,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"],
@@ -375,9 +386,13 @@ def run_gpu(args):
         result["max_pooled_blocks"] = measure_max_pool(w, cache, step, stream, flush, peaks, idx_full_ms)
         result["fp8_indexer_keys"] = measure_fp8_keys(
             w, stream, flush, peaks, {"step": ms_per_step, "full": idx_full_ms, "reindex": idx_ri_ms})
-        result["workloads"] = measure_workloads(stream, flush, rank)
+        result["workloads"] = measure_workloads(stream, flush, peaks, rank)
+        result["sharded_1m"] = measure_sharded_1m(stream, flush, result["workloads"]["config2"]["step_ms"], rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(args, seqs=tuple(range(w.batch)))
+        result["cpu_baseline"] = cpu_baseline(args)
+        if "workloads" in result:
+            for k, v in workload_baselines().items():
+                result["workloads"][k]["cpu_baseline"] = v
     finish_ranks(world)
     if rank == 0:
         print(json.dumps(result), flush=True)
@@ -502,69 +517,179 @@ def measure_max_pool(w, cache, step, stream, flush, peaks, mean_full_ms):
             "note": "median of CUDA-graph replays, L2 flushed first; bytes = every visible bf16 key once"}
 
 
-def measure_workloads(stream, flush, seed_rank: int = 0):
-    """Throughput of the other seeded workloads on this GPU, outside the timed
-    region: each step captured once as a CUDA graph and replayed (median of 5, L2
-    flushed first); inputs generated before the graph.  A decode layer-step is
-    one layer over the whole batch; a prefill chunk is the chunk's append, its
-    flat indexer over 8,192 queries and its Full + 5 Reuse attention layers."""
+def _set_rows(idx, lens):
+    """Attended rows of index sets (selected positions outside the window, plus
+    the window) given each query's visible length."""
+    return sum(_attended_rows(r, int(L)) for r, L in zip(idx, lens))
+
+
+def measure_workloads(stream, flush, peaks, seed_rank: int = 0):
+    """The other seeded workloads on this GPU, outside the timed region, each
+    step captured once as a CUDA graph and replayed (median of 5, L2 flushed
+    before each replay); inputs generated before the graph.  A decode
+    layer-step is one layer over the whole batch.  Algorithmic bytes: gathered
+    FP4 rows (288 B each, counted from the step's own index sets), indexer keys
+    read (block keys and pool keys, 128 B each) and, for the ragged batch, the
+    replay's rows in and out; the prefill is tensor-bound and reports FLOPs."""
     import torch
 
     import workload as wl
     from workload import device as wdev
     from fp4_kv_cache_decode_b200 import csa2, synthetic
+    hbm = peaks["hbm_gbs"]
     out = {}
-    for cid in (0, 2, 4):
+
+    def hbm_leg(w, ms, nbytes, units, what):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return {"workload": w.name, "step": what, "step_ms": ms, "layer_steps_per_s": units / (ms * 1e-3),
+                "tokens_per_s": w.batch / (ms * 1e-3), "algorithmic_bytes": nbytes, "hbm_gbs": gbs,
+                "hbm_frac": gbs / hbm}
+
+    for cid in (0, 2):
         w = wl.workload(cid)
         w.seed = rank_seed(w.seed, seed_rank)
         cache = synthetic.new_cache(w)
         synthetic.fill_decode_cache(w, cache)
-        if cid == 4:
-            step = synthetic.RaggedStep(w, cache)
-            step.setup()
-            layers = 1
-        else:
-            step = synthetic.DecodeStep(w, cache)
-            layers = len(w.layers)
+        step = synthetic.DecodeStep(w, cache)
         step.run()
+        full = synthetic.DecodeStep(w, cache, layers=["F"])
+        full.run(append=False)
         torch.cuda.synchronize()
         assert csa2.csa2_check_device_error(cache) == 0
         ms = _graph_ms(step.run, flush, stream)
-        out[f"config{cid}"] = {"workload": w.name, "step_ms": ms, "layer_steps_per_s": layers / (ms * 1e-3),
-                               "tokens_per_s": w.batch / (ms * 1e-3)}
-        del step, cache
+        lens = [w.lengths[s] for s in step.seqs]
+        rows_f = _set_rows(full.iset.idx.cpu().numpy(), lens)
+        rows_ri = _set_rows(step.iset.idx.cpu().numpy(), lens)
+        nbytes, group = 0, rows_f
+        for m in w.layers:
+            if m == "RI":
+                group = rows_ri
+            nbytes += group * 288
+            nb = [(L + 7) // 8 for L in lens]
+            if m == "F":   # flat: every key; hierarchical: block keys + the pool's keys
+                nbytes += sum(n * 8 * 128 if n <= 2048 else n * 128 + 16384 * 128 for n in nb)
+            elif m == "RI":
+                nbytes += sum(min(n, 2048) * 8 * 128 for n in nb)
+        out[f"config{cid}"] = hbm_leg(w, ms, nbytes, len(w.layers), "append + every layer")
+        del step, full, cache
         torch.cuda.empty_cache()
-    # encoder chunked prefill: the last chunk (the longest visible prefix)
+
+    w = wl.workload(4)
+    w.seed = rank_seed(w.seed, seed_rank)
+    cache = synthetic.new_cache(w)
+    synthetic.fill_decode_cache(w, cache)
+    st = synthetic.RaggedStep(w, cache)
+    st.setup()
+    st.run()
+    torch.cuda.synchronize()
+    assert csa2.csa2_check_device_error(cache) == 0
+    ms = _graph_ms(st.run, flush, stream)
+    ri, ru = st.groups["ri"], st.groups["ru"]
+    rows = (_set_rows(ri["iset"].idx.cpu().numpy(), [w.lengths[s] for s in st.ri]) +
+            _set_rows(ru["iset"].idx.cpu().numpy(), [w.lengths[s] for s in st.ru]))
+    pool_keys = sum(min((w.lengths[s] + 7) // 8, 2048) * 8 * 128 for s in st.ri)
+    n_rep = sum(min(128, w.lengths[b]) if w.miss_mask[b] else 1 for b in range(w.batch))
+    nbytes = rows * 288 + pool_keys + n_rep * (1024 + 128 + 288 + 128)
+    out["config4"] = hbm_leg(w, ms, nbytes, 1, "replay + one layer (16 Reindex, 48 Reuse)")
+    del st, cache
+    torch.cuda.empty_cache()
+
+    # encoder chunked prefill, the whole sequence: 16 chunks, each the append of
+    # its 8,192 raw tokens, the flat indexer of its 8,192 queries and the Full +
+    # 5 Reuse attention layers (one query tensor serves every layer and chunk:
+    # the work does not depend on the values)
     w = wl.workload(3)
     w.seed = rank_seed(w.seed, seed_rank)
     cache = synthetic.new_cache(w)
     nchunk = w.raw_tokens // w.chunk
-    for ci in range(nchunk):
-        synthetic.fill_prefill_chunk(w, cache, ci)
-    ch = synthetic.PrefillChunk(w, cache, nchunk - 1)
-    r0 = (nchunk - 1) * w.chunk
-    col = torch.from_numpy(wl.kv_col_scale(w.seed)).cuda()
-    kv = wdev.kv_rows(w.seed, 0, r0, w.chunk, col_scale=col)
-    k = wdev.idxk_rows(w.seed, 0, r0, w.chunk)
     n_e = w.chunk // w.compress
-    eseq = torch.zeros(n_e, dtype=torch.int32, device="cuda")
-    epos = torch.arange(r0 // w.compress, r0 // w.compress + n_e, dtype=torch.int32, device="cuda")
-    q = ch.queries(0).clone()
+    last_vis = w.raw_tokens // w.compress
+    ws = torch.empty(csa2.csa2_workspace_bytes(csa2.OP_INDEXER, w.chunk, 0, last_vis, False), dtype=torch.uint8,
+                     device="cuda")
+    obuf = torch.empty((w.chunk, w.heads, 512), dtype=torch.bfloat16, device="cuda")
+    col = torch.from_numpy(wl.kv_col_scale(w.seed)).cuda()
+    chunks, inputs = [], []
+    for ci in range(nchunk):
+        r0 = ci * w.chunk
+        chunks.append(synthetic.PrefillChunk(w, cache, ci, ws_idx=ws, out=obuf))
+        inputs.append((wdev.kv_rows(w.seed, 0, r0, w.chunk, col_scale=col), wdev.idxk_rows(w.seed, 0, r0, w.chunk),
+                       torch.zeros(n_e, dtype=torch.int32, device="cuda"),
+                       torch.arange(r0 // w.compress, r0 // w.compress + n_e, dtype=torch.int32, device="cuda")))
+    q = chunks[-1].queries(0).clone()
+    cache.seq_lens[0] = last_vis
 
-    def chunk_step():
+    def prefill():
+        for ch, (kv, k, eseq, epos) in zip(chunks, inputs):
+            csa2.csa2_kv_quant_append(cache, kv, k, eseq, epos, w.compress)
+            ch.indexer()
+            for layer in range(len(w.layers)):
+                ch.attention(layer, q=q)
+    # one eager pass: attended rows of every query (for the FLOP count)
+    rows = 0
+    for ch, (kv, k, eseq, epos) in zip(chunks, inputs):
         csa2.csa2_kv_quant_append(cache, kv, k, eseq, epos, w.compress)
         ch.indexer()
-        for layer in range(len(w.layers)):
-            ch.attention(layer, q=q)
-    chunk_step()
-    torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        rows += _set_rows(ch.iset.idx.cpu().numpy(), ch.q_vis.cpu().numpy())
     assert csa2.csa2_check_device_error(cache) == 0
-    ms = _graph_ms(chunk_step, flush, stream)
-    out["config3"] = {"workload": w.name, "step_ms": ms, "layer_steps_per_s": len(w.layers) / (ms * 1e-3),
-                      "tokens_per_s": w.chunk / (ms * 1e-3), "step": "one 8,192-token chunk"}
-    del ch, cache
+    ms = _graph_ms(prefill, flush, stream, reps=3)
+    vis = np.concatenate([ch.q_vis.cpu().numpy() for ch in chunks]).astype(np.float64)
+    flops_attn = 4.0 * w.heads * 512 * rows * len(w.layers)
+    flops_idx = 2.0 * 4 * 64 * float(vis.sum())
+    tf = (flops_attn + flops_idx) / (ms * 1e-3) / 1e12
+    out["config3"] = {"workload": w.name, "step": f"the whole prefill: {nchunk} chunks of {w.chunk} queries",
+                      "step_ms": ms, "tokens_per_s": w.raw_tokens / (ms * 1e-3),
+                      "layer_steps_per_s": len(w.layers) * nchunk / (ms * 1e-3),
+                      "flops": flops_attn + flops_idx, "flops_attention": flops_attn, "flops_indexer": flops_idx,
+                      "tflops": tf, "bound": "tensor", "tensor_frac": tf / peaks["bf16_tflops"],
+                      "append_bytes": w.raw_tokens * (1024 + 128) + last_vis * (288 + 128)}
+    del chunks, inputs, cache, ws, obuf
     torch.cuda.empty_cache()
     return out
+
+
+def measure_sharded_1m(stream, flush, unsharded_ms: float | None, seed_rank: int = 0, nshard: int = 4):
+    """The 4 x 1M decode step position-sharded over `nshard` shards, every shard
+    emulated on this GPU (the shards are separate sequences of one cache; the
+    all-gathers become strided reads): Full, Reindex and Reuse layers of the
+    20-layer schedule through the sharded calls, as one CUDA graph.  The time is
+    the sum of all shards' work on one GPU -- what one GPU of S would do is
+    about a 1/S share of the sharded calls plus the exchanges."""
+    import torch
+
+    import workload as wl
+    from workload import device as wdev
+    from fp4_kv_cache_decode_b200 import synthetic
+    from fp4_kv_cache_decode_b200.sharded import EmulatedDecoder, shard_bounds
+    w = wl.workload(2)
+    w.seed = rank_seed(w.seed, seed_rank)
+    bounds = [shard_bounds(L, nshard) for L in w.lengths]
+    lens = [hi - lo for sh in bounds for lo, hi in sh]
+    cache = synthetic.new_cache(w, lengths=lens)
+    synthetic.fill_sharded_cache(w, cache, bounds)
+    B = w.batch
+    off = torch.tensor([lo for sh in bounds for lo, _ in sh], dtype=torch.int32, device="cuda")
+    wstart = torch.tensor([max(0, L - 128) for L in w.lengths], dtype=torch.int32, device="cuda")
+    dec = EmulatedDecoder(cache, nshard, off, wstart, w.heads, max(lens))
+    iq = {l: wdev.idxq_batch(w.seed, l, 0, B) for l, m in enumerate(w.layers) if m in ("F", "RI")}
+    q = [wdev.q_batch(w.seed, l, 0, B, w.heads) for l in range(len(w.layers))]
+
+    def step():
+        for l, m in enumerate(w.layers):
+            if m == "F":
+                dec.full(iq[l], q[l])
+            elif m == "RI":
+                dec.reindex(iq[l], q[l])
+            else:
+                dec.reuse(q[l])
+    step()
+    torch.cuda.synchronize()
+    ms = _graph_ms(step, flush, stream)
+    del dec, cache
+    torch.cuda.empty_cache()
+    return {"workload": w.name, "shards": nshard, "step_ms": ms, "layer_steps_per_s": len(w.layers) / (ms * 1e-3),
+            "unsharded_step_ms": unsharded_ms,
+            "note": "all shards emulated on one GPU (sum of every shard's work), CUDA graph, L2 flushed first"}
 
 
 def measure_fp8_keys(w, stream, flush, peaks, bf16_ms):
@@ -687,93 +812,325 @@ def run_e2e(args, w, step, stream, flush):
 # CPU oracle arm
 # ---------------------------------------------------------------------------
 
-def _oracle_sample(w, seqs):
-    """Host inputs of a bounded sample (whole sequences of the workload)."""
-    import workload as wl
+def host_threads() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+class _Rows:
+    """bf16 KV rows of one sequence by entry position, generated on first use and
+    kept (input generation, not oracle work: the warm-up step fills it).  At
+    compression ratio 2 an entry is made of raw rows 2e and 2e + 1."""
+
+    def __init__(self, seed: int, seq: int, compress: int = 1):
+        self.seed, self.seq, self.compress = seed, seq, compress
+        self.bits = {}
+
+    def __call__(self, pos):
+        import workload as wl
+        c = self.compress
+        for p in pos.tolist():
+            if p not in self.bits:
+                self.bits[p] = wl.kv_rows(self.seed, self.seq, c * p, c)
+        return np.concatenate([self.bits[p] for p in pos.tolist()]) if len(pos) else \
+            np.zeros((0, 512), np.uint16)
+
+
+def _decoded(rows: _Rows, pos):
+    """The oracle's decoded FP4 rows of the given entry positions."""
     from oracle import codec as ocodec
-    L = w.lengths[0]
-    data = []
+    c, sc = ocodec.unpack_rows(ocodec.encode_entries(rows(pos), rows.compress))
+    return ocodec.dequantize(c, sc)
+
+
+def _decode_setup(w, seqs):
+    import workload as wl
+    out = []
     for s in seqs:
-        keys = wl.idxk_rows(w.seed, s, 0, L)
-        kv_bits = wl.kv_rows(w.seed, s, 0, L)
-        iq = {l: wl.idxq_rows(w.seed, l, s) for l, m in enumerate(w.layers) if m in ("F", "RI")}
-        q = {l: wl.q_rows(w.seed, l, s, w.heads) for l in range(len(w.layers))}
-        data.append((keys, kv_bits, iq, q))
-    return data
+        L = w.lengths[s]
+        out.append({
+            "s": s, "L": L, "keys": wl.idxk_rows(w.seed, s, 0, L), "rows": _Rows(w.seed, s),
+            "new": wl.kv_rows(w.seed, s, L - 1, 1),
+            "iq": {l: wl.idxq_rows(w.seed, l, s) for l, m in enumerate(w.layers) if m in ("F", "RI")},
+            "q": {l: wl.q_rows(w.seed, l, s, w.heads) for l in range(len(w.layers))}})
+    return out
 
 
-def _oracle_step(w, sample):
-    """The oracle's whole decode step for the sampled sequences: encode the cache
-    rows the step reads, then run the layer schedule."""
+def _decode_step(w, state):
+    """One decode step of the oracle for its sequences: encode the appended token,
+    then the layer schedule (Full / Reindex indexer, attention over decoded rows)."""
     from oracle import codec as ocodec
     from oracle import modes as omodes
-    L = w.lengths[0]
-    for keys, kv_bits, iq, q in sample:
-        rows_cache = {}
+    for st in state:
+        ocodec.encode_bf16_rows(st["new"])
+        dec = {}
 
-        def rows(pos, kv_bits=kv_bits, rows_cache=rows_cache):
-            miss = [p for p in pos.tolist() if p not in rows_cache]
-            if miss:
-                enc = ocodec.encode_bf16_rows(kv_bits[np.asarray(miss)])
-                c, s = ocodec.unpack_rows(enc)
-                dec = ocodec.dequantize(c, s)
-                for p, r in zip(miss, dec):
-                    rows_cache[p] = r
-            return np.stack([rows_cache[p] for p in pos.tolist()])
+        def rows_fn(pos, st=st, dec=dec):
+            miss = np.asarray([p for p in pos.tolist() if p not in dec], dtype=np.int64)
+            if miss.size:
+                for p, r in zip(miss.tolist(), _decoded(st["rows"], miss)):
+                    dec[p] = r
+            return np.stack([dec[p] for p in pos.tolist()])
 
-        omodes.run_layers(w.layers, L, keys, lambda l: iq[l], lambda l: q[l], rows)
+        omodes.run_layers(w.layers, st["L"], st["keys"], lambda l, st=st: st["iq"][l],
+                          lambda l, st=st: st["q"][l], rows_fn)
 
 
-def _blas_threads() -> int:
+def _ragged_setup(w, seqs):
+    """Per sequence: keys, the earlier Full layer's pool and set (outside the step,
+    as on the GPU), the replay block and the layer's queries."""
+    import workload as wl
+    from oracle import indexer as oidx
+    out = []
+    for s in seqs:
+        L = w.lengths[s]
+        keys = wl.idxk_rows(w.seed, s, 0, L)
+        pool, idx, _ = oidx.full_indexer(wl.idxq_rows(w.seed, 0, s), keys, L)
+        n = min(128, L)
+        kv_last = np.zeros((128, 512), np.uint16)
+        k_last = np.zeros((128, 64), np.uint16)
+        kv_last[128 - n:] = wl.kv_rows(w.seed, s, L - n, n)
+        k_last[128 - n:] = wl.idxk_rows(w.seed, s, L - n, n)
+        out.append({"s": s, "L": L, "keys": keys, "pool": pool, "idx": idx, "rows": _Rows(w.seed, s),
+                    "kv_last": kv_last, "k_last": k_last, "ri": bool(w.reindex_mask[s]),
+                    "miss": bool(w.miss_mask[s]), "iq1": wl.idxq_rows(w.seed, 1, s),
+                    "q1": wl.q_rows(w.seed, 1, s, w.heads)})
+    return out
+
+
+def _ragged_step(w, state):
+    """Bounded replay (miss: the last 128 entries, else the newest), then one layer:
+    Reindex sequences rank the Full pool with their own query, Reuse sequences keep
+    the Full set; both attend."""
+    from oracle import attention as oattn
+    from oracle import indexer as oidx
+    from oracle import modes as omodes
+    for st in state:
+        omodes.replay_entries(st["kv_last"], st["L"], st["miss"])
+        omodes.replay_keys(st["k_last"], st["L"], st["miss"])
+        idx = oidx.reindex_indexer(st["iq1"], st["keys"], st["L"], st["pool"])[0] if st["ri"] else st["idx"]
+        pos = oattn.attended_positions(idx, st["L"])
+        oattn.attend(st["q1"], _decoded(st["rows"], pos))
+
+
+def prefill_queries(w, n: int = 1024) -> np.ndarray:
+    """Stratified sample of prefill query positions: every chunk's first and last
+    position, the rest a seeded draw from all positions (ascending)."""
+    import workload as wl
+    fixed = set()
+    for c in range(w.raw_tokens // w.chunk):
+        fixed.update((c * w.chunk, (c + 1) * w.chunk - 1))
+    perm = wl.permutation(w.seed, wl.stream_id(wl.TAG_LENS, 3), w.raw_tokens)
+    extra = [int(p) for p in perm if int(p) not in fixed][:n - len(fixed)]
+    return np.asarray(sorted(fixed | set(extra)), dtype=np.int64)
+
+
+def _prefill_setup(w, items):
+    """items: ("append", entry range) and ("query", raw position) units."""
+    import workload as wl
+    from oracle import codec as ocodec
+    st = {"append": [], "query": []}
+    keys = None
+    for kind, x in items:
+        if kind == "append":
+            e0, e1 = x
+            st["append"].append((wl.kv_rows(w.seed, 0, 2 * e0, 2 * (e1 - e0)),
+                                 wl.idxk_rows(w.seed, 0, 2 * e0, 2 * (e1 - e0))))
+        else:
+            if keys is None:
+                keys = ocodec.idxk_entries(wl.idxk_rows(w.seed, 0, 0, w.raw_tokens), w.compress)
+            st["query"].append({"P": x, "iq": wl.idxq_rows(w.seed, 0, x),
+                                "q": [wl.q_rows(w.seed, l, x, w.heads) for l in range(len(w.layers))]})
+    st["keys"], st["rows"] = keys, _Rows(w.seed, 0, w.compress)
+    return st
+
+
+def _prefill_step(w, st):
+    """The append of this worker's entry ranges (2:1 compression, FP4 encode, keys)
+    and, for each sampled query, the flat causal indexer plus the Full and Reuse
+    attention layers over the same set."""
+    from oracle import attention as oattn
+    from oracle import codec as ocodec
+    from oracle import indexer as oidx
+    for kv, k in st["append"]:
+        ocodec.encode_entries(kv, w.compress)
+        ocodec.idxk_entries(k, w.compress)
+    for qq in st["query"]:
+        v = oattn.prefill_visible(qq["P"], w.compress)
+        idx, _ = oidx.flat_indexer(qq["iq"], st["keys"], v)
+        pos = oattn.attended_positions(idx, v)
+        rows = _decoded(st["rows"], pos)
+        for q in qq["q"]:
+            oattn.attend(q, rows)
+
+
+_ORACLE_KINDS = {"decode": (_decode_setup, _decode_step), "ragged": (_ragged_setup, _ragged_step),
+                 "prefill": (_prefill_setup, _prefill_step)}
+
+
+def _oracle_worker(conn, cid: int, seed: int, kind: str, items) -> None:
+    """A spawned process: builds the inputs of its share of the sample once, then
+    runs the oracle over them each time the parent asks and reports the time."""
+    import workload as wl
+    w = wl.workload(cid)
+    w.seed = seed
+    setup, step = _ORACLE_KINDS[kind]
+    state = setup(w, items)
+    conn.send("ready")
+    while True:
+        msg = conn.recv()
+        if msg != "step":
+            break
+        t0 = time.perf_counter()
+        step(w, state)
+        conn.send(time.perf_counter() - t0)
+
+
+class OraclePool:
+    """The CPU oracle on the host cores: one spawned process per share of a
+    sample (started before or apart from any GPU work, never forked), one BLAS
+    thread each.  step() runs every share at once and returns the wall time."""
+
+    def __init__(self, cid: int, seed: int, kind: str, items, procs: int):
+        import multiprocessing as mp
+        items = list(items)
+        self.procs = max(1, min(procs, len(items)))
+        shares = [items[i::self.procs] for i in range(self.procs)]
+        ctx = mp.get_context("spawn")
+        saved = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+        for k in saved:
+            os.environ[k] = "1"
+        try:
+            self.conns, self.ps = [], []
+            for sh in shares:
+                a, b = ctx.Pipe()
+                p = ctx.Process(target=_oracle_worker, args=(b, cid, seed, kind, sh), daemon=True)
+                p.start()
+                self.conns.append(a)
+                self.ps.append(p)
+        finally:
+            for k, v in saved.items():
+                if v is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = v
+        for c in self.conns:
+            if c.recv() != "ready":
+                raise RuntimeError("oracle worker failed to start")
+
+    def step(self) -> float:
+        t0 = time.perf_counter()
+        for c in self.conns:
+            c.send("step")
+        for c in self.conns:
+            c.recv()
+        return time.perf_counter() - t0
+
+    def close(self) -> None:
+        for c in self.conns:
+            try:
+                c.send("stop")
+            except (BrokenPipeError, OSError):
+                pass
+        for p in self.ps:
+            p.join(timeout=30)
+
+
+def _baseline(cid, seed, kind, items, warmup, steps, procs=None):
+    """Wall seconds per step of the oracle over a sample (after `warmup` steps)."""
+    pool = OraclePool(cid, seed, kind, items, procs or host_threads())
     try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info()]
-        return max(n) if n else 1
-    except Exception:
-        return 1
+        for _ in range(warmup):
+            pool.step()
+        ts = [pool.step() for _ in range(steps)]
+    finally:
+        pool.close()
+    return float(np.median(ts)), pool.procs, ts
 
 
-def cpu_baseline(args, seqs=(0,)):
+def cpu_baseline(args, steps: int = 3, seed: int | None = None):
+    """The oracle's whole decode step (all 32 sequences, 8 layers) on the host cores."""
     import workload as wl
     w = wl.workload(CONFIG_ID)
-    sample = _oracle_sample(w, list(seqs))
-    t0 = time.perf_counter()
-    _oracle_step(w, sample)
-    dt = time.perf_counter() - t0
-    # layer-steps over the whole batch: the sample covers len(seqs) of B sequences
-    per_batch_step = dt * w.batch / len(seqs)
-    scale = "" if len(seqs) == w.batch else f", scaled x{w.batch / len(seqs):g} to the batch"
-    return {"value": len(w.layers) / per_batch_step, "unit": UNIT, "cores": _blas_threads(),
-            "kind": "oracle",
-            "sample": f"{len(seqs)} of {w.batch} sequences, all {len(w.layers)} layers of one step "
-                      f"(indexer + fp64 attention){scale}; {dt:.1f} s of CPU work"}
+    sec, procs, _ = _baseline(CONFIG_ID, w.seed if seed is None else seed, "decode", range(w.batch), 1, steps)
+    return {"value": len(w.layers) / sec, "unit": UNIT, "cores": procs, "nproc": host_threads(),
+            "cpu": _cpu_model(), "kind": "oracle", "ms_per_step": sec * 1e3,
+            "sample": f"the whole step: {w.batch} of {w.batch} sequences, all {len(w.layers)} layers "
+                      f"(append, indexer, fp64 attention); median of {steps} steps after 1 warm-up, "
+                      f"{procs} processes with one BLAS thread each"}
+
+
+def workload_baselines(seed_rank: int = 0):
+    """The oracle on the other workloads (bounded samples, host cores)."""
+    import workload as wl
+    out = {}
+    for cid, unit_per_step in ((0, 1), (2, 20), (4, 1)):
+        w = wl.workload(cid)
+        kind = "ragged" if cid == 4 else "decode"
+        sec, procs, _ = _baseline(cid, rank_seed(w.seed, seed_rank), kind, range(w.batch), 1, 2)
+        out[f"config{cid}"] = {
+            "value": unit_per_step / sec, "unit": UNIT, "cores": procs, "kind": "oracle",
+            "tokens_per_s": w.batch / sec, "ms_per_step": sec * 1e3,
+            "sample": f"the whole step ({w.batch} sequences); median of 2 steps after 1 warm-up"}
+    # prefill: the whole append plus a stratified sample of queries, extrapolated
+    w = wl.workload(3)
+    n_e = w.raw_tokens // w.compress
+    qs = prefill_queries(w)
+    procs = host_threads()
+    ranges = [("append", (e, min(n_e, e + 4096))) for e in range(0, n_e, 4096)]
+    sec_app, _, _ = _baseline(3, rank_seed(w.seed, seed_rank), "prefill", ranges, 0, 1, procs)
+    sec_q, used, _ = _baseline(3, rank_seed(w.seed, seed_rank), "prefill", [("query", int(p)) for p in qs],
+                               0, 1, procs)
+    total = sec_app + sec_q * w.raw_tokens / len(qs)
+    out["config3"] = {
+        "value": w.raw_tokens / total, "unit": "tokens/s", "cores": used, "kind": "oracle",
+        "extrapolated": True, "prefill_s": total, "append_s": sec_app,
+        "sample": f"the whole append ({w.raw_tokens} raw tokens -> {n_e} entries) timed in full; "
+                  f"{len(qs)} stratified queries (every chunk's first and last position + seeded draws; "
+                  f"flat indexer + {len(w.layers)} attention layers) timed and scaled x{w.raw_tokens / len(qs):g} "
+                  f"to all {w.raw_tokens} queries"}
+    return out
 
 
 def run_reference(args):
+    """The oracle as it stands on the host cores, on the same workload and metric:
+    every timed step is the whole decode step of all 32 sequences."""
     world, rank, _ = rank_env()
     if rank != 0:
         return
     import workload as wl
     w = wl.workload(CONFIG_ID)
-    seqs = list(range(8))
-    sample = _oracle_sample(w, seqs)
-    for _ in range(args.warmup):
-        _oracle_step(w, sample)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        _oracle_step(w, sample)
-    dt = time.perf_counter() - t0
-    per_batch_step = dt / args.steps * w.batch / len(seqs)
-    value = len(w.layers) / per_batch_step
-    cores = _blas_threads()
+    pool = OraclePool(CONFIG_ID, w.seed, "decode", range(w.batch), host_threads())
+    try:
+        for _ in range(args.warmup):
+            pool.step()
+        ts = [pool.step() for _ in range(args.steps)]
+    finally:
+        pool.close()
+    total = float(sum(ts))
+    value = len(w.layers) * args.steps / total
     result = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_batch_step * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded)", "config": _config_json(w, world),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"{len(seqs)} of {w.batch} sequences per step (all "
-                                   f"{len(w.layers)} layers), scaled x{w.batch // len(seqs)} to the batch"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": pool.procs, "nproc": host_threads(),
+                         "cpu": _cpu_model(), "kind": "oracle",
+                         "sample": f"the whole step every step: {w.batch} of {w.batch} sequences, all "
+                                   f"{len(w.layers)} layers, {pool.procs} processes with one BLAS thread each"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(result), flush=True)

@@ -176,7 +176,10 @@ class PrefillChunk:
     """Queries of one prefill chunk (encoder, flat indexer, causal visibility):
     Full indexer over [0, v(P)) per query, then the Full + Reuse attention layers."""
 
-    def __init__(self, w: wl.Workload, cache: csa2.Cache, chunk_index: int, queries=None):
+    def __init__(self, w: wl.Workload, cache: csa2.Cache, chunk_index: int, queries=None, ws_idx=None,
+                 out=None):
+        """ws_idx / out: an indexer workspace and an output buffer to use instead
+        of allocating them (chunks run one after another can share them)."""
         self.w, self.cache = w, cache
         r0 = chunk_index * w.chunk
         qpos = np.arange(r0, r0 + w.chunk) if queries is None else np.asarray(queries)
@@ -188,18 +191,23 @@ class PrefillChunk:
         self.q_seq = torch.zeros(self.nq, dtype=torch.int32, device=dev)
         self.max_visible = int(vis.max())
         self.iset = csa2.IndexSet(self.nq)
-        self.ws_idx = torch.empty(csa2.csa2_workspace_bytes(csa2.OP_INDEXER, self.nq, 0, self.max_visible,
-                                                            False), dtype=torch.uint8, device=dev)
+        need = csa2.csa2_workspace_bytes(csa2.OP_INDEXER, self.nq, 0, self.max_visible, False)
+        if ws_idx is not None and ws_idx.numel() < need:
+            raise ValueError("shared indexer workspace too small")
+        self.ws_idx = ws_idx if ws_idx is not None else torch.empty(need, dtype=torch.uint8, device=dev)
         self.ws_attn = torch.empty(csa2.csa2_workspace_bytes(csa2.OP_ATTENTION, self.nq, w.heads),
                                    dtype=torch.uint8, device=dev)
         contiguous = queries is None
         self.idxq = (wdev.idxq_batch(w.seed, 0, int(qpos[0]), self.nq) if contiguous else
                      torch.cat([wdev.idxq_batch(w.seed, 0, int(p), 1) for p in qpos]))
-        self.out = torch.empty((self.nq, w.heads, 512), dtype=torch.bfloat16, device=dev)
-        self.q_buf = torch.empty((self.nq, w.heads, 512), dtype=torch.bfloat16, device=dev)
+        self.out = out if out is not None else torch.empty((self.nq, w.heads, 512), dtype=torch.bfloat16,
+                                                           device=dev)
+        self.q_buf = None
 
     def queries(self, layer: int):
         if len(self.qpos) and np.all(np.diff(self.qpos) == 1):
+            if self.q_buf is None:
+                self.q_buf = torch.empty((self.nq, self.w.heads, 512), dtype=torch.bfloat16, device="cuda")
             return wdev.q_batch(self.w.seed, layer, int(self.qpos[0]), self.nq, self.w.heads, out=self.q_buf)
         return torch.cat([wdev.q_batch(self.w.seed, layer, int(p), 1, self.w.heads) for p in self.qpos])
 

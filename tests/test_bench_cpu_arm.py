@@ -1,0 +1,39 @@
+"""The benchmark's CPU oracle arm, on CPU: the spawned worker pool runs a small
+workload's whole step and reports wall times; the prefill query sample holds
+every chunk's first and last position and nothing twice."""
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def test_prefill_query_sample_is_stratified():
+    import bench
+    import workload as wl
+    w = wl.workload(3)
+    qs = bench.prefill_queries(w)
+    assert len(qs) == 1024 and np.all(np.diff(qs) > 0)
+    assert qs[0] >= 0 and qs[-1] < w.raw_tokens
+    for c in range(w.raw_tokens // w.chunk):
+        assert c * w.chunk in qs and (c + 1) * w.chunk - 1 in qs
+    np.testing.assert_array_equal(qs, bench.prefill_queries(w))     # seeded
+
+
+def test_oracle_pool_times_a_whole_step():
+    import bench
+    sec, procs, ts = bench._baseline(0, 0, "decode", [0], warmup=1, steps=2, procs=2)
+    assert procs == 1 and len(ts) == 2 and all(t > 0 for t in ts) and sec > 0
+
+
+def test_oracle_pool_splits_items_over_processes():
+    import bench
+    pool = bench.OraclePool(3, 3, "prefill", [("query", 5), ("query", 70000), ("append", (0, 64))], 2)
+    try:
+        assert pool.procs == 2 and pool.step() > 0
+    finally:
+        pool.close()
+    assert all(p.exitcode == 0 for p in pool.ps)
