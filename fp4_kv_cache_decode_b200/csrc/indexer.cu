@@ -551,18 +551,20 @@ __device__ __forceinline__ void topk_registers(const float* __restrict__ srow, i
   const uint32_t tot_gt = tot >> 16, tot_eq = tot & 0xFFFFu;
   uint32_t slot = gt_before + min(eq_before, need_eq);
   uint32_t eq_rank = eq_before;
+  if (ngt + neq > 0) {   // most threads select nothing
 #pragma unroll
-  for (int j = 0; j < kKeysPerThread; ++j) {
-    const uint32_t kj = key[j];
-    bool sel = kj != 0u && kj > T;
-    if (kj != 0u && kj == T) sel = eq_rank++ < need_eq;
-    if (sel && slot < (uint32_t)k) {
-      int32_t o;
-      if (SRC == SRC_POOL) o = (j < 8 ? pb0 : pb1) * kBlock + (int32_t)((lo + j) & 7);
-      else if (SRC == SRC_CAND) o = pool_row[lo + j];
-      else o = (int32_t)(lo + j);
-      if (oscore) oscore[slot] = key_score(kj);
-      orow[slot++] = o + id_off;
+    for (int j = 0; j < kKeysPerThread; ++j) {
+      const uint32_t kj = key[j];
+      bool sel = kj != 0u && kj > T;
+      if (kj != 0u && kj == T) sel = eq_rank++ < need_eq;
+      if (sel && slot < (uint32_t)k) {
+        int32_t o;
+        if (SRC == SRC_POOL) o = (j < 8 ? pb0 : pb1) * kBlock + (int32_t)((lo + j) & 7);
+        else if (SRC == SRC_CAND) o = pool_row[lo + j];
+        else o = (int32_t)(lo + j);
+        if (oscore) oscore[slot] = key_score(kj);
+        orow[slot++] = o + id_off;
+      }
     }
   }
   const uint32_t total = tot_gt + min(tot_eq, need_eq);

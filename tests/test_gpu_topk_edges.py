@@ -15,18 +15,19 @@ from tests.gpu_util import small_workload
 
 pytestmark = pytest.mark.gpu
 
-LENGTHS = [20000, 20000, 3000, 16400, 20000]
-CASES = ["zero", "few", "few", "random", "random"]
+LENGTHS = [20000, 20000, 3000, 16400, 20000, 20000]
+CASES = ["zero", "few", "few", "random", "random", "two"]
 HEAD_W = [[1.0, 1.0, 1.0, 1.0], [1.0, 1.0, 1.0, 1.0], [1.0, 0.5, 2.0, 1.0],
-          [1.0, -1.0, 0.5, -2.0], [-1.0, -0.25, -3.0, -0.5]]
+          [1.0, -1.0, 0.5, -2.0], [-1.0, -0.25, -3.0, -0.5], [1.0, 1.0, 1.0, 1.0]]
 
 
 def _keys(case: str, seed: int, seq: int, L: int) -> np.ndarray:
     if case == "zero":
         return np.zeros((L, 64), dtype=np.uint16)
-    if case == "few":
-        base = wl.idxk_rows(seed + 1, seq, 0, 5)
-        pick = (np.arange(L, dtype=np.uint64) * np.uint64(2654435761) >> np.uint64(7)) % np.uint64(5)
+    if case in ("few", "two"):   # keys drawn from 5 (or 2: thousands of equal scores) vectors
+        m = 5 if case == "few" else 2
+        base = wl.idxk_rows(seed + 1, seq, 0, m)
+        pick = (np.arange(L, dtype=np.uint64) * np.uint64(2654435761) >> np.uint64(7)) % np.uint64(m)
         return base[pick.astype(np.int64)]
     return wl.idxk_rows(seed, seq, 0, L)
 
