@@ -35,7 +35,9 @@ METRIC = "CSA2 decode layer-steps/s at 64K ctx; achieved HBM GB/s vs B200 peak"
 UNIT = "layer-steps/s"
 CONFIG_ID = 1
 # dram__bytes_read.sum + dram__bytes_write.sum of one attn_pipe_kernel launch on this
-# workload (ncu, three launches: 9.708, 9.704, 9.800 MB read, 0 written)
+# workload (ncu, three launches: 9.709, 9.703, 9.799 MB read, 0 written), captured with
+# the pool sized to the batch -- the same rows, queries and outputs per launch as the
+# 4 GiB pool, only the rows' page addresses differ
 ATTN_DRAM_BYTES_PER_LAUNCH = 9.74e6
 L2_FLUSH_BYTES = 256 << 20
 
