@@ -739,9 +739,6 @@ namespace csa2 {
 size_t topk_smem_bytes() { return sizeof(TopkSmem); }
 
 cudaError_t score_mma_set_attributes();
-cudaError_t launch_score_mma_fp8(const CacheView& c, const uint16_t* idx_q, const float* head_w,
-                                 const int32_t* q_seq, const int32_t* q_vis, const int32_t* pool, int nq,
-                                 int64_t max_units, int64_t stride, float* scores, cudaStream_t st);
 cudaError_t launch_score_mma(int src, const CacheView& c, const uint16_t* idx_q, const float* head_w,
                              const int32_t* q_seq, const int32_t* q_vis, const int32_t* pool, int nq,
                              int64_t max_units, int64_t stride, float* scores, float* block_max, int64_t bstride,
@@ -758,7 +755,8 @@ cudaError_t indexer_set_attributes() {
   cudaError_t e = cudaSuccess;
   for (const void* k : topk_kernels)
     if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  const void* score_kernels[] = {(const void*)score_units_kernel<SRC_FLAT, true>};
+  const void* score_kernels[] = {(const void*)score_units_kernel<SRC_FLAT, true>,
+                                 (const void*)score_units_kernel<SRC_POOL, true>};
   for (const void* k : score_kernels)
     if (e == cudaSuccess) e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreSmemMax);
   if (e == cudaSuccess) e = score_mma_set_attributes();
@@ -771,13 +769,10 @@ cudaError_t launch_score(int src, const CacheView& c, const uint16_t* idx_q, con
                          int64_t max_units, int64_t stride, float* scores, float* block_max,
                          int64_t bstride, cudaStream_t st) {
   // bf16 keys (and block keys, always bf16): tensor-core scoring (score_mma.cu);
-  // FP8 keys: the pool on the tensor cores (score_mma.cu), flat scoring on the
-  // FFMA kernel below
+  // FP8 keys: the FFMA kernel below
   if (!c.idxk_fp8 || src == SRC_BLOCKKEYS)
     return launch_score_mma(src, c, idx_q, head_w, q_seq, q_vis, pool, nq, max_units, stride, scores, block_max,
                             bstride, st);
-  if (src == SRC_POOL)
-    return launch_score_mma_fp8(c, idx_q, head_w, q_seq, q_vis, pool, nq, max_units, stride, scores, st);
   // units per CTA: enough CTAs for two per SM over the whole batch, in whole
   // 32-unit stages, at most 256
   int sms = 148, dev = 0;
@@ -792,8 +787,12 @@ cudaError_t launch_score(int src, const CacheView& c, const uint16_t* idx_q, con
   if (upc < stage_units) upc = stage_units;
   dim3 grid((unsigned)((max_units + upc - 1) / upc), (unsigned)nq);
   if (grid.x == 0) return cudaSuccess;
-  launch_pdl(score_units_kernel<SRC_FLAT, true>, grid, kScoreThreads, smem, st, c, idx_q, head_w, q_seq, q_vis, pool,
-             max_units, stride, (int)upc, scores, block_max, bstride);
+  if (src == SRC_FLAT)
+    launch_pdl(score_units_kernel<SRC_FLAT, true>, grid, kScoreThreads, smem, st, c, idx_q, head_w, q_seq, q_vis,
+               pool, max_units, stride, (int)upc, scores, block_max, bstride);
+  else
+    launch_pdl(score_units_kernel<SRC_POOL, true>, grid, kScoreThreads, smem, st, c, idx_q, head_w, q_seq, q_vis,
+               pool, max_units, stride, (int)upc, scores, block_max, bstride);
   return cudaGetLastError();
 }
 

@@ -493,330 +493,6 @@ __global__ void __launch_bounds__(kSmThreads, 1) score_mma_group_kernel(
   }
 }
 
-// Two fp32 -> f16x2 (round to nearest even), the first in the low half.
-__device__ __forceinline__ uint32_t pack_f16x2_rn(float lo, float hi) {
-  uint32_t d;
-  asm("cvt.rn.f16x2.f32 %0, %2, %1;" : "=r"(d) : "f"(lo), "f"(hi));
-  return d;
-}
-
-// Two E4M3 codes (low byte first) -> f16x2 (exact).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t pair) {
-  uint32_t h;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((unsigned short)(pair & 0xFFFFu)));
-  return h;
-}
-
-// ---- pool scoring with FP8 keys ----
-//
-// FP8 indexer keys (E4M3 codes, one fp32 scale per key; a page holds its 64
-// keys' codes, 64 B each, then their 64 scales) on the tensor cores.  Per
-// 8-key unit the producer copies the 512 B of codes with one TMA tile copy
-// into a ring of kF8RawStages landing stages; eight converter warps turn a
-// tile's codes into f16 (exact: every E4M3 value is an f16 value) in one of
-// two 128-byte-swizzled K-major operand buffers -- two lanes per key, each
-// taking two of its four 16-code chunks -- release the landing stage at once,
-// and one tile later the four warps of that tile's parity turn their keys'
-// accumulator rows into scores.  The conversion is a chain of dependent
-// shared-memory and convert instructions per thread, so it is spread over
-// eight warps: with four (one key per thread) the kernel ran at about ten
-// cycles per instruction, issue- and DRAM-idle.  The key's scale comes by a
-// plain load issued a tile ahead of its use (a second 32-B tensor copy per
-// unit doubled the copies issued and measured slower).  The query enters as
-// f16 scaled by 2^qexp so that
-// its largest element lies in [2^14, 2^15) (exact for elements down to 2^-28
-// of it); the score is (sum_h w_h ReLU(q_h . code)) * 2^-qexp * scale, in fp32.
-constexpr int kF8Threads = 320;   // warps 0..7 convert and finish, 8 producer, 9 MMA
-constexpr int kF8Conv = 8;        // converter warps
-constexpr int kF8CtasPerSm = 3;
-constexpr int kF8RawStages = 4;
-constexpr int kF8OpStages = 2;
-constexpr uint32_t kF8RawBytes = kTileUnits * 512u;                     // 8 KiB of codes per stage
-constexpr uint32_t kF8TmemCols = 32;                                    // two accumulators of 16 columns
-constexpr uint32_t kF8OffA = 0;                                         // [2][16 KiB] f16 keys
-constexpr uint32_t kF8OffB = kF8OpStages * kTileBytesS;                 // Q^T [16 x 64] f16, 2 KiB
-constexpr uint32_t kF8OffRaw = kF8OffB + 2048;                          // [8][8 KiB] codes
-constexpr uint32_t kF8OffRow = kF8OffRaw + kF8RawStages * kF8RawBytes;  // int32 page x 8 + block slot (-1: none)
-constexpr uint32_t kF8OffNr = kF8OffRow + 4 * kSmUnitsPerCta;
-constexpr uint32_t kF8OffBar = kF8OffNr + 4 * kSmUnitsPerCta;           // landed / freed per landing stage,
-                                                                        // converted / done per operand stage
-constexpr uint32_t kF8OffMisc = kF8OffBar + 8 * (2 * kF8RawStages + 2 * kF8OpStages);  // TMEM base, abort, |q| max
-constexpr uint32_t kScoreF8Smem = kF8OffMisc + 16 + 1024;
-// A and B f16 (type fields 0), D fp32, N = 16, M = 128
-constexpr uint32_t kIdescScoreF16 = (1u << 4) | ((16u >> 3) << 17) | ((128u >> 4) << 24);
-static_assert(kScoreF8Smem <= 232448 / kF8CtasPerSm - 1024, "CTAs per SM");
-static_assert(kF8OffRaw % 1024 == 0 && kF8OffB % 1024 == 0, "operand and landing alignment");
-
-__global__ void __launch_bounds__(kF8Threads, kF8CtasPerSm) score_mma_fp8_kernel(
-    const __grid_constant__ CUtensorMap cmap, CacheView c, const uint16_t* __restrict__ idx_q,
-    const float* __restrict__ head_w, const int32_t* __restrict__ q_seq, const int32_t* __restrict__ q_vis,
-    const int32_t* __restrict__ pool, int64_t max_units, int64_t stride, int upc, float* __restrict__ scores) {
-  pdl_wait();
-  pdl_trigger();
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  const uint32_t raw = (uint32_t)__cvta_generic_to_shared(smem_raw);
-  const uint32_t sb = (raw + 1023u) & ~1023u;
-  uint8_t* const sp = smem_raw + (sb - raw);
-  const int r = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int seq = q_seq[r];
-  const int64_t v = visible_of(c, q_seq, q_vis, r);
-  int64_t nunits = units_of(SRC_POOL, v);
-  if (nunits > max_units) {
-    if (blockIdx.x == 0 && tid == 0) raise_error(c.err, CSA2_DEVERR_POS);
-    nunits = max_units;
-  }
-  const int64_t u0 = (int64_t)blockIdx.x * upc;
-  if (u0 >= nunits) return;
-  const int nu = (int)(nunits - u0 < upc ? nunits - u0 : upc);
-  const int ntiles = (nu + kTileUnits - 1) / kTileUnits;
-  const int64_t nb = (v + kBlock - 1) / kBlock;
-  int32_t* const urow = reinterpret_cast<int32_t*>(sp + kF8OffRow);
-  int32_t* const unr = reinterpret_cast<int32_t*>(sp + kF8OffNr);
-  uint32_t* const misc = reinterpret_cast<uint32_t*>(sp + kF8OffMisc);
-  volatile int* const abort_flag = reinterpret_cast<volatile int*>(sp + kF8OffMisc + 4);
-  auto landed = [&](int s) { return sb + kF8OffBar + 8u * s; };
-  auto freed = [&](int s) { return sb + kF8OffBar + 8u * (kF8RawStages + s); };
-  auto conv = [&](int a) { return sb + kF8OffBar + 8u * (2 * kF8RawStages + a); };
-  auto done = [&](int a) { return sb + kF8OffBar + 8u * (2 * kF8RawStages + kF8OpStages + a); };
-
-  // the query (warp 0: lane l holds dims 8 (l & 7) .. + 7 of head l >> 3), loaded
-  // while the unit lookups below run
-  uint4 qv = make_uint4(0, 0, 0, 0);
-  if (warp == 0) qv = __ldg(reinterpret_cast<const uint4*>(idx_q + (int64_t)r * kIdxHeads * kIdxDim) + lane);
-  if (tid == 0) {
-    for (int s = 0; s < kF8RawStages; ++s) {
-      mbar_init(landed(s), 1);
-      mbar_init(freed(s), kF8Conv);
-    }
-    for (int a = 0; a < kF8OpStages; ++a) {
-      mbar_init(conv(a), kF8Conv * 32);
-      mbar_init(done(a), 1);
-    }
-    *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  // units: page x 8 + the block's slot in its page (the TMA coordinates)
-  for (int j = tid; j < kSmUnitsPerCta; j += kF8Threads) {
-    int32_t row = -1, nr = 0;
-    if (j < nu) {
-      const int32_t blk = pool[(int64_t)r * kPoolBlocks + u0 + j];
-      if (blk >= 0) {
-        if ((int64_t)blk >= nb) {
-          raise_error(c.err, CSA2_DEVERR_POS);
-        } else {
-          const int64_t pg = page_of(c, seq, (int64_t)blk * kBlock);
-          if (pg >= 0) {
-            row = (int32_t)(pg * kBlocksPerPage + (blk & (kBlocksPerPage - 1)));
-            nr = (int)(v - (int64_t)blk * kBlock < kBlock ? v - (int64_t)blk * kBlock : kBlock);
-          }
-        }
-      }
-    }
-    urow[j] = row;
-    unr[j] = nr;
-  }
-  if (warp == kF8Conv && lane == 0)
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&cmap)) : "memory");
-  __syncthreads();   // the units and the barriers: the producer starts at once
-
-  // the rest of the set-up, behind a barrier the producer does not take part in
-  uint32_t tmem = 0;
-  int qexp = 0;
-  if (warp != kF8Conv) {
-    if (warp == 0) {
-      // the query's largest |element| (bf16 bits order like magnitudes) sets
-      // qexp; Q^T in f16: row h = head h (rows 4..15 zero), 128-B swizzled K-major
-      uint32_t m = __vmaxu2(__vmaxu2(qv.x & 0x7FFF7FFFu, qv.y & 0x7FFF7FFFu),
-                            __vmaxu2(qv.z & 0x7FFF7FFFu, qv.w & 0x7FFF7FFFu));
-      m = max(m & 0xFFFFu, m >> 16);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-      const int qe = m == 0 ? 0 : max(-100, min(100, 141 - (int)(m >> 7)));
-      const float qs = __uint_as_float((uint32_t)(127 + qe) << 23);
-      uint4 o;
-      o.x = pack_f16x2_rn(bf16_lo(qv.x) * qs, bf16_hi(qv.x) * qs);
-      o.y = pack_f16x2_rn(bf16_lo(qv.y) * qs, bf16_hi(qv.y) * qs);
-      o.z = pack_f16x2_rn(bf16_lo(qv.z) * qs, bf16_hi(qv.z) * qs);
-      o.w = pack_f16x2_rn(bf16_lo(qv.w) * qs, bf16_hi(qv.w) * qs);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {   // chunk 32 k + lane: row h, 16-B chunk ch
-        const int h = (32 * k + lane) >> 3, ch = lane & 7;
-        *reinterpret_cast<uint4*>(sp + kF8OffB + h * 128 + ((ch ^ (h & 7)) << 4)) =
-            k == 0 ? o : make_uint4(0, 0, 0, 0);
-      }
-      fence_async_smem();
-      if (lane == 0) misc[2] = (uint32_t)qe;
-    }
-    if (warp == kF8Conv + 1) tmem_alloc_warp(sb + kF8OffMisc, kF8TmemCols);
-    tc_fence_before();
-    asm volatile("bar.sync 1, %0;" ::"n"(kF8Threads - 32) : "memory");
-    tc_fence_after();
-    tmem = *reinterpret_cast<volatile uint32_t*>(sp + kF8OffMisc);
-    qexp = (int)misc[2];
-  }
-
-  if (warp == kF8Conv) {
-    // ---- producer: lane j copies unit j's codes ----
-    int t = 0;
-#pragma unroll 1
-    for (; t < ntiles; ++t) {
-      if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-      const int s = t % kF8RawStages, n = t / kF8RawStages;
-      bool ok = true;
-      if (n > 0) ok = __all_sync(0xffffffffu, lane != 0 || mbar_wait(freed(s), (n - 1) & 1));
-      if (!ok) {
-        if (lane == 0) {
-          *abort_flag = 1;
-          raise_error(c.err, CSA2_DEVERR_TIMEOUT);
-        }
-        break;
-      }
-      const int uj = t * kTileUnits + lane;
-      const int32_t row = (lane < kTileUnits && uj < nu) ? urow[uj] : -1;
-      const uint32_t mask = __ballot_sync(0xffffffffu, row >= 0);
-      if (lane == 0) mbar_arrive_expect_tx(landed(s), (uint32_t)__popc(mask) * 512u);
-      __syncwarp();
-      if (row >= 0)
-        tma_load_3d(sb + kF8OffRaw + (uint32_t)s * kF8RawBytes + (uint32_t)lane * 512u, &cmap, 0,
-                    8 * (row & 7), row >> 3, landed(s));
-      __syncwarp();
-    }
-    // before the CTA exits, the copies it issued have landed
-    if (lane == 0)
-      for (int k = (t > kF8RawStages ? t - kF8RawStages : 0); k < t; ++k)
-        mbar_wait(landed(k % kF8RawStages), (k / kF8RawStages) & 1);
-  } else if (warp == kF8Conv + 1) {
-    // ---- MMA issue: a tile once its keys are converted ----
-    if (lane == 0) {
-      const uint64_t bdesc = smem_desc(sb + kF8OffB, 16, 1024);
-      int t = 0;
-      for (; t < ntiles; ++t) {
-        if (*abort_flag) break;
-        const int a = t & 1;
-        if (!mbar_wait(conv(a), (t >> 1) & 1)) {
-          *abort_flag = 1;
-          raise_error(c.err, CSA2_DEVERR_TIMEOUT);
-          break;
-        }
-        tc_fence_after();
-        const uint64_t adesc = smem_desc(sb + kF8OffA + (uint32_t)a * kTileBytesS, 16, 1024);
-#pragma unroll
-        for (int k = 0; k < kIdxDim / 16; ++k)
-          mma_f16(tmem + (uint32_t)a * 16u, adesc + 2u * k, bdesc + 2u * k, kIdescScoreF16, k > 0 ? 1u : 0u);
-        mma_commit(done(a));
-      }
-      if (t > 0) mbar_wait(done((t - 1) & 1), ((t - 1) >> 1) & 1);
-    }
-  } else {
-    // ---- warps 0..7: convert half of tile t's codes, then (tiles of this
-    // warp's parity) finish tile t - 1's scores ----
-    float wv[kIdxHeads];
-#pragma unroll
-    for (int h = 0; h < kIdxHeads; ++h) wv[h] = head_w ? __ldg(head_w + (int64_t)r * kIdxHeads + h) : 1.0f;
-    const float unscale = __uint_as_float((uint32_t)(127 - qexp) << 23);
-    const int row = 32 * (warp & 3) + lane;   // the key this thread finishes (its TMEM lane)
-    const int half = warp >> 2;               // this warp finishes the tiles of parity `half`
-    // the key this thread converts, and which of its 16-code chunks: ch16 and
-    // ch16 + 2, in the order that keeps each quarter warp's shared-memory reads
-    // (landing rows 64 B apart) and swizzled writes on eight distinct bank groups
-    const int crow = 32 * (warp & 3) + 16 * half + (lane >> 1);
-    const int ch16 = lane & 1;
-    const int flip = (crow >> 1) & 1;
-    float* const srow = scores + (int64_t)r * stride;
-    auto finish = [&](int t, float kscale) -> bool {   // score of key `row` of tile t
-      const int a = t & 1;
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(done(a), (t >> 1) & 1));
-      if (!ok) {
-        if (lane == 0) {
-          *abort_flag = 1;
-          raise_error(c.err, CSA2_DEVERR_TIMEOUT);
-        }
-        return false;
-      }
-      tc_fence_after();
-      const float4 d = tmem_ld4(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)a * 16u);
-      tc_fence_before();
-      const int j = t * kTileUnits + (row >> 3);
-      float sc = __fmul_rn(wv[0], fmaxf(d.x, 0.0f));
-      sc = __fadd_rn(sc, __fmul_rn(wv[1], fmaxf(d.y, 0.0f)));
-      sc = __fadd_rn(sc, __fmul_rn(wv[2], fmaxf(d.z, 0.0f)));
-      sc = __fadd_rn(sc, __fmul_rn(wv[3], fmaxf(d.w, 0.0f)));
-      sc = __fmul_rn(__fmul_rn(sc, unscale), kscale);
-      if (j < nu) srow[(u0 + j) * kBlock + (row & 7)] = (row & 7) < unr[j] ? sc : -INFINITY;
-      return true;
-    };
-    // key `row`'s scale of tile t: a plain load issued one tile before its use
-    auto scale_of = [&](int t) -> float {
-      const int j = t * kTileUnits + (row >> 3);
-      const int32_t u = j < nu ? urow[j] : -1;
-      if (u < 0) return 0.0f;
-      return __ldg(reinterpret_cast<const float*>(c.idxk + (int64_t)(u >> 3) * kIdx8PageBytes + kIdx8ScaleOff) +
-                   (u & 7) * kBlock + (row & 7));
-    };
-    int t = 0;
-    bool go = true;
-    float ks_hold = 0.0f;
-    for (; t < ntiles; ++t) {
-      if (__any_sync(0xffffffffu, *abort_flag != 0)) {
-        go = false;
-        break;
-      }
-      const bool mine = (t & 1) == half;
-      const float ks = mine ? scale_of(t) : 0.0f;
-      const int s = t % kF8RawStages;
-      bool ok = mbar_wait(landed(s), (t / kF8RawStages) & 1);
-      // operand buffer t & 1 was last read by the MMA of tile t - 2: the warps
-      // of the other parity did not finish that tile, so they see it complete here
-      if (ok && !mine && t >= 2) ok = mbar_wait(done(t & 1), ((t - 2) >> 1) & 1);
-      if (!__all_sync(0xffffffffu, ok)) {
-        if (lane == 0) {
-          *abort_flag = 1;
-          raise_error(c.err, CSA2_DEVERR_TIMEOUT);
-        }
-        go = false;
-        break;
-      }
-      // key `crow`, two 16-code chunks (16 B each) -> four swizzled 16-B f16 chunks
-      const uint8_t* src = sp + kF8OffRaw + (uint32_t)s * kF8RawBytes + (uint32_t)crow * 64u;
-      uint8_t* dst = sp + kF8OffA + (uint32_t)(t & 1) * kTileBytesS + (uint32_t)crow * 128u;
-      const bool have = (t * kTileUnits + (crow >> 3)) < nu && urow[t * kTileUnits + (crow >> 3)] >= 0;
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int q = ch16 + 2 * (i ^ flip);   // codes 16 q .. 16 q + 15
-        const uint4 cw = have ? *reinterpret_cast<const uint4*>(src + 16 * q) : make_uint4(0, 0, 0, 0);
-        uint4 o0, o1;   // f16 chunks 2 q and 2 q + 1
-        o0.x = e4m3x2_to_f16x2(cw.x & 0xFFFFu);
-        o0.y = e4m3x2_to_f16x2(cw.x >> 16);
-        o0.z = e4m3x2_to_f16x2(cw.y & 0xFFFFu);
-        o0.w = e4m3x2_to_f16x2(cw.y >> 16);
-        o1.x = e4m3x2_to_f16x2(cw.z & 0xFFFFu);
-        o1.y = e4m3x2_to_f16x2(cw.z >> 16);
-        o1.z = e4m3x2_to_f16x2(cw.w & 0xFFFFu);
-        o1.w = e4m3x2_to_f16x2(cw.w >> 16);
-        *reinterpret_cast<uint4*>(dst + (((2 * q) ^ (crow & 7)) << 4)) = o0;
-        *reinterpret_cast<uint4*>(dst + (((2 * q + 1) ^ (crow & 7)) << 4)) = o1;
-      }
-      fence_async_smem();
-      mbar_arrive(conv(t & 1));
-      __syncwarp();
-      if (lane == 0) mbar_arrive(freed(s));   // this warp's half of the landing stage is read
-      if (t > 0 && !mine && !finish(t - 1, ks_hold)) {
-        go = false;
-        break;
-      }
-      if (mine) ks_hold = ks;
-    }
-    if (go && t > 0 && ((t - 1) & 1) == half) finish(t - 1, ks_hold);
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == kF8Conv + 1) {
-    tc_fence_after();
-    tmem_dealloc_warp(tmem, kF8TmemCols);
-  }
-}
-
 // ---- host side ----
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
@@ -851,20 +527,6 @@ static bool key_map(CUtensorMap* m, void* base, uint64_t rows, uint32_t box_rows
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// FP8 keys: the codes as a [pages][64 keys][64 B] tensor, copied as 8-key
-// boxes without swizzle.
-static bool fp8_code_map(CUtensorMap* codes, void* base, uint64_t pages) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  const cuuint64_t cd[3] = {(cuuint64_t)kIdx8RowBytes, (cuuint64_t)kPageTokens, (cuuint64_t)pages};
-  const cuuint64_t cs[2] = {(cuuint64_t)kIdx8RowBytes, (cuuint64_t)kIdx8PageBytes};
-  const cuuint32_t cb[3] = {(cuuint32_t)kIdx8RowBytes, (cuuint32_t)kBlock, 1};
-  const cuuint32_t ce[3] = {1, 1, 1};
-  return enc(codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, cd, cs, cb, ce, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 cudaError_t score_mma_set_attributes() {
   cudaError_t e = cudaFuncSetAttribute(score_mma_kernel<SRC_FLAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kScoreMmaSmem);
@@ -876,30 +538,7 @@ cudaError_t score_mma_set_attributes() {
                              (int)kScoreMmaSmem);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(score_mma_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGrpSmem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(score_mma_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScoreF8Smem);
   return e;
-}
-
-// Pool scoring of FP8 keys: the work split of the bf16 kernel at kF8CtasPerSm CTAs per SM.
-cudaError_t launch_score_mma_fp8(const CacheView& c, const uint16_t* idx_q, const float* head_w,
-                                 const int32_t* q_seq, const int32_t* q_vis, const int32_t* pool, int nq,
-                                 int64_t max_units, int64_t stride, float* scores, cudaStream_t st) {
-  CUtensorMap cm;
-  if (!fp8_code_map(&cm, c.idxk, (uint64_t)c.n_pages)) return cudaErrorInvalidValue;
-  int sms = 148, dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int64_t per_query = nq > 0 ? ((int64_t)kF8CtasPerSm * sms) / nq : 1;
-  if (per_query < 1) per_query = 1;
-  int64_t upc = (max_units + per_query - 1) / per_query;
-  upc = (upc + kTileUnits - 1) / kTileUnits * kTileUnits;
-  if (upc > kSmUnitsPerCta) upc = kSmUnitsPerCta;
-  if (upc < kTileUnits) upc = kTileUnits;
-  const dim3 grid((unsigned)((max_units + upc - 1) / upc), (unsigned)nq);
-  if (grid.x == 0 || nq == 0) return cudaSuccess;
-  launch_pdl(score_mma_fp8_kernel, grid, kF8Threads, kScoreF8Smem, st, cm, c, idx_q, head_w, q_seq, q_vis, pool,
-             max_units, stride, (int)upc, scores);
-  return cudaGetLastError();
 }
 
 // bf16 keys: the same work split as the FFMA kernel (units per CTA chosen so
