@@ -377,8 +377,9 @@ __device__ __forceinline__ void reduce_slices(const uint16_t* __restrict__ part,
 __global__ void __launch_bounds__(kPipeThreads, 1)
 attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_scale,
                  const int32_t* __restrict__ q_seq, const int32_t* __restrict__ q_vis,
-                 const int32_t* __restrict__ idx, int nsplit, int range_slots, uint16_t* __restrict__ out,
-                 uint16_t* __restrict__ part, int32_t* __restrict__ rcache, int rmode, AttnShardIO shard) {
+                 const int32_t* __restrict__ idx, int nsplit, int range_slots, int groups,
+                 uint16_t* __restrict__ out, uint16_t* __restrict__ part, int32_t* __restrict__ rcache, int rmode,
+                 AttnShardIO shard) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -403,7 +404,12 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
   const uint32_t qready = bar0 + 64u;
 
   const int split = blockIdx.x;                            // rank in the query's cluster
-  const int r = blockIdx.y;
+  // head group g of query r: heads [g H, (g + 1) H) of its groups x H.  The
+  // query, output and log-sum-exp rows of (r, g) are row rv of those arrays
+  // viewed as [nq x groups][H]; the positions, index set and row cache are r's.
+  const int rv = blockIdx.y;
+  const int r = rv / groups;
+  const bool rows_owner = rv - r * groups == 0;            // records the resolved rows
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int32_t* idx_row = idx + (int64_t)r * kTopK;
   // the cluster's CTAs all run before any touches another's shared memory:
@@ -416,7 +422,7 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
   constexpr int kQPerThread = (kQChunks + kPipeThreads - 1) / kPipeThreads;   // 10
   uint4 qv[kQPerThread];
   {
-    const uint4* qsrc = reinterpret_cast<const uint4*>(q + (int64_t)r * H * kD);
+    const uint4* qsrc = reinterpret_cast<const uint4*>(q + (int64_t)rv * H * kD);
 #pragma unroll
     for (int i = 0; i < kQPerThread; ++i) {
       const int e = tid + kPipeThreads * i;
@@ -538,7 +544,7 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
     const uint32_t at = before + incl - cnt;
     if (u0) rows_s[at] = id0;
     if (u1) rows_s[at + (u0 ? 1u : 0u)] = id1;
-    if (rmode == 1) {   // record them for the Reuse layers
+    if (rmode == 1 && rows_owner) {   // record them for the Reuse layers
       if (u0) rc_row[lo + at] = (int32_t)id0;
       if (u1) rc_row[lo + at + (u0 ? 1u : 0u)] = (int32_t)id1;
       if (tid == 0) rc_row[kMaxRows + split] = (int32_t)total;
@@ -815,7 +821,7 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
   if (warp == kMmaWarp && shard.lse2 != nullptr && nsplit == 1) {
     for (int h = lane; h < H; h += 32) {
       const float2 ml = lse_ml[h];
-      shard.lse2[(int64_t)r * H + h] = ml.y > 0.0f ? ml.x + __log2f(ml.y) : -INFINITY;
+      shard.lse2[(int64_t)rv * H + h] = ml.y > 0.0f ? ml.x + __log2f(ml.y) : -INFINITY;
     }
   }
   // f . O^T straight from TMEM to global [H][512]: the lanes of a warp hold 32
@@ -823,7 +829,7 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
   // Warps 0..11 share the work, three per TMEM sub-partition (warp % 4).
   tc_fence_after();   // the last PV's completion was observed before the barriers above
   if (warp < kMmaWarp) {
-    uint16_t* dst = nsplit == 1 ? out + (int64_t)r * H * kD : part + ((int64_t)r * nsplit + split) * H * kD;
+    uint16_t* dst = nsplit == 1 ? out + (int64_t)rv * H * kD : part + ((int64_t)rv * nsplit + split) * H * kD;
     const int sub = warp & 3;
 #pragma unroll 1
     for (int pr = warp >> 2; pr < 8; pr += 3) {   // (channel tile mt, head half h2)
@@ -862,11 +868,11 @@ attn_pipe_kernel(CacheView c, const uint16_t* __restrict__ q, int H, float sm_sc
         const float2 x = ml[j * 64 + tid];
         if (x.y > 0.0f) L += ex2(x.x - M) * x.y;
       }
-      shard.lse2[(int64_t)r * H + tid] = L > 0.0f ? M + __log2f(L) : -INFINITY;
+      shard.lse2[(int64_t)rv * H + tid] = L > 0.0f ? M + __log2f(L) : -INFINITY;
     }
-    if (nsplit == 2) reduce_slices<2>(part, out, ml, r, split, H, tid);
-    else if (nsplit == 4) reduce_slices<4>(part, out, ml, r, split, H, tid);
-    else reduce_slices<8>(part, out, ml, r, split, H, tid);
+    if (nsplit == 2) reduce_slices<2>(part, out, ml, rv, split, H, tid);
+    else if (nsplit == 4) reduce_slices<4>(part, out, ml, rv, split, H, tid);
+    else reduce_slices<8>(part, out, ml, rv, split, H, tid);
   }
 
   // teardown
@@ -893,14 +899,46 @@ static int attn_split_bound(int nq) {
   return s;
 }
 
-// Ranges per query: the largest cluster size whose clusters all fit at once.
-static int attn_splits(int nq) {
+// Co-resident clusters of s CTAs (s = 1: one CTA per SM).
+static int attn_cluster_cap(int dev, int s) {
+  if (s == 1) {
+    int sms = 0;
+    return cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? sms : 0;
+  }
+  return g_max_clusters[dev][s == 8 ? 3 : s == 4 ? 2 : 1];
+}
+
+// Head groups per query for s ranges: the largest divisor G of H / 16 for
+// which nq x G clusters of s still fit at once (a query's heads are
+// independent until the output; 16 heads is the least the P.V product's N
+// takes).
+static int attn_head_groups(int dev, int nq, int H, int s) {
+  const int cap = attn_cluster_cap(dev, s);
+  int best = 1;
+  for (int g = 2; g <= H / 16; ++g)
+    if ((H / 16) % g == 0 && (int64_t)nq * g <= cap) best = g;
+  return best;
+}
+
+// Ranges per query: among the cluster sizes s <= the workspace bound whose nq
+// clusters all fit at once, the one that puts the most CTAs to work with its
+// head groups (s x G x nq), the larger s on a tie; 1 if none fits.
+static int attn_splits(int nq, int H) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 8) return 1;
   const int bound = attn_split_bound(nq);
-  for (int lg = 3; lg >= 1; --lg)
-    if ((1 << lg) <= bound && nq <= g_max_clusters[dev][lg]) return 1 << lg;
-  return 1;
+  int best = 1;
+  int64_t best_ctas = 0;
+  for (int lg = 3; lg >= 1; --lg) {
+    const int s = 1 << lg;
+    if (s > bound || nq > g_max_clusters[dev][lg]) continue;
+    const int64_t ctas = (int64_t)s * attn_head_groups(dev, nq, H, s) * nq;
+    if (ctas > best_ctas) {
+      best = s;
+      best_ctas = ctas;
+    }
+  }
+  return best;
 }
 
 size_t attn_workspace_bytes(int nq, int H) {
@@ -937,7 +975,7 @@ cudaError_t attention_set_attributes() {
   return cudaSuccess;
 }
 
-int attn_splits_for(int nq) { return attn_splits(nq); }
+int attn_splits_for(int nq, int H) { return attn_splits(nq, H); }
 
 cudaError_t launch_attention(const CacheView& c, const uint16_t* q, int H, float sm_scale,
                              const int32_t* q_seq, const int32_t* q_vis, const int32_t* idx, int nq,
@@ -948,8 +986,10 @@ cudaError_t launch_attention(const CacheView& c, const uint16_t* q, int H, float
   if (s != 1 && s != 2 && s != 4 && s != 8) return cudaErrorInvalidValue;
   if (!rcache) rmode = 0;
   const int range = (kMaxRows + s - 1) / s;
+  int dev = 0;
+  const int groups = cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 8 ? attn_head_groups(dev, nq, H, s) : 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(s, nq);
+  cfg.gridDim = dim3(s, nq * groups);
   cfg.blockDim = dim3(kPipeThreads);
   cfg.dynamicSmemBytes = kPipeSmem;
   cfg.stream = st;
@@ -963,8 +1003,8 @@ cudaError_t launch_attention(const CacheView& c, const uint16_t* q, int H, float
   cfg.attrs = at;
   cfg.numAttrs = s > 1 ? 2 : 1;
   const AttnShardIO shard{wstart, lse2};
-  return cudaLaunchKernelEx(&cfg, attn_pipe_kernel, c, q, H, sm_scale, q_seq, q_vis, idx, s, range, out,
-                            reinterpret_cast<uint16_t*>(ws), rcache, rmode, shard);
+  return cudaLaunchKernelEx(&cfg, attn_pipe_kernel, c, q, H / groups, sm_scale, q_seq, q_vis, idx, s, range,
+                            groups, out, reinterpret_cast<uint16_t*>(ws), rcache, rmode, shard);
 }
 
 }  // namespace csa2
