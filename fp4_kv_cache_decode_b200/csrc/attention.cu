@@ -10,7 +10,9 @@
 //
 // Work split: the 640 slots of a query are cut into S contiguous ranges, one
 // CTA each (S chosen so that the grid fills the GPU; S = 1 for large
-// batches).  A CTA compacts the used slots of its range into a row list and
+// batches); a small batch also splits each query's heads into G groups of
+// H / G >= 16, one cluster of S CTAs per (query, group), since heads are
+// independent until the output.  A CTA compacts the used slots of its range into a row list and
 // walks it in 64-row tiles through a warp-specialised pipeline:
 //   * producer warps (8) keep the FP4 bytes of the next two tiles in flight
 //     in registers while they decode the current tile to bf16 (16 lanes per
