@@ -28,7 +28,7 @@ cudaError_t launch_shard_combine(const uint16_t*, const float*, int, int, int, i
                                  cudaStream_t);
 cudaError_t attention_set_attributes();
 size_t attn_workspace_bytes(int nq, int H);
-int attn_splits_for(int nq, int H);
+int attn_splits_for(int nq);
 cudaError_t launch_attention(const CacheView&, const uint16_t*, int, float, const int32_t*,
                              const int32_t*, const int32_t*, int, uint16_t*, void*, int32_t*, int, int,
                              cudaStream_t, const int32_t* = nullptr, float* = nullptr);
@@ -325,7 +325,7 @@ int csa2_sparse_attn(const csa2_cache* cache, const uint16_t* q, int32_t heads, 
   if ((st = ensure_device_setup())) return st;
   // row cache: Full / Reindex record the resolved rows, Reuse reads them when they
   // come from the set's current indexer layer with the same queries and ranges
-  const int split = attn_splits_for(nq, heads);
+  const int split = attn_splits_for(nq);
   int rmode = 0;
   if (set->attn_rows) {
     if (mode != CSA2_REUSE) rmode = 1;
@@ -483,7 +483,7 @@ int csa2_sparse_attn_shard(const csa2_cache* cache, const uint16_t* q, int32_t h
                                         nq, s);
   if (e == cudaSuccess)
     e = launch_attention(v, q, heads, sm_scale, q_seq, nullptr, lidx, nq, out, workspace, nullptr, 0,
-                         attn_splits_for(nq, heads), s, lwin, lse2);
+                         attn_splits_for(nq), s, lwin, lse2);
   return from_cuda(e);
 }
 

@@ -922,25 +922,17 @@ static int attn_head_groups(int dev, int nq, int H, int s) {
   return best;
 }
 
-// Ranges per query: among the cluster sizes s <= the workspace bound whose nq
-// clusters all fit at once, the one that puts the most CTAs to work with its
-// head groups (s x G x nq), the larger s on a tie; 1 if none fits.
-static int attn_splits(int nq, int H) {
+// Ranges per query: the largest cluster size whose clusters all fit at once
+// (fewer rows per CTA shorten its pipeline; head groups then fill the SMs
+// left idle -- trading ranges for groups, e.g. 2 ranges x 4 groups instead of
+// 4 x 1 at 17 queries, measured slower: 20.2 against 18.8 us per launch).
+static int attn_splits(int nq) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 8) return 1;
   const int bound = attn_split_bound(nq);
-  int best = 1;
-  int64_t best_ctas = 0;
-  for (int lg = 3; lg >= 1; --lg) {
-    const int s = 1 << lg;
-    if (s > bound || nq > g_max_clusters[dev][lg]) continue;
-    const int64_t ctas = (int64_t)s * attn_head_groups(dev, nq, H, s) * nq;
-    if (ctas > best_ctas) {
-      best = s;
-      best_ctas = ctas;
-    }
-  }
-  return best;
+  for (int lg = 3; lg >= 1; --lg)
+    if ((1 << lg) <= bound && nq <= g_max_clusters[dev][lg]) return 1 << lg;
+  return 1;
 }
 
 size_t attn_workspace_bytes(int nq, int H) {
@@ -977,7 +969,7 @@ cudaError_t attention_set_attributes() {
   return cudaSuccess;
 }
 
-int attn_splits_for(int nq, int H) { return attn_splits(nq, H); }
+int attn_splits_for(int nq) { return attn_splits(nq); }
 
 cudaError_t launch_attention(const CacheView& c, const uint16_t* q, int H, float sm_scale,
                              const int32_t* q_seq, const int32_t* q_vis, const int32_t* idx, int nq,
