@@ -9,7 +9,8 @@ from oracle import codec as ocodec
 from oracle import formats as ofmt
 from oracle import indexer as oidx
 from oracle import modes as omodes
-from tests.gpu_util import bits, cache_block_keys, cache_keys, cache_rows, small_workload
+from oracle import idxk_fp8 as ofp8
+from tests.gpu_util import bits, cache_block_keys, cache_keys, cache_keys_fp8, cache_rows, small_workload
 
 pytestmark = pytest.mark.gpu
 
@@ -125,6 +126,48 @@ def test_seeded_cache_pages_bit_exact(gpu):
         np.testing.assert_array_equal(cache_keys(cache, b, pos), keys)
         np.testing.assert_array_equal(cache_block_keys(cache, b, np.arange((L + 7) // 8)),
                                       oidx.block_keys(keys, L))
+
+
+@pytest.mark.parametrize("fmt", ["bf16", "fp8"])
+def test_small_appends_in_any_order_bit_exact(gpu, fmt):
+    """Small append calls (64, 50 and 23 entries, as a decode step's): entries of two
+    sequences in shuffled order, several of one block in one call (not contiguous)
+    and one block's entries spread over calls, pages in reverse order -- rows, keys
+    and block keys equal the oracle's."""
+    csa2, _ = gpu
+    lengths = [100, 37]
+    pages = [(L + 63) // 64 for L in lengths]
+    fmt_id = csa2.IDXK_FP8 if fmt == "fp8" else csa2.IDXK_BF16
+    cache = csa2.Cache(sum(pages), 2, max(pages), idxk_format=fmt_id)
+    order_pages = list(range(sum(pages)))[::-1]
+    cache.page_table[0, :pages[0]] = torch.tensor(order_pages[:pages[0]], dtype=torch.int32)
+    cache.page_table[1, :pages[1]] = torch.tensor(order_pages[pages[0]:], dtype=torch.int32)
+    cache.seq_lens[:] = torch.tensor(lengths, dtype=torch.int32)
+    rng = np.random.default_rng(11)
+    kv = [ofmt.f32_to_bf16(rng.standard_normal((L, 512)).astype(np.float32)) for L in lengths]
+    keys = [ofmt.f32_to_bf16(rng.standard_normal((L, 64)).astype(np.float32)) for L in lengths]
+    entries = [(b, p) for b, L in enumerate(lengths) for p in range(L)]
+    order = rng.permutation(len(entries))
+    for call in np.split(order, [64, 114]):   # 64, 50 and 23 entries
+        es = np.array([entries[i][0] for i in call], dtype=np.int32)
+        ep = np.array([entries[i][1] for i in call], dtype=np.int32)
+        kv_t = torch.from_numpy(np.stack([kv[b][p] for b, p in zip(es, ep)]).view(np.int16)).cuda()
+        k_t = torch.from_numpy(np.stack([keys[b][p] for b, p in zip(es, ep)]).view(np.int16)).cuda()
+        csa2.csa2_kv_quant_append(cache, kv_t, k_t, torch.from_numpy(es).cuda(), torch.from_numpy(ep).cuda())
+    assert csa2.csa2_check_device_error(cache) == 0
+    for b, L in enumerate(lengths):
+        pos = np.arange(L)
+        np.testing.assert_array_equal(cache_rows(cache, b, pos), ocodec.encode_bf16_rows(kv[b]))
+        if fmt == "fp8":
+            want = ofp8.Fp8Keys.from_bf16(keys[b])
+            codes, scales = cache_keys_fp8(cache, b, pos)
+            np.testing.assert_array_equal(codes, want.codes)
+            np.testing.assert_array_equal(scales.view(np.uint32), want.scales.astype(np.float32).view(np.uint32))
+        else:
+            want = keys[b]
+            np.testing.assert_array_equal(cache_keys(cache, b, pos), want)
+        np.testing.assert_array_equal(cache_block_keys(cache, b, np.arange((L + 7) // 8)),
+                                      oidx.block_keys(want, L))
 
 
 def test_replay_restores_poisoned_rows(gpu):
