@@ -1063,30 +1063,63 @@ def _baseline(cid, seed, kind, items, warmup, steps, procs=None):
     return float(np.median(ts)), pool.procs, ts
 
 
-def cpu_baseline(args, steps: int = 3, seed: int | None = None):
-    """The oracle's whole decode step (all 32 sequences, 8 layers) on the host cores."""
+def c_decode_baseline(cid: int, seed: int, warmup: int, steps: int, threads: int | None = None):
+    """Decode steps of the C oracle (oracle/c/csa2_oracle.c) over a workload's whole
+    batch on host threads, one sequence per thread at a time: wall seconds of each
+    timed step.  Inputs are drawn before the timing; a KV row is drawn from the
+    seeded generator the first time a set needs it and kept (the warm-up step)."""
     import workload as wl
-    w = wl.workload(CONFIG_ID)
-    sec, procs, _ = _baseline(CONFIG_ID, w.seed if seed is None else seed, "decode", range(w.batch), 1, steps)
-    return {"value": len(w.layers) / sec, "unit": UNIT, "cores": procs, "nproc": host_threads(),
-            "cpu": _cpu_model(), "kind": "oracle", "ms_per_step": sec * 1e3,
+    from oracle import c_oracle as co
+    w = wl.workload(cid)
+    seqs = [{"L": w.lengths[s], "seq": s, "keys": wl.idxk_rows(seed, s, 0, w.lengths[s]),
+             "iq": {l: wl.idxq_rows(seed, l, s) for l, m in enumerate(w.layers) if m in ("F", "RI")},
+             "q": {l: wl.q_rows(seed, l, s, w.heads) for l in range(len(w.layers))},
+             "new": wl.kv_rows(seed, s, w.lengths[s] - 1, 1)} for s in range(w.batch)]
+    threads = max(1, min(threads or host_threads(), w.batch))
+    ds = co.DecodeSteps(w.layers, w.heads, seed, seqs)
+    for _ in range(warmup):
+        ds.step(threads)
+    ts = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        ds.step(threads)
+        ts.append(time.perf_counter() - t0)
+    return w, ts, threads
+
+
+def cpu_baseline(args, steps: int = 3, seed: int | None = None):
+    """The C oracle's whole decode step (all 32 sequences, 8 layers) on the host cores."""
+    import workload as wl
+    w0 = wl.workload(CONFIG_ID)
+    w, ts, threads = c_decode_baseline(CONFIG_ID, w0.seed if seed is None else seed, 1, steps)
+    sec = float(np.median(ts))
+    return {"value": len(w.layers) / sec, "unit": UNIT, "cores": threads, "nproc": host_threads(),
+            "cpu": _cpu_model(), "kind": "oracle", "impl": "C (oracle/c/csa2_oracle.c), pthreads",
+            "ms_per_step": sec * 1e3,
             "sample": f"the whole step: {w.batch} of {w.batch} sequences, all {len(w.layers)} layers "
                       f"(append, indexer, fp64 attention); median of {steps} steps after 1 warm-up, "
-                      f"{procs} processes with one BLAS thread each"}
+                      f"{threads} host threads"}
 
 
 def workload_baselines(seed_rank: int = 0):
     """The oracle on the other workloads (bounded samples, host cores)."""
     import workload as wl
     out = {}
-    for cid, unit_per_step in ((0, 1), (2, 20), (4, 1)):
-        w = wl.workload(cid)
-        kind = "ragged" if cid == 4 else "decode"
-        sec, procs, _ = _baseline(cid, rank_seed(w.seed, seed_rank), kind, range(w.batch), 1, 2)
+    for cid, unit_per_step in ((0, 1), (2, 20)):   # decode workloads: the C oracle
+        w0 = wl.workload(cid)
+        w, ts, threads = c_decode_baseline(cid, rank_seed(w0.seed, seed_rank), 1, 2)
+        sec = float(np.median(ts))
         out[f"config{cid}"] = {
-            "value": unit_per_step / sec, "unit": UNIT, "cores": procs, "kind": "oracle",
-            "tokens_per_s": w.batch / sec, "ms_per_step": sec * 1e3,
+            "value": unit_per_step / sec, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "impl": "C, pthreads", "tokens_per_s": w.batch / sec, "ms_per_step": sec * 1e3,
             "sample": f"the whole step ({w.batch} sequences); median of 2 steps after 1 warm-up"}
+    # ragged decode with bounded replay: the numpy oracle (replay is outside the C oracle's scope)
+    w = wl.workload(4)
+    sec, procs, _ = _baseline(4, rank_seed(w.seed, seed_rank), "ragged", range(w.batch), 1, 2)
+    out["config4"] = {
+        "value": 1 / sec, "unit": UNIT, "cores": procs, "kind": "oracle", "impl": "numpy, spawned processes",
+        "tokens_per_s": w.batch / sec, "ms_per_step": sec * 1e3,
+        "sample": f"the whole step ({w.batch} sequences); median of 2 steps after 1 warm-up"}
     # prefill: the whole append plus a stratified sample of queries, extrapolated
     w = wl.workload(3)
     n_e = w.raw_tokens // w.compress
@@ -1099,6 +1132,7 @@ def workload_baselines(seed_rank: int = 0):
     total = sec_app + sec_q * w.raw_tokens / len(qs)
     out["config3"] = {
         "value": w.raw_tokens / total, "unit": "tokens/s", "cores": used, "kind": "oracle",
+        "impl": "numpy, spawned processes",
         "extrapolated": True, "prefill_s": total, "append_s": sec_app,
         "sample": f"the whole append ({w.raw_tokens} raw tokens -> {n_e} entries) timed in full; "
                   f"{len(qs)} stratified queries (every chunk's first and last position + seeded draws; "
@@ -1108,20 +1142,14 @@ def workload_baselines(seed_rank: int = 0):
 
 
 def run_reference(args):
-    """The oracle as it stands on the host cores, on the same workload and metric:
+    """The C oracle as it stands on the host cores, on the same workload and metric:
     every timed step is the whole decode step of all 32 sequences."""
     world, rank, _ = rank_env()
     if rank != 0:
         return
     import workload as wl
-    w = wl.workload(CONFIG_ID)
-    pool = OraclePool(CONFIG_ID, w.seed, "decode", range(w.batch), host_threads())
-    try:
-        for _ in range(args.warmup):
-            pool.step()
-        ts = [pool.step() for _ in range(args.steps)]
-    finally:
-        pool.close()
+    w0 = wl.workload(CONFIG_ID)
+    w, ts, threads = c_decode_baseline(CONFIG_ID, w0.seed, args.warmup, args.steps)
     total = float(sum(ts))
     value = len(w.layers) * args.steps / total
     result = {
@@ -1129,10 +1157,10 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded)", "config": _config_json(w, world),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": pool.procs, "nproc": host_threads(),
-                         "cpu": _cpu_model(), "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "nproc": host_threads(),
+                         "cpu": _cpu_model(), "kind": "oracle", "impl": "C (oracle/c/csa2_oracle.c), pthreads",
                          "sample": f"the whole step every step: {w.batch} of {w.batch} sequences, all "
-                                   f"{len(w.layers)} layers, {pool.procs} processes with one BLAS thread each"},
+                                   f"{len(w.layers)} layers, {threads} host threads"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(result), flush=True)

@@ -9,7 +9,12 @@ computes, written from the pages' description of the method:
                    hierarchical 2,048 x 8 candidate pool, Full/Reindex selection;
 * ``attention`` -- the attended set (selected tokens joined with the 128-token
                    sliding window) and exact softmax attention in fp64;
-* ``modes``     -- the Full / Reindex / Reuse layer schedule and the replay rule.
+* ``modes``     -- the Full / Reindex / Reuse layer schedule and the replay rule;
+* ``c_oracle``  -- a second restatement of the decode path in plain C
+                   (``c/csa2_oracle.c``, brute-force roundings, fp64 attention,
+                   whole decode steps on host threads), pinned on its own and
+                   checked against the numpy functions; the benchmark's CPU
+                   baseline for the decode workloads.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (its CPU
 baseline and reference arm) may import this package.  It shares no code with

@@ -1,6 +1,7 @@
-"""The benchmark's CPU oracle arm, on CPU: the spawned worker pool runs a small
-workload's whole step and reports wall times; the prefill query sample holds
-every chunk's first and last position and nothing twice."""
+"""The benchmark's CPU oracle arm, on CPU: the C oracle's threaded decode steps
+and the spawned numpy worker pool run a small workload's whole step and report
+wall times; the prefill query sample holds every chunk's first and last
+position and nothing twice."""
 import os
 import sys
 
@@ -37,3 +38,9 @@ def test_oracle_pool_splits_items_over_processes():
     finally:
         pool.close()
     assert all(p.exitcode == 0 for p in pool.ps)
+
+
+def test_c_oracle_decode_steps_time_a_whole_step():
+    import bench
+    w, ts, threads = bench.c_decode_baseline(0, 0, warmup=1, steps=2, threads=4)
+    assert threads == 1 and len(ts) == 2 and all(t > 0 for t in ts)   # one sequence: one thread
