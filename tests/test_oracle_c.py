@@ -226,6 +226,10 @@ def test_attention_textbook_closed_forms_and_union():
     np.testing.assert_allclose(co.attend(np.zeros((2, 512), np.uint16), rows),
                                np.repeat(rows.mean(0, keepdims=True), 2, 0), rtol=1e-12, atol=1e-14)
     assert np.all(co.attend(q, rows[:0]) == 0)
+    r = np.zeros((3, 512))                     # a dominant logit puts all weight on its row
+    r[1, 0] = 1.0
+    qb = _bf16(np.array([[1000.0] + [0.0] * 511]))
+    np.testing.assert_allclose(co.attend(qb, r)[0], r[1], atol=1e-300)
     idx = np.array([0, 5, 900, 950, 999] + [-1] * 507)
     np.testing.assert_array_equal(co.attended_positions(idx, 1000),
                                   np.concatenate([[0, 5], np.arange(872, 1000)]))
