@@ -760,16 +760,12 @@ def run_e2e(args, w, step, stream, flush):
     from fp4_kv_cache_decode_b200 import synthetic
     sets = [step, synthetic.DecodeStep(w, step.cache)]
 
-    def inputs(st):   # the layers' queries travel as one tensor
-        d = {"new_kv": st.new_kv, "new_k": st.new_k, "q": st.q_all}
-        for i, q in st.idxq.items():
-            d[f"iq{i}"] = q
-        return d
-    pinned = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in inputs(step).items()}
-    for k, v in inputs(step).items():
-        pinned[k].copy_(v)
+    # a step's inputs (new token, indexer and attention queries) are views of one
+    # device buffer: one host->device copy per step
+    pinned = torch.empty(step.inputs.shape, dtype=step.inputs.dtype, pin_memory=True)
+    pinned.copy_(step.inputs)
     outs = [torch.empty(st.out_all.shape, dtype=st.out_all.dtype, pin_memory=True) for st in sets]
-    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    h2d = pinned.numel() * pinned.element_size()
     d2h = outs[0].numel() * outs[0].element_size()
     up, down = torch.cuda.Stream(), torch.cuda.Stream()
 
@@ -785,8 +781,7 @@ def run_e2e(args, w, step, stream, flush):
             with torch.cuda.stream(up):   # inputs of step k (its buffer set was last used by step k-2)
                 if k >= 2:
                     up.wait_event(done[k - 2])
-                for name, t in inputs(st).items():
-                    t.copy_(pinned[name], non_blocking=True)
+                st.inputs.copy_(pinned, non_blocking=True)
                 ready[k].record(up)
             stream.wait_event(ready[k])
             if k >= 2:
