@@ -105,6 +105,39 @@ def test_attention_on_oracle_sets(ragged, heads):
                 assert np.all(g[b] == 0)
 
 
+@pytest.mark.parametrize("nq,heads", [(1, 64), (2, 64), (3, 48), (2, 32), (5, 64), (1, 16)])
+def test_attention_small_batches_split_heads(ragged, nq, heads):
+    """Small batches split each query's heads over several clusters (4 groups of 16 at
+    one or two queries of 64 heads, 3 of 16 at 48 heads, 2 of 16 or 32 at five queries
+    or 32 heads) beside the row ranges: Full and Reuse outputs match the oracle on its
+    own sets."""
+    csa2, syn, w, cache, oseqs = ragged
+    from workload import device as wdev
+    seqs = [16, 15, 14, 13, 12][:nq]      # 33,333 / 20,000 / 16,385 / 16,384 / 4,096 tokens
+    qs = torch.tensor(seqs, dtype=torch.int32, device="cuda")
+    iset = csa2.IndexSet(nq)
+    idxq = torch.cat([wdev.idxq_batch(w.seed, 0, s, 1) for s in seqs])
+    ws_i = torch.empty(csa2.csa2_workspace_bytes(csa2.OP_INDEXER, nq, 0, 33333, True), dtype=torch.uint8,
+                       device="cuda")
+    csa2.csa2_indexer_score_topk(cache, idxq, qs, csa2.FULL, 0, iset, ws_i, 33333)
+    want = np.full((nq, 512), -1, dtype=np.int32)
+    for j, s in enumerate(seqs):
+        _, idx, _ = oidx.full_indexer(wl.idxq_rows(w.seed, 0, s), oseqs[s].keys, LENGTHS[s])
+        want[j] = idx
+    iset.idx.copy_(torch.from_numpy(want))
+    ws = torch.empty(csa2.csa2_workspace_bytes(csa2.OP_ATTENTION, nq, heads), dtype=torch.uint8, device="cuda")
+    for layer, mode in ((0, csa2.FULL), (2, csa2.REUSE)):
+        q = torch.cat([wdev.q_batch(w.seed, layer, s, 1, heads) for s in seqs])
+        out = torch.empty((nq, heads, 512), dtype=torch.bfloat16, device="cuda")
+        csa2.csa2_sparse_attn(cache, q, qs, mode, layer, iset, out, ws, 1.0)
+        assert csa2.csa2_check_device_error(cache) == 0
+        g = bits(out)
+        for j, s in enumerate(seqs):
+            ref = parity.oracle_attention(oseqs[s], want[j], wl.q_rows(w.seed, layer, s, heads), LENGTHS[s])
+            err, bound = parity.attention_error(g[j], ref)
+            assert err <= bound, f"nq={nq} H={heads} seq {s} layer={layer}: err {err} > {bound}"
+
+
 def test_reuse_with_full_query_reproduces_full_output(ragged):
     csa2, syn, w, cache, oseqs = ragged
     from workload import device as wdev
