@@ -274,22 +274,13 @@ def run_gpu(args):
         for j in range(n_ev - 1):
             per_call[k, j] = diag[k][j].elapsed_time(diag[k][j + 1])   # ms
     reuse_layers = [i for i, m in enumerate(w.layers) if m == "R" and i > w.layers.index("RI")]
-    attn_graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(attn_graph):
+
+    def reuse_run():   # the step's last Reuse layers, twice, back to back as in the step
         for _ in range(2):
             for i in reuse_layers:
                 step.layer(i)
     n_attn = 2 * len(reuse_layers)
-    attn_ms = []
-    for k in range(5):
-        flush.fill_(k & 0xFF)
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        attn_graph.replay()
-        a1.record(stream)
-        torch.cuda.synchronize()
-        attn_ms.append(a0.elapsed_time(a1) / n_attn)
-    attn_launch_ms = float(np.median(attn_ms))
+    attn_launch_ms = _graph_ms(reuse_run, flush, stream, reps=7) / n_attn
 
     def graph_ms(fn, reps=5):
         return _graph_ms(fn, flush, stream, reps)
@@ -342,10 +333,12 @@ def run_gpu(args):
         t = idx_full_ms * 1e-3
         dom = {"kernel": "csa2_indexer_score_topk (Full: block + pool scoring, two top-k)",
                "bound": "hbm", "achieved": b / t / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-               "launch_ms": idx_full_ms, "launches_timed": "the Full indexer call as one CUDA graph"}
+               "launch_ms": idx_full_ms,
+               "launches_timed": "the Full indexer call after an L2 flush, 10 in one CUDA graph minus the flushes"}
     if attn_total_ms >= idx_total_ms:
         dom["launch_ms"] = reuse_ms
-        dom["launches_timed"] = "2 x 3 Reuse attention calls back to back in one CUDA graph"
+        dom["launches_timed"] = ("2 x 3 Reuse attention calls back to back after an L2 flush, 10 such "
+                                 "groups in one CUDA graph minus a graph of the 10 flushes")
     dom["frac"] = dom["achieved"] / dom["peak"]
     dom["peak_source"] = peaks["source"]
     # DRAM bytes per launch of the dominant kernel from an ncu capture of this
@@ -400,21 +393,35 @@ def run_gpu(args):
         print(json.dumps(result), flush=True)
 
 
-def _graph_ms(fn, flush, stream, reps=5):
-    """Median device time of fn() captured as a CUDA graph (L2 flushed first)."""
+def _graph_ms(fn, flush, stream, reps=5, n=10):
+    """Device time of one fn() call with the L2 flushed before it: a CUDA graph of
+    n x (flush + call) minus a graph of the same n flushes, divided by n, so that the
+    graph's launch latency and the events' 2.048-us steps drop out; median of reps."""
     import torch
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        fn()
-    ts = []
-    for k in range(reps):
-        flush.fill_(k & 0xFF)
+
+    def capture(with_call):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(n):
+                flush.fill_(i & 0xFF)
+                if with_call:
+                    fn()
+        return g
+
+    def timed(g):
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record(stream)
         g.replay()
         a1.record(stream)
         torch.cuda.synchronize()
-        ts.append(a0.elapsed_time(a1))
+        return a0.elapsed_time(a1)
+
+    g_call, g_flush = capture(True), capture(False)
+    for _ in range(2):
+        timed(g_call)
+        timed(g_flush)
+    ts = [(timed(g_call) - timed(g_flush)) / n for _ in range(reps)]
+    del g_call, g_flush
     return float(np.median(ts))
 
 
@@ -634,7 +641,7 @@ def measure_workloads(stream, flush, peaks, seed_rank: int = 0):
         torch.cuda.synchronize()
         rows += _set_rows(ch.iset.idx.cpu().numpy(), ch.q_vis.cpu().numpy())
     assert csa2.csa2_check_device_error(cache) == 0
-    ms = _graph_ms(prefill, flush, stream, reps=3)
+    ms = _graph_ms(prefill, flush, stream, reps=3, n=1)   # 16 chunks: launch latency is negligible
     vis = np.concatenate([ch.q_vis.cpu().numpy() for ch in chunks]).astype(np.float64)
     flops_attn = 4.0 * w.heads * 512 * rows * len(w.layers)
     flops_idx = 2.0 * 4 * 64 * float(vis.sum())
