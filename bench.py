@@ -834,102 +834,6 @@ def _cpu_model() -> str:
     return "unknown"
 
 
-class _Rows:
-    """bf16 KV rows of one sequence by entry position, generated on first use and
-    kept (input generation, not oracle work: the warm-up step fills it).  At
-    compression ratio 2 an entry is made of raw rows 2e and 2e + 1."""
-
-    def __init__(self, seed: int, seq: int, compress: int = 1):
-        self.seed, self.seq, self.compress = seed, seq, compress
-        self.bits = {}
-
-    def __call__(self, pos):
-        import workload as wl
-        c = self.compress
-        for p in pos.tolist():
-            if p not in self.bits:
-                self.bits[p] = wl.kv_rows(self.seed, self.seq, c * p, c)
-        return np.concatenate([self.bits[p] for p in pos.tolist()]) if len(pos) else \
-            np.zeros((0, 512), np.uint16)
-
-
-def _decoded(rows: _Rows, pos):
-    """The oracle's decoded FP4 rows of the given entry positions."""
-    from oracle import codec as ocodec
-    c, sc = ocodec.unpack_rows(ocodec.encode_entries(rows(pos), rows.compress))
-    return ocodec.dequantize(c, sc)
-
-
-def _decode_setup(w, seqs):
-    import workload as wl
-    out = []
-    for s in seqs:
-        L = w.lengths[s]
-        out.append({
-            "s": s, "L": L, "keys": wl.idxk_rows(w.seed, s, 0, L), "rows": _Rows(w.seed, s),
-            "new": wl.kv_rows(w.seed, s, L - 1, 1),
-            "iq": {l: wl.idxq_rows(w.seed, l, s) for l, m in enumerate(w.layers) if m in ("F", "RI")},
-            "q": {l: wl.q_rows(w.seed, l, s, w.heads) for l in range(len(w.layers))}})
-    return out
-
-
-def _decode_step(w, state):
-    """One decode step of the oracle for its sequences: encode the appended token,
-    then the layer schedule (Full / Reindex indexer, attention over decoded rows)."""
-    from oracle import codec as ocodec
-    from oracle import modes as omodes
-    for st in state:
-        ocodec.encode_bf16_rows(st["new"])
-        dec = {}
-
-        def rows_fn(pos, st=st, dec=dec):
-            miss = np.asarray([p for p in pos.tolist() if p not in dec], dtype=np.int64)
-            if miss.size:
-                for p, r in zip(miss.tolist(), _decoded(st["rows"], miss)):
-                    dec[p] = r
-            return np.stack([dec[p] for p in pos.tolist()])
-
-        omodes.run_layers(w.layers, st["L"], st["keys"], lambda l, st=st: st["iq"][l],
-                          lambda l, st=st: st["q"][l], rows_fn)
-
-
-def _ragged_setup(w, seqs):
-    """Per sequence: keys, the earlier Full layer's pool and set (outside the step,
-    as on the GPU), the replay block and the layer's queries."""
-    import workload as wl
-    from oracle import indexer as oidx
-    out = []
-    for s in seqs:
-        L = w.lengths[s]
-        keys = wl.idxk_rows(w.seed, s, 0, L)
-        pool, idx, _ = oidx.full_indexer(wl.idxq_rows(w.seed, 0, s), keys, L)
-        n = min(128, L)
-        kv_last = np.zeros((128, 512), np.uint16)
-        k_last = np.zeros((128, 64), np.uint16)
-        kv_last[128 - n:] = wl.kv_rows(w.seed, s, L - n, n)
-        k_last[128 - n:] = wl.idxk_rows(w.seed, s, L - n, n)
-        out.append({"s": s, "L": L, "keys": keys, "pool": pool, "idx": idx, "rows": _Rows(w.seed, s),
-                    "kv_last": kv_last, "k_last": k_last, "ri": bool(w.reindex_mask[s]),
-                    "miss": bool(w.miss_mask[s]), "iq1": wl.idxq_rows(w.seed, 1, s),
-                    "q1": wl.q_rows(w.seed, 1, s, w.heads)})
-    return out
-
-
-def _ragged_step(w, state):
-    """Bounded replay (miss: the last 128 entries, else the newest), then one layer:
-    Reindex sequences rank the Full pool with their own query, Reuse sequences keep
-    the Full set; both attend."""
-    from oracle import attention as oattn
-    from oracle import indexer as oidx
-    from oracle import modes as omodes
-    for st in state:
-        omodes.replay_entries(st["kv_last"], st["L"], st["miss"])
-        omodes.replay_keys(st["k_last"], st["L"], st["miss"])
-        idx = oidx.reindex_indexer(st["iq1"], st["keys"], st["L"], st["pool"])[0] if st["ri"] else st["idx"]
-        pos = oattn.attended_positions(idx, st["L"])
-        oattn.attend(st["q1"], _decoded(st["rows"], pos))
-
-
 def prefill_queries(w, n: int = 1024) -> np.ndarray:
     """Stratified sample of prefill query positions: every chunk's first and last
     position, the rest a seeded draw from all positions (ascending)."""
@@ -940,129 +844,6 @@ def prefill_queries(w, n: int = 1024) -> np.ndarray:
     perm = wl.permutation(w.seed, wl.stream_id(wl.TAG_LENS, 3), w.raw_tokens)
     extra = [int(p) for p in perm if int(p) not in fixed][:n - len(fixed)]
     return np.asarray(sorted(fixed | set(extra)), dtype=np.int64)
-
-
-def _prefill_setup(w, items):
-    """items: ("append", entry range) and ("query", raw position) units."""
-    import workload as wl
-    from oracle import codec as ocodec
-    st = {"append": [], "query": []}
-    keys = None
-    for kind, x in items:
-        if kind == "append":
-            e0, e1 = x
-            st["append"].append((wl.kv_rows(w.seed, 0, 2 * e0, 2 * (e1 - e0)),
-                                 wl.idxk_rows(w.seed, 0, 2 * e0, 2 * (e1 - e0))))
-        else:
-            if keys is None:
-                keys = ocodec.idxk_entries(wl.idxk_rows(w.seed, 0, 0, w.raw_tokens), w.compress)
-            st["query"].append({"P": x, "iq": wl.idxq_rows(w.seed, 0, x),
-                                "q": [wl.q_rows(w.seed, l, x, w.heads) for l in range(len(w.layers))]})
-    st["keys"], st["rows"] = keys, _Rows(w.seed, 0, w.compress)
-    return st
-
-
-def _prefill_step(w, st):
-    """The append of this worker's entry ranges (2:1 compression, FP4 encode, keys)
-    and, for each sampled query, the flat causal indexer plus the Full and Reuse
-    attention layers over the same set."""
-    from oracle import attention as oattn
-    from oracle import codec as ocodec
-    from oracle import indexer as oidx
-    for kv, k in st["append"]:
-        ocodec.encode_entries(kv, w.compress)
-        ocodec.idxk_entries(k, w.compress)
-    for qq in st["query"]:
-        v = oattn.prefill_visible(qq["P"], w.compress)
-        idx, _ = oidx.flat_indexer(qq["iq"], st["keys"], v)
-        pos = oattn.attended_positions(idx, v)
-        rows = _decoded(st["rows"], pos)
-        for q in qq["q"]:
-            oattn.attend(q, rows)
-
-
-_ORACLE_KINDS = {"decode": (_decode_setup, _decode_step), "ragged": (_ragged_setup, _ragged_step),
-                 "prefill": (_prefill_setup, _prefill_step)}
-
-
-def _oracle_worker(conn, cid: int, seed: int, kind: str, items) -> None:
-    """A spawned process: builds the inputs of its share of the sample once, then
-    runs the oracle over them each time the parent asks and reports the time."""
-    import workload as wl
-    w = wl.workload(cid)
-    w.seed = seed
-    setup, step = _ORACLE_KINDS[kind]
-    state = setup(w, items)
-    conn.send("ready")
-    while True:
-        msg = conn.recv()
-        if msg != "step":
-            break
-        t0 = time.perf_counter()
-        step(w, state)
-        conn.send(time.perf_counter() - t0)
-
-
-class OraclePool:
-    """The CPU oracle on the host cores: one spawned process per share of a
-    sample (started before or apart from any GPU work, never forked), one BLAS
-    thread each.  step() runs every share at once and returns the wall time."""
-
-    def __init__(self, cid: int, seed: int, kind: str, items, procs: int):
-        import multiprocessing as mp
-        items = list(items)
-        self.procs = max(1, min(procs, len(items)))
-        shares = [items[i::self.procs] for i in range(self.procs)]
-        ctx = mp.get_context("spawn")
-        saved = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
-        for k in saved:
-            os.environ[k] = "1"
-        try:
-            self.conns, self.ps = [], []
-            for sh in shares:
-                a, b = ctx.Pipe()
-                p = ctx.Process(target=_oracle_worker, args=(b, cid, seed, kind, sh), daemon=True)
-                p.start()
-                self.conns.append(a)
-                self.ps.append(p)
-        finally:
-            for k, v in saved.items():
-                if v is None:
-                    os.environ.pop(k, None)
-                else:
-                    os.environ[k] = v
-        for c in self.conns:
-            if c.recv() != "ready":
-                raise RuntimeError("oracle worker failed to start")
-
-    def step(self) -> float:
-        t0 = time.perf_counter()
-        for c in self.conns:
-            c.send("step")
-        for c in self.conns:
-            c.recv()
-        return time.perf_counter() - t0
-
-    def close(self) -> None:
-        for c in self.conns:
-            try:
-                c.send("stop")
-            except (BrokenPipeError, OSError):
-                pass
-        for p in self.ps:
-            p.join(timeout=30)
-
-
-def _baseline(cid, seed, kind, items, warmup, steps, procs=None):
-    """Wall seconds per step of the oracle over a sample (after `warmup` steps)."""
-    pool = OraclePool(cid, seed, kind, items, procs or host_threads())
-    try:
-        for _ in range(warmup):
-            pool.step()
-        ts = [pool.step() for _ in range(steps)]
-    finally:
-        pool.close()
-    return float(np.median(ts)), pool.procs, ts
 
 
 def c_decode_baseline(cid: int, seed: int, warmup: int, steps: int, threads: int | None = None):
@@ -1087,6 +868,66 @@ def c_decode_baseline(cid: int, seed: int, warmup: int, steps: int, threads: int
         ds.step(threads)
         ts.append(time.perf_counter() - t0)
     return w, ts, threads
+
+
+def c_ragged_baseline(seed: int, warmup: int, steps: int, threads: int | None = None):
+    """Ragged decode steps with bounded replay (the 64-sequence workload) on the C
+    oracle: per sequence the Full layer's pool and set are computed before the timing
+    (as on the GPU, where an earlier Full layer made them), then each timed step
+    replays, re-ranks (Reindex sequences) or keeps the set (Reuse) and attends."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import workload as wl
+    from oracle import c_oracle as co
+    w = wl.workload(4)
+    threads = max(1, min(threads or host_threads(), w.batch))
+
+    def one(s):
+        L = w.lengths[s]
+        keys = wl.idxk_rows(seed, s, 0, L)
+        pool, idx = co.full_indexer(wl.idxq_rows(seed, 0, s), keys, L)
+        n = min(128, L)
+        kv_last = np.zeros((128, 512), np.uint16)
+        kv_last[128 - n:] = wl.kv_rows(seed, s, L - n, n)
+        return {"L": L, "seq": s, "ri": bool(w.reindex_mask[s]), "miss": bool(w.miss_mask[s]), "kv_last": kv_last,
+                "keys": keys, "pool": pool, "set": idx, "iq": wl.idxq_rows(seed, 1, s),
+                "q": wl.q_rows(seed, 1, s, w.heads)}
+    with ThreadPoolExecutor(max_workers=threads) as ex:   # the C calls release the GIL
+        seqs = list(ex.map(one, range(w.batch)))
+    rs = co.RaggedSteps(w.heads, seed, seqs)
+    for _ in range(warmup):
+        rs.step(threads)
+    ts = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        rs.step(threads)
+        ts.append(time.perf_counter() - t0)
+    return w, ts, threads
+
+
+def c_prefill_baseline(seed: int, threads: int | None = None):
+    """The encoder prefill on the C oracle: the whole append (2:1 compression, FP4
+    encode, stored keys) timed in full, and the stratified query sample (flat causal
+    indexer + every layer's attention) timed and scaled to all queries.  Inputs are
+    drawn before the timing.  Returns (workload, append s, sample s, queries, threads)."""
+    import workload as wl
+    from oracle import c_oracle as co
+    w = wl.workload(3)
+    threads = threads or host_threads()
+    raw_kv = wl.kv_rows(seed, 0, 0, w.raw_tokens)
+    raw_k = wl.idxk_rows(seed, 0, 0, w.raw_tokens)
+    keys = co.key_entries(raw_k, w.compress)
+    qs = [{"P": int(P), "iq": wl.idxq_rows(seed, 0, int(P)),
+           "q": np.stack([wl.q_rows(seed, l, int(P), w.heads) for l in range(len(w.layers))])}
+          for P in prefill_queries(w)]
+    pq = co.PrefillQueries(len(w.layers), w.heads, w.compress, keys, raw_kv, raw_k, qs)
+    t0 = time.perf_counter()
+    pq.append(threads)
+    t_app = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    pq.queries(threads)
+    t_q = time.perf_counter() - t0
+    return w, t_app, t_q, len(qs), threads
 
 
 def cpu_baseline(args, steps: int = 3, seed: int | None = None):
@@ -1115,30 +956,25 @@ def workload_baselines(seed_rank: int = 0):
             "value": unit_per_step / sec, "unit": UNIT, "cores": threads, "kind": "oracle",
             "impl": "C, pthreads", "tokens_per_s": w.batch / sec, "ms_per_step": sec * 1e3,
             "sample": f"the whole step ({w.batch} sequences); median of 2 steps after 1 warm-up"}
-    # ragged decode with bounded replay: the numpy oracle (replay is outside the C oracle's scope)
-    w = wl.workload(4)
-    sec, procs, _ = _baseline(4, rank_seed(w.seed, seed_rank), "ragged", range(w.batch), 1, 2)
+    # ragged decode with bounded replay
+    w0 = wl.workload(4)
+    w, ts, threads = c_ragged_baseline(rank_seed(w0.seed, seed_rank), 1, 2)
+    sec = float(np.median(ts))
     out["config4"] = {
-        "value": 1 / sec, "unit": UNIT, "cores": procs, "kind": "oracle", "impl": "numpy, spawned processes",
+        "value": 1 / sec, "unit": UNIT, "cores": threads, "kind": "oracle", "impl": "C, pthreads",
         "tokens_per_s": w.batch / sec, "ms_per_step": sec * 1e3,
-        "sample": f"the whole step ({w.batch} sequences); median of 2 steps after 1 warm-up"}
+        "sample": f"the whole step ({w.batch} sequences: replay, then one Reindex or Reuse layer); "
+                  f"median of 2 steps after 1 warm-up"}
     # prefill: the whole append plus a stratified sample of queries, extrapolated
-    w = wl.workload(3)
+    w, t_app, t_q, nq, threads = c_prefill_baseline(rank_seed(wl.workload(3).seed, seed_rank))
     n_e = w.raw_tokens // w.compress
-    qs = prefill_queries(w)
-    procs = host_threads()
-    ranges = [("append", (e, min(n_e, e + 4096))) for e in range(0, n_e, 4096)]
-    sec_app, _, _ = _baseline(3, rank_seed(w.seed, seed_rank), "prefill", ranges, 0, 1, procs)
-    sec_q, used, _ = _baseline(3, rank_seed(w.seed, seed_rank), "prefill", [("query", int(p)) for p in qs],
-                               0, 1, procs)
-    total = sec_app + sec_q * w.raw_tokens / len(qs)
+    total = t_app + t_q * w.raw_tokens / nq
     out["config3"] = {
-        "value": w.raw_tokens / total, "unit": "tokens/s", "cores": used, "kind": "oracle",
-        "impl": "numpy, spawned processes",
-        "extrapolated": True, "prefill_s": total, "append_s": sec_app,
+        "value": w.raw_tokens / total, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+        "impl": "C, pthreads", "extrapolated": True, "prefill_s": total, "append_s": t_app,
         "sample": f"the whole append ({w.raw_tokens} raw tokens -> {n_e} entries) timed in full; "
-                  f"{len(qs)} stratified queries (every chunk's first and last position + seeded draws; "
-                  f"flat indexer + {len(w.layers)} attention layers) timed and scaled x{w.raw_tokens / len(qs):g} "
+                  f"{nq} stratified queries (every chunk's first and last position + seeded draws; "
+                  f"flat indexer + {len(w.layers)} attention layers) timed and scaled x{w.raw_tokens / nq:g} "
                   f"to all {w.raw_tokens} queries"}
     return out
 

@@ -54,6 +54,7 @@
 #define POOL_BLOCKS 2048
 #define TOP_K 512
 #define WINDOW 128
+#define REPLAY 128
 
 /* ---------------- number formats ---------------- */
 
@@ -107,34 +108,73 @@ static int nearest_even(double t, const double* grid, int n) {
   return best;
 }
 
-/* Encode rows of 512 bf16 channels into 288-byte cache rows. */
-void csa2o_encode_rows(const uint16_t* kv, int64_t n, uint8_t* out) {
+/* Encode one row of 512 exact float values into a 288-byte cache row. */
+static void encode_row(const float* x, uint8_t* row) {
   double scale6[127], mag[8];
   for (int c = 0; c < 127; ++c) scale6[c] = 6.0 * csa2o_e4m3_value(c);   /* amax vs 6 x scale: exact */
   for (int c = 0; c < 8; ++c) mag[c] = csa2o_e2m1_value(c);
-  for (int64_t r = 0; r < n; ++r) {
-    const uint16_t* x = kv + r * D_LAT;
-    uint8_t* row = out + r * ROW_BYTES;
-    uint8_t code[D_LAT];
-    for (int g = 0; g < N_GROUPS; ++g) {
-      double amax = 0.0;
-      for (int j = 0; j < GROUP; ++j) {
-        const double v = fabs((double)bf16_to_float(x[g * GROUP + j]));
-        if (v > amax) amax = v;
-      }
-      const int sc = nearest_even(amax, scale6, 127);
-      const double s = csa2o_e4m3_value(sc);
-      row[CODE_BYTES + g] = (uint8_t)sc;
-      double grid[8];
-      for (int c = 0; c < 8; ++c) grid[c] = s * mag[c];   /* |x| vs scale x magnitude: exact */
-      for (int j = 0; j < GROUP; ++j) {
-        const float v = bf16_to_float(x[g * GROUP + j]);
-        int cd = 0;
-        if (s != 0.0) cd = nearest_even(fabs((double)v), grid, 8) | (signbit(v) ? 8 : 0);
-        code[g * GROUP + j] = (uint8_t)cd;
-      }
+  uint8_t code[D_LAT];
+  for (int g = 0; g < N_GROUPS; ++g) {
+    double amax = 0.0;
+    for (int j = 0; j < GROUP; ++j) {
+      const double v = fabs((double)x[g * GROUP + j]);
+      if (v > amax) amax = v;
     }
-    for (int j = 0; j < CODE_BYTES; ++j) row[j] = (uint8_t)(code[2 * j] | (code[2 * j + 1] << 4));
+    const int sc = nearest_even(amax, scale6, 127);
+    const double s = csa2o_e4m3_value(sc);
+    row[CODE_BYTES + g] = (uint8_t)sc;
+    double grid[8];
+    for (int c = 0; c < 8; ++c) grid[c] = s * mag[c];   /* fp32 |x| vs scale x magnitude: exact in double */
+    for (int j = 0; j < GROUP; ++j) {
+      const float v = x[g * GROUP + j];
+      int cd = 0;
+      if (s != 0.0) cd = nearest_even(fabs((double)v), grid, 8) | (signbit(v) ? 8 : 0);
+      code[g * GROUP + j] = (uint8_t)cd;
+    }
+  }
+  for (int j = 0; j < CODE_BYTES; ++j) row[j] = (uint8_t)(code[2 * j] | (code[2 * j + 1] << 4));
+}
+
+/* Encode rows of 512 bf16 channels into 288-byte cache rows. */
+void csa2o_encode_rows(const uint16_t* kv, int64_t n, uint8_t* out) {
+  float x[D_LAT];
+  for (int64_t r = 0; r < n; ++r) {
+    for (int c = 0; c < D_LAT; ++c) x[c] = bf16_to_float(kv[r * D_LAT + c]);
+    encode_row(x, out + r * ROW_BYTES);
+  }
+}
+
+/* Entries at compression ratio 1 or 2: entry e is made of raw bf16 rows
+ * [compress e, compress e + compress); at ratio 2 its value per channel is
+ * fl32(fl32(a + b) x 0.5) (mean of the pair, the reading for the encoder's
+ * compressed layers), encoded like a row. */
+static void entry_values(const uint16_t* raw, int64_t e, int compress, int width, float* x) {
+  for (int c = 0; c < width; ++c) {
+    if (compress == 1) {
+      x[c] = bf16_to_float(raw[e * width + c]);
+    } else {
+      const float a = bf16_to_float(raw[(2 * e) * width + c]), b = bf16_to_float(raw[(2 * e + 1) * width + c]);
+      const float sum = a + b;
+      x[c] = sum * 0.5f;
+    }
+  }
+}
+
+void csa2o_encode_entries(const uint16_t* raw, int64_t n, int compress, uint8_t* out) {
+  float x[D_LAT];
+  for (int64_t e = 0; e < n; ++e) {
+    entry_values(raw, e, compress, D_LAT, x);
+    encode_row(x, out + e * ROW_BYTES);
+  }
+}
+
+/* Stored indexer keys of entries: the raw key at ratio 1, bf16 of the pair
+ * mean at ratio 2. */
+void csa2o_key_entries(const uint16_t* raw, int64_t n, int compress, uint16_t* out) {
+  float x[IDX_DIM];
+  for (int64_t e = 0; e < n; ++e) {
+    entry_values(raw, e, compress, IDX_DIM, x);
+    for (int d = 0; d < IDX_DIM; ++d) out[e * IDX_DIM + d] = float_to_bf16(x[d]);
   }
 }
 
@@ -280,6 +320,14 @@ void csa2o_reindex_indexer(const uint16_t* q, const float* w, const uint16_t* ke
   int64_t* cand = (int64_t*)malloc((size_t)POOL_BLOCKS * BLOCK * sizeof(int64_t));
   const int64_t ncand = pool_tokens(pool, POOL_BLOCKS, L, cand);
   select_tokens(q, w, keys, cand, ncand, idx);
+  free(cand);
+}
+
+/* Flat indexer (encoder Full layer): the top 512 of positions [0, visible). */
+void csa2o_flat_indexer(const uint16_t* q, const float* w, const uint16_t* keys, int64_t visible, int64_t* idx) {
+  int64_t* cand = (int64_t*)malloc((size_t)(visible > 0 ? visible : 1) * sizeof(int64_t));
+  for (int64_t p = 0; p < visible; ++p) cand[p] = p;
+  select_tokens(q, w, keys, cand, visible, idx);
   free(cand);
 }
 
@@ -454,4 +502,203 @@ int csa2o_decode_steps(const csa2o_schedule* sc, csa2o_sequence* seqs, int nseq,
   free(args);
   free(th);
   return st;
+}
+
+/* ---------------- prefill queries and ragged steps over host threads ---------------- */
+
+/* Encoder prefill at compression ratio `compress`: the stored keys and the raw
+ * bf16 KV rows of the whole sequence are given. */
+typedef struct {
+  int nlayers;
+  int heads;
+  double sm_scale;
+  int compress;
+  int64_t n_entries;
+  const uint16_t* keys;       /* [n_entries][64] stored keys */
+  const uint16_t* raw_kv;     /* [compress x n_entries][512] raw bf16 rows */
+} csa2o_prefill;
+
+typedef struct {
+  int64_t P;                  /* raw position of the query */
+  const uint16_t* iq;         /* [4][64] indexer query */
+  const uint16_t* q;          /* [nlayers][heads][512] attention queries */
+  int64_t* idx;               /* [512] out */
+  double* out;                /* [nlayers][heads][512] out */
+} csa2o_prefill_query;
+
+/* One prefill query: it sees entries [0, (P + 1) / compress); the flat indexer
+ * selects over them; every layer of the group (Full, then Reuse) attends over
+ * the same set, its rows encoded from the raw rows and decoded. */
+static void prefill_query(const csa2o_prefill* pf, csa2o_prefill_query* pq) {
+  const int64_t v = (pq->P + 1) / pf->compress;
+  int64_t pos[TOP_K + WINDOW];
+  csa2o_flat_indexer(pq->iq, NULL, pf->keys, v, pq->idx);
+  const int64_t T = csa2o_attended_positions(pq->idx, v, pos);
+  uint8_t* rows8 = (uint8_t*)malloc((TOP_K + WINDOW) * ROW_BYTES);
+  double* rows = (double*)malloc((size_t)(TOP_K + WINDOW) * D_LAT * sizeof(double));
+  float x[D_LAT];
+  for (int64_t t = 0; t < T; ++t) {
+    entry_values(pf->raw_kv, pos[t], pf->compress, D_LAT, x);
+    encode_row(x, rows8 + t * ROW_BYTES);
+  }
+  csa2o_decode_rows(rows8, T, rows);
+  for (int l = 0; l < pf->nlayers; ++l)
+    csa2o_attend(pq->q + (int64_t)l * pf->heads * D_LAT, pf->heads, rows, T, pf->sm_scale,
+                 pq->out + (int64_t)l * pf->heads * D_LAT);
+  free(rows);
+  free(rows8);
+}
+
+typedef struct {
+  const csa2o_prefill* pf;
+  csa2o_prefill_query* qs;
+  int n, first, stride;
+  /* append ranges */
+  const uint16_t* raw_k;
+  uint8_t* rows_out;
+  uint16_t* keys_out;
+  int64_t e0, e1;
+} prefill_arg;
+
+static void* prefill_worker(void* p) {
+  prefill_arg* a = (prefill_arg*)p;
+  for (int i = a->first; i < a->n; i += a->stride) prefill_query(a->pf, &a->qs[i]);
+  return NULL;
+}
+
+static void* append_worker(void* p) {
+  prefill_arg* a = (prefill_arg*)p;
+  const int c = a->pf->compress;
+  if (a->e1 > a->e0) {
+    csa2o_encode_entries(a->pf->raw_kv + a->e0 * c * D_LAT, a->e1 - a->e0, c, a->rows_out + a->e0 * ROW_BYTES);
+    csa2o_key_entries(a->raw_k + a->e0 * c * IDX_DIM, a->e1 - a->e0, c, a->keys_out + a->e0 * IDX_DIM);
+  }
+  return NULL;
+}
+
+static void run_threads(void* (*fn)(void*), prefill_arg* args, int nthreads) {
+  pthread_t* th = (pthread_t*)malloc((size_t)nthreads * sizeof(pthread_t));
+  for (int t = 1; t < nthreads; ++t) pthread_create(&th[t], NULL, fn, &args[t]);
+  fn(&args[0]);
+  for (int t = 1; t < nthreads; ++t) pthread_join(th[t], NULL);
+  free(th);
+}
+
+/* The sampled prefill queries, dealt round-robin to host threads. */
+void csa2o_prefill_queries(const csa2o_prefill* pf, csa2o_prefill_query* qs, int nq, int nthreads) {
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > nq) nthreads = nq > 0 ? nq : 1;
+  prefill_arg* args = (prefill_arg*)calloc((size_t)nthreads, sizeof(prefill_arg));
+  for (int t = 0; t < nthreads; ++t) {
+    args[t].pf = pf;
+    args[t].qs = qs;
+    args[t].n = nq;
+    args[t].first = t;
+    args[t].stride = nthreads;
+  }
+  run_threads(prefill_worker, args, nthreads);
+  free(args);
+}
+
+/* The whole append of a prefill: every entry encoded (rows_out [n_entries][288])
+ * and its key stored (keys_out [n_entries][64]), entry ranges split over host
+ * threads. */
+void csa2o_prefill_append(const csa2o_prefill* pf, const uint16_t* raw_k, uint8_t* rows_out, uint16_t* keys_out,
+                          int nthreads) {
+  if (nthreads < 1) nthreads = 1;
+  prefill_arg* args = (prefill_arg*)calloc((size_t)nthreads, sizeof(prefill_arg));
+  for (int t = 0; t < nthreads; ++t) {
+    args[t].pf = pf;
+    args[t].raw_k = raw_k;
+    args[t].rows_out = rows_out;
+    args[t].keys_out = keys_out;
+    args[t].e0 = pf->n_entries * t / nthreads;
+    args[t].e1 = pf->n_entries * (t + 1) / nthreads;
+  }
+  run_threads(append_worker, args, nthreads);
+  free(args);
+}
+
+/* Ragged decode with bounded replay (one layer per sequence): a sequence
+ * flagged as a cache miss re-encodes its last min(128, L) entries from the
+ * supplied raw rows, any other its newest entry (its stored keys at ratio 1 are
+ * the raw keys); a Reindex sequence ranks the Full layer's pool with its own
+ * query, a Reuse one keeps the Full layer's set; then it attends. */
+typedef struct {
+  int64_t L;
+  int reindex;                /* 1: Reindex, 0: Reuse */
+  int miss;
+  const uint16_t* kv_last;    /* [128][512] raw rows behind the last 128 entries */
+  const uint16_t* keys;       /* [L][64] */
+  const int64_t* pool;        /* [2048] the Full layer's pool */
+  const int64_t* set;         /* [512] the Full layer's set (Reuse) */
+  const uint16_t* iq;         /* [4][64] (Reindex) */
+  const uint16_t* q;          /* [heads][512] */
+  uint64_t kv_stream;
+  uint16_t* row_cache;        /* [L][512] */
+  uint8_t* drawn;             /* [L] */
+  int64_t* idx;               /* [512] out */
+  double* out;                /* [heads][512] out */
+  uint8_t* replayed;          /* [128][288] out: the re-encoded entries, oldest first */
+  int64_t nreplayed;          /* out: how many */
+} csa2o_ragged_sequence;
+
+static void ragged_step(const csa2o_schedule* sc, csa2o_ragged_sequence* sq) {
+  const int64_t n = sq->miss ? (sq->L < REPLAY ? sq->L : REPLAY) : (sq->L > 0 ? 1 : 0);
+  uint8_t* rows8 = (uint8_t*)malloc((TOP_K + WINDOW) * ROW_BYTES);
+  csa2o_encode_rows(sq->kv_last + (REPLAY - n) * D_LAT, n, sq->replayed);   /* the replayed entries */
+  sq->nreplayed = n;
+  if (sq->reindex)
+    csa2o_reindex_indexer(sq->iq, NULL, sq->keys, sq->L, sq->pool, sq->idx);
+  else
+    memcpy(sq->idx, sq->set, TOP_K * sizeof(int64_t));
+  int64_t pos[TOP_K + WINDOW];
+  const int64_t T = csa2o_attended_positions(sq->idx, sq->L, pos);
+  double* rows = (double*)malloc((size_t)(TOP_K + WINDOW) * D_LAT * sizeof(double));
+  for (int64_t t = 0; t < T; ++t) {
+    const int64_t p = pos[t];
+    if (!sq->drawn[p]) {
+      sc->gen(sc->seed, sq->kv_stream, (uint64_t)p * D_LAT, D_LAT, 1.0f, sc->kv_col_scale, D_LAT,
+              sq->row_cache + p * D_LAT, 1);
+      sq->drawn[p] = 1;
+    }
+    csa2o_encode_rows(sq->row_cache + p * D_LAT, 1, rows8 + t * ROW_BYTES);
+  }
+  csa2o_decode_rows(rows8, T > 0 ? T : 0, rows);
+  csa2o_attend(sq->q, sc->heads, rows, T > 0 ? T : 0, sc->sm_scale, sq->out);
+  free(rows);
+  free(rows8);
+}
+
+typedef struct {
+  const csa2o_schedule* sc;
+  csa2o_ragged_sequence* seqs;
+  int n, first, stride;
+} ragged_arg;
+
+static void* ragged_worker(void* p) {
+  ragged_arg* a = (ragged_arg*)p;
+  for (int i = a->first; i < a->n; i += a->stride) ragged_step(a->sc, &a->seqs[i]);
+  return NULL;
+}
+
+/* One ragged step of every sequence on host threads (the schedule supplies
+ * heads, sm_scale and the generator; its modes are not used). */
+void csa2o_ragged_steps(const csa2o_schedule* sc, csa2o_ragged_sequence* seqs, int n, int nthreads) {
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > n) nthreads = n > 0 ? n : 1;
+  pthread_t* th = (pthread_t*)malloc((size_t)nthreads * sizeof(pthread_t));
+  ragged_arg* args = (ragged_arg*)malloc((size_t)nthreads * sizeof(ragged_arg));
+  for (int t = 0; t < nthreads; ++t) {
+    args[t].sc = sc;
+    args[t].seqs = seqs;
+    args[t].n = n;
+    args[t].first = t;
+    args[t].stride = nthreads;
+  }
+  for (int t = 1; t < nthreads; ++t) pthread_create(&th[t], NULL, ragged_worker, &args[t]);
+  ragged_worker(&args[0]);
+  for (int t = 1; t < nthreads; ++t) pthread_join(th[t], NULL);
+  free(args);
+  free(th);
 }

@@ -5,14 +5,18 @@ A second CPU oracle, written in plain C independently of this package's
 numpy functions (it shares no code with them or with the CUDA path): the FP4
 codec, block keys, fp32 indexer scores, the lowest-position top-k, the
 hierarchical Full and the Reindex selection, the attended set and fp64
-softmax attention, and a driver that runs whole decode steps of many
-sequences on host threads (the benchmark's CPU baseline).  Its roundings are
+softmax attention, ratio-2 entries and the flat causal indexer, and drivers
+that run whole decode steps, sampled prefill queries (with the whole append)
+and ragged steps with bounded replay on host threads (the benchmark's CPU
+baselines).  Its roundings are
 brute-force nearest-grid searches rather than the numpy oracle's midpoint
 counts; ``tests/test_oracle_c.py`` pins it to the pages' value tables, closed
 forms and brute force, and checks it against the numpy oracle.
 
-Scope: the decode path with bf16 indexer keys (FP8 keys, 2:1 compression,
-replay and the prefill visibility rule are the numpy oracle's only).
+Scope: bf16 indexer keys -- the decode path, the encoder prefill at 2:1
+compression (entry encoding, stored keys, the flat causal indexer) and the
+ragged decode with bounded replay (FP8 keys and the sliding-window store are
+the numpy oracle's only).
 
 Only ``tests/``, ``__graft_entry__`` (build) and ``bench.py`` (CPU baseline)
 use it.
@@ -60,6 +64,26 @@ class Sequence(ctypes.Structure):
                 ("out", ctypes.c_void_p), ("status", ctypes.c_int)]
 
 
+class Prefill(ctypes.Structure):
+    _fields_ = [("nlayers", ctypes.c_int), ("heads", ctypes.c_int), ("sm_scale", ctypes.c_double),
+                ("compress", ctypes.c_int), ("n_entries", ctypes.c_int64), ("keys", ctypes.c_void_p),
+                ("raw_kv", ctypes.c_void_p)]
+
+
+class PrefillQuery(ctypes.Structure):
+    _fields_ = [("P", ctypes.c_int64), ("iq", ctypes.c_void_p), ("q", ctypes.c_void_p), ("idx", ctypes.c_void_p),
+                ("out", ctypes.c_void_p)]
+
+
+class RaggedSequence(ctypes.Structure):
+    _fields_ = [("L", ctypes.c_int64), ("reindex", ctypes.c_int), ("miss", ctypes.c_int),
+                ("kv_last", ctypes.c_void_p), ("keys", ctypes.c_void_p), ("pool", ctypes.c_void_p),
+                ("set", ctypes.c_void_p), ("iq", ctypes.c_void_p), ("q", ctypes.c_void_p),
+                ("kv_stream", ctypes.c_uint64), ("row_cache", ctypes.c_void_p), ("drawn", ctypes.c_void_p),
+                ("idx", ctypes.c_void_p), ("out", ctypes.c_void_p), ("replayed", ctypes.c_void_p),
+                ("nreplayed", ctypes.c_int64)]
+
+
 def lib():
     global _lib
     if _lib is None:
@@ -78,6 +102,12 @@ def lib():
             "csa2o_attended_positions": (i64, [vp, i64, vp]),
             "csa2o_attend": (None, [vp, i32, vp, i64, f64, vp]),
             "csa2o_decode_steps": (i32, [ctypes.POINTER(Schedule), ctypes.POINTER(Sequence), i32, i32]),
+            "csa2o_encode_entries": (None, [vp, i64, i32, vp]),
+            "csa2o_key_entries": (None, [vp, i64, i32, vp]),
+            "csa2o_flat_indexer": (None, [vp, vp, vp, i64, vp]),
+            "csa2o_prefill_queries": (None, [ctypes.POINTER(Prefill), ctypes.POINTER(PrefillQuery), i32, i32]),
+            "csa2o_prefill_append": (None, [ctypes.POINTER(Prefill), vp, vp, vp, i32]),
+            "csa2o_ragged_steps": (None, [ctypes.POINTER(Schedule), ctypes.POINTER(RaggedSequence), i32, i32]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -107,6 +137,24 @@ def encode_rows(kv_bits) -> np.ndarray:
     kv = _c(kv_bits, np.uint16).reshape(-1, D)
     out = np.zeros((kv.shape[0], 288), np.uint8)
     lib().csa2o_encode_rows(_p(kv), kv.shape[0], _p(out))
+    return out
+
+
+def encode_entries(raw_bits, compress: int) -> np.ndarray:
+    """Raw bf16 rows [compress x n, 512] -> n cache rows (ratio 2: pair means)."""
+    raw = _c(raw_bits, np.uint16).reshape(-1, D)
+    n = raw.shape[0] // compress
+    out = np.zeros((n, 288), np.uint8)
+    lib().csa2o_encode_entries(_p(raw), n, int(compress), _p(out))
+    return out
+
+
+def key_entries(raw_bits, compress: int) -> np.ndarray:
+    """Raw bf16 indexer keys [compress x n, 64] -> n stored keys."""
+    raw = _c(raw_bits, np.uint16).reshape(-1, 64)
+    n = raw.shape[0] // compress
+    out = np.zeros((n, 64), np.uint16)
+    lib().csa2o_key_entries(_p(raw), n, int(compress), _p(out))
     return out
 
 
@@ -154,6 +202,14 @@ def reindex_indexer(q_bits, key_bits, length: int, pool) -> np.ndarray:
     q, k, pl = _c(q_bits, np.uint16), _c(key_bits, np.uint16), _c(pool, np.int64)
     idx = np.zeros(TOP_K, np.int64)
     lib().csa2o_reindex_indexer(_p(q), None, _p(k), length, _p(pl), _p(idx))
+    return idx
+
+
+def flat_indexer(q_bits, key_bits, visible: int) -> np.ndarray:
+    """Top-512 positions among [0, visible), ascending, -1 padded."""
+    q, k = _c(q_bits, np.uint16), _c(key_bits, np.uint16)
+    idx = np.zeros(TOP_K, np.int64)
+    lib().csa2o_flat_indexer(_p(q), None, _p(k), int(visible), _p(idx))
     return idx
 
 
@@ -218,3 +274,74 @@ class DecodeSteps:
     def step(self, threads: int) -> None:
         if lib().csa2o_decode_steps(ctypes.byref(self.sched), self.arr, self.n, int(threads)) != 0:
             raise ValueError("decode step failed (schedule or position)")
+
+
+class PrefillQueries:
+    """Sampled queries of an encoder prefill on host threads, and the whole append.
+
+    keys: stored keys [n_entries, 64]; raw_kv / raw_k: the sequence's raw bf16 rows
+    [compress x n_entries, 512 / 64]; queries: per sampled raw position P a dict
+    with ``P``, ``iq`` [4, 64] and ``q`` [nlayers, heads, 512]."""
+
+    def __init__(self, nlayers: int, heads: int, compress: int, keys, raw_kv, raw_k, queries,
+                 sm_scale: float = 1.0):
+        self._keys, self._kv, self._k = _c(keys, np.uint16), _c(raw_kv, np.uint16), _c(raw_k, np.uint16)
+        n_e = self._keys.shape[0]
+        self.pf = Prefill(nlayers, heads, sm_scale, compress, n_e, _p(self._keys).value, _p(self._kv).value)
+        self.rows_out = np.zeros((n_e, 288), np.uint8)
+        self.keys_out = np.zeros((n_e, 64), np.uint16)
+        self._keep, self.idx, self.out = [], [], []
+        self.arr = (PrefillQuery * len(queries))()
+        for i, qq in enumerate(queries):
+            iq, q = _c(qq["iq"], np.uint16), _c(qq["q"], np.uint16)
+            idx, out = np.zeros(TOP_K, np.int64), np.zeros((nlayers, heads, D), np.float64)
+            self._keep += [iq, q]
+            self.idx.append(idx)
+            self.out.append(out)
+            self.arr[i] = PrefillQuery(int(qq["P"]), _p(iq).value, _p(q).value, _p(idx).value, _p(out).value)
+
+    def queries(self, threads: int) -> None:
+        lib().csa2o_prefill_queries(ctypes.byref(self.pf), self.arr, len(self.arr), int(threads))
+
+    def append(self, threads: int) -> None:
+        lib().csa2o_prefill_append(ctypes.byref(self.pf), _p(self._k), _p(self.rows_out), _p(self.keys_out),
+                                   int(threads))
+
+
+class RaggedSteps:
+    """Ragged decode steps with bounded replay on host threads: per sequence a dict
+    with ``L``, ``seq``, ``ri`` (Reindex, else Reuse), ``miss``, ``kv_last`` [128, 512],
+    ``keys`` [L, 64], the Full layer's ``pool`` [2048] and ``set`` [512], ``iq`` [4, 64]
+    and ``q`` [heads, 512]."""
+
+    def __init__(self, heads: int, seed: int, seqs, sm_scale: float = 1.0):
+        import workload as wl
+        self.n = len(seqs)
+        self._col = wl.kv_col_scale(seed).astype(np.float32)
+        gen = ctypes.cast(wl.host_lib().wl_fill_normal_bf16, ctypes.c_void_p).value
+        self.sched = Schedule(0, b"", heads, sm_scale, seed, _p(self._col).value, gen)
+        self._keep, self.idx, self.out, self.replayed = [], [], [], []
+        self.arr = (RaggedSequence * self.n)()
+        for i, s in enumerate(seqs):
+            L = int(s["L"])
+            parts = [_c(s["kv_last"], np.uint16), _c(s["keys"], np.uint16), _c(s["pool"], np.int64),
+                     _c(s["set"], np.int64), _c(s["iq"], np.uint16), _c(s["q"], np.uint16),
+                     np.zeros((max(L, 1), D), np.uint16), np.zeros(max(L, 1), np.uint8)]
+            idx, out = np.zeros(TOP_K, np.int64), np.zeros((heads, D), np.float64)
+            rep = np.zeros((WINDOW, 288), np.uint8)
+            self._keep += parts
+            self.idx.append(idx)
+            self.out.append(out)
+            self.replayed.append(rep)
+            self.arr[i] = RaggedSequence(L, int(bool(s["ri"])), int(bool(s["miss"])),
+                                         *[_p(x).value for x in parts[:6]],
+                                         wl.stream_id(wl.TAG_KV, 0, int(s["seq"])),
+                                         _p(parts[6]).value, _p(parts[7]).value, _p(idx).value, _p(out).value,
+                                         _p(rep).value, 0)
+
+    def replayed_rows(self, i: int) -> np.ndarray:
+        """The entries sequence i re-encoded in the last step (oldest first)."""
+        return self.replayed[i][:self.arr[i].nreplayed].copy()
+
+    def step(self, threads: int) -> None:
+        lib().csa2o_ragged_steps(ctypes.byref(self.sched), self.arr, self.n, int(threads))

@@ -1,7 +1,6 @@
 """The benchmark's CPU oracle arm, on CPU: the C oracle's threaded decode steps
-and the spawned numpy worker pool run a small workload's whole step and report
-wall times; the prefill query sample holds every chunk's first and last
-position and nothing twice."""
+time a small workload's whole step; the prefill query sample holds every
+chunk's first and last position and nothing twice."""
 import os
 import sys
 
@@ -22,22 +21,6 @@ def test_prefill_query_sample_is_stratified():
     for c in range(w.raw_tokens // w.chunk):
         assert c * w.chunk in qs and (c + 1) * w.chunk - 1 in qs
     np.testing.assert_array_equal(qs, bench.prefill_queries(w))     # seeded
-
-
-def test_oracle_pool_times_a_whole_step():
-    import bench
-    sec, procs, ts = bench._baseline(0, 0, "decode", [0], warmup=1, steps=2, procs=2)
-    assert procs == 1 and len(ts) == 2 and all(t > 0 for t in ts) and sec > 0
-
-
-def test_oracle_pool_splits_items_over_processes():
-    import bench
-    pool = bench.OraclePool(3, 3, "prefill", [("query", 5), ("query", 70000), ("append", (0, 64))], 2)
-    try:
-        assert pool.procs == 2 and pool.step() > 0
-    finally:
-        pool.close()
-    assert all(p.exitcode == 0 for p in pool.ps)
 
 
 def test_c_oracle_decode_steps_time_a_whole_step():

@@ -294,3 +294,83 @@ def test_codec_and_indexer_agree_with_the_numpy_oracle():
     np.testing.assert_array_equal(pool, p2)
     np.testing.assert_array_equal(idx, i2)
     np.testing.assert_array_equal(co.attended_positions(idx, 40000), oattn.attended_positions(i2, 40000))
+
+
+def test_ratio2_entries_pins_and_agreement():
+    rng = np.random.default_rng(7)
+    a = _bf16(rng.standard_normal((6, 512)))
+    # (a, a) pairs are entries a; (a, -a) pairs average to zero rows
+    np.testing.assert_array_equal(co.encode_entries(np.repeat(a, 2, axis=0), 2), co.encode_rows(a))
+    neg = np.empty((12, 512), np.uint16)
+    neg[0::2], neg[1::2] = a, a ^ np.uint16(0x8000)
+    assert np.all(co.encode_entries(neg, 2) == 0)
+    k = _bf16(rng.standard_normal((8, 64)))
+    np.testing.assert_array_equal(co.key_entries(np.repeat(k, 2, axis=0), 2), k)
+    # hand values: the pair (1, 2) averages to 1.5 in every channel
+    pair = np.stack([_bf16(np.ones(512)), _bf16(np.full(512, 2.0))])
+    np.testing.assert_array_equal(co.decode_rows(co.encode_entries(pair, 2)), co.decode_rows(co.encode_rows(
+        _bf16(np.full((1, 512), 1.5)))))
+    # against the numpy oracle on wide-range pairs
+    raw = _bf16(rng.standard_normal((800, 512)) * np.exp(rng.uniform(-8, 8, (800, 1))))
+    np.testing.assert_array_equal(co.encode_entries(raw, 2), ocodec.encode_entries(raw, 2))
+    kr = _bf16(rng.standard_normal((800, 64)))
+    np.testing.assert_array_equal(co.key_entries(kr, 2), ocodec.idxk_entries(kr, 2))
+
+
+def test_flat_indexer_brute_force():
+    rng = np.random.default_rng(8)
+    keys = _bf16(rng.standard_normal((3000, 64)))
+    q = _bf16(rng.standard_normal((4, 64)))
+    for v in (0, 1, 511, 512, 513, 3000):
+        assert list(co.flat_indexer(q, keys, v)) == _brute_topk(co.index_scores(q, keys[:v]), 512)
+
+
+def test_prefill_queries_and_append_agree_with_the_numpy_oracle():
+    rng = np.random.default_rng(9)
+    n_raw, heads, nl = 4000, 16, 3
+    raw_kv = _bf16(rng.standard_normal((n_raw, 512)))
+    raw_k = _bf16(rng.standard_normal((n_raw, 64)))
+    keys = ocodec.idxk_entries(raw_k, 2)
+    qs = [{"P": P, "iq": _bf16(rng.standard_normal((4, 64))),
+           "q": _bf16(rng.standard_normal((nl, heads, 512)) / np.sqrt(512))} for P in (0, 1, 2, 255, 2047, 3999)]
+    pq = co.PrefillQueries(nl, heads, 2, keys, raw_kv, raw_k, qs, 0.5)
+    pq.append(3)
+    np.testing.assert_array_equal(pq.rows_out, ocodec.encode_entries(raw_kv, 2))
+    np.testing.assert_array_equal(pq.keys_out, keys)
+    pq.queries(2)
+    rows_all = ocodec.dequantize(*ocodec.unpack_rows(ocodec.encode_entries(raw_kv, 2)))
+    for i, qq in enumerate(qs):
+        v = oattn.prefill_visible(qq["P"], 2)
+        idx, _ = oidx.flat_indexer(qq["iq"], keys, v)
+        np.testing.assert_array_equal(pq.idx[i], idx)
+        pos = oattn.attended_positions(idx, v)
+        for l in range(nl):
+            np.testing.assert_allclose(pq.out[i][l], oattn.attend(qq["q"][l], rows_all[pos], 0.5),
+                                       rtol=1e-12, atol=1e-14)
+        if v == 0:
+            assert np.all(pq.out[i] == 0)
+
+
+def test_ragged_steps_agree_with_the_numpy_oracle():
+    seed, heads = 4, 16
+    lengths, ri, miss = [20011, 3000, 130, 1], [True, False, True, False], [True, True, False, False]
+    seqs = []
+    for s, L in enumerate(lengths):
+        keys = wl.idxk_rows(seed, s, 0, L)
+        pool, idx, _ = oidx.full_indexer(wl.idxq_rows(seed, 0, s), keys, L)
+        n = min(128, L)
+        kv_last = np.zeros((128, 512), np.uint16)
+        kv_last[128 - n:] = wl.kv_rows(seed, s, L - n, n)
+        seqs.append({"L": L, "seq": s, "ri": ri[s], "miss": miss[s], "kv_last": kv_last, "keys": keys,
+                     "pool": pool, "set": idx, "iq": wl.idxq_rows(seed, 1, s), "q": wl.q_rows(seed, 1, s, heads)})
+    rs = co.RaggedSteps(heads, seed, seqs, 0.7)
+    rs.step(3)
+    for i, s in enumerate(seqs):
+        _, want_rows = omodes.replay_entries(s["kv_last"], s["L"], s["miss"])
+        np.testing.assert_array_equal(rs.replayed_rows(i), want_rows)
+        want = oidx.reindex_indexer(s["iq"], s["keys"], s["L"], s["pool"])[0] if s["ri"] else s["set"]
+        np.testing.assert_array_equal(rs.idx[i], want)
+        pos = oattn.attended_positions(want, s["L"])
+        rows = ocodec.dequantize(*ocodec.unpack_rows(ocodec.encode_bf16_rows(
+            np.concatenate([wl.kv_rows(seed, i, int(p), 1) for p in pos]))))
+        np.testing.assert_allclose(rs.out[i], oattn.attend(s["q"], rows, 0.7), rtol=1e-12, atol=1e-14)

@@ -15,6 +15,8 @@ PINS = [pins.test_row_layout_zero_scale_and_saturation, pins.test_decode_is_code
         pins.test_scores_closed_forms_and_fp64_bound, pins.test_block_key_identities,
         pins.test_topk_brute_force_ties_and_padding, pins.test_attention_textbook_closed_forms_and_union,
         pins.test_hierarchy_brute_force, pins.test_decode_steps_invariants_and_agreement_with_the_numpy_oracle,
+        pins.test_ratio2_entries_pins_and_agreement, pins.test_flat_indexer_brute_force,
+        pins.test_ragged_steps_agree_with_the_numpy_oracle,
         pins.test_scale_byte_of_every_bf16_group_maximum, pins.test_codes_of_every_bf16_value_under_every_scale]
 
 SLIPS = {
@@ -37,6 +39,10 @@ SLIPS = {
     "no max subtraction": ("s[t] = exp(s[t] - m);", "s[t] = exp(s[t]);"),
     "Reuse selects again": ("} else if (m != 'R' || !have_set) {",
                             "} else if (m == 'R' && have_set) {\n      csa2o_full_indexer(iq, NULL, sq->keys, sq->L, pool, latest);\n      fresh = 1;\n    } else {"),
+    "no pair averaging": ("x[c] = sum * 0.5f;", "x[c] = a;"),
+    "flat indexer sees one position too many": ("for (int64_t p = 0; p < visible; ++p) cand[p] = p;\n  select_tokens(q, w, keys, cand, visible, idx);",
+                                                "for (int64_t p = 0; p < visible; ++p) cand[p] = p;\n  select_tokens(q, w, keys, cand, visible > 0 ? visible - 1 : 0, idx);"),
+    "replay window of 127": ("(sq->L < REPLAY ? sq->L : REPLAY)", "(sq->L < REPLAY - 1 ? sq->L : REPLAY - 1)"),
     "Reindex builds its own pool": ("csa2o_reindex_indexer(iq, NULL, sq->keys, sq->L, pool, latest);",
                                     "csa2o_full_indexer(iq, NULL, sq->keys, sq->L, pool, latest);"),
 }
