@@ -237,8 +237,9 @@ int csa2_indexer_score_topk(const csa2_cache* cache, const uint16_t* idx_q, cons
  * product is exact in f16 and bf16); s = sm_scale * q . k; p = softmax over
  * the set; out[r] = sum p k, rounded to bf16.  The products run on the tensor
  * cores in f16 with fp32 accumulation: q is scaled by a power of two per
- * query so that it is exact in f16 down to 2^-28 of its largest element, and
- * the weights p are rounded to f16.  q: bf16 [nq][heads][512]; out: bf16 [nq][heads][512]; heads in
+ * query (per group of its heads when a small batch splits the heads over
+ * several clusters) so that it is exact in f16 down to 2^-28 of the largest
+ * element it is scaled with, and the weights p are rounded to f16.  q: bf16 [nq][heads][512]; out: bf16 [nq][heads][512]; heads in
  * {16, 32, 48, 64}; nq <= 65535.  Mode checks (host): CSA2_FULL / CSA2_REINDEX need
  * set->layer == layer and set->mode == mode (the set is this layer's own);
  * CSA2_REUSE needs set->layer < layer (the latest Full or Reindex set).  An
