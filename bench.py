@@ -310,6 +310,13 @@ def run_gpu(args):
     bytes_full_idx = B * (nb * 128 + 16384 * 128)
     bytes_ri_idx = B * 16384 * 128
     step_bytes = bytes_full_idx + bytes_ri_idx + sum(bytes_attn)
+    # compulsory bytes: the algorithmic bytes plus every layer's attention query and
+    # output (bf16), the indexer queries and the index sets written (pool, Full and
+    # Reindex token sets, int32)
+    n_idx = sum(1 for m in w.layers if m in ("F", "RI"))
+    qo_bytes = 2 * len(w.layers) * B * w.heads * 512 * 2
+    set_bytes = B * (n_idx * 4 * 64 * 2 + 2048 * 4 + n_idx * 512 * 4)
+    compulsory_bytes = step_bytes + qo_bytes + set_bytes
     mean_call = per_call.mean(axis=0)        # ms per call type (append, L0..L7)
 
     peaks = _peaks()
@@ -363,6 +370,8 @@ def run_gpu(args):
         "tokens_per_s": B * world * args.steps / (total_ms * 1e-3),
         "hbm_gbs_achieved": hbm_gbs, "hbm_frac": hbm_gbs / peaks["hbm_gbs"],
         "step_algorithmic_bytes": step_bytes,
+        "step_compulsory_bytes": compulsory_bytes,
+        "compulsory_frac": compulsory_bytes / (ms_per_step * 1e-3) / 1e9 / peaks["hbm_gbs"],
         "ms_per_call": {c: float(m) for c, m in zip(calls, mean_call)},
         "ms_per_call_note": "diagnostic: eager steps outside the timed region, one event between calls",
         "ms_graph": {"attention_launch": reuse_ms, "indexer_full": idx_full_ms, "indexer_reindex": idx_ri_ms},
