@@ -40,6 +40,7 @@ CONFIG_ID = 1
 # 4 GiB pool, only the rows' page addresses differ
 ATTN_DRAM_BYTES_PER_LAUNCH = 9.74e6
 L2_FLUSH_BYTES = 256 << 20
+NOMINAL_HBM_GBS = 8000.0   # the B200's nominal HBM3e bandwidth, for context beside the measured peak
 
 
 def _peaks():
@@ -369,6 +370,7 @@ def run_gpu(args):
         "config": _config_json(w, world),
         "tokens_per_s": B * world * args.steps / (total_ms * 1e-3),
         "hbm_gbs_achieved": hbm_gbs, "hbm_frac": hbm_gbs / peaks["hbm_gbs"],
+        "hbm_frac_of_nominal": hbm_gbs / NOMINAL_HBM_GBS,
         "step_algorithmic_bytes": step_bytes,
         "step_compulsory_bytes": compulsory_bytes,
         "compulsory_frac": compulsory_bytes / (ms_per_step * 1e-3) / 1e9 / peaks["hbm_gbs"],
