@@ -394,6 +394,8 @@ def run_gpu(args):
             w, stream, flush, peaks, {"step": ms_per_step, "full": idx_full_ms, "reindex": idx_ri_ms})
         result["workloads"] = measure_workloads(stream, flush, peaks, rank)
         result["sharded_1m"] = measure_sharded_1m(stream, flush, result["workloads"]["config2"]["step_ms"], rank)
+        result["access_ceilings"] = measure_access_ceilings(
+            stream, flush, {"attention_launch": reuse_ms, "indexer_reindex": idx_ri_ms})
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args)
         if "workloads" in result:
@@ -764,6 +766,101 @@ def launches_per_step(w) -> int:
         elif m == "RI":
             n += 2                          # pool scores, top-k
     return n
+
+
+def measure_access_ceilings(stream, flush, ms_graph: dict) -> dict:
+    """The least time this GPU takes to move the bytes of each CSA2 kernel in its
+    access pattern (kernels that load, sum and discard: the ceilings library),
+    timed like the calls (flush-subtracted CUDA graphs, L2 flushed before each
+    launch unless stated), each checked to have read every byte it was given
+    (the sum of its loaded words against torch's sum of the same words)."""
+    import ctypes
+
+    import torch
+
+    from fp4_kv_cache_decode_b200 import _build
+    lib = ctypes.CDLL(_build.CEIL_LIB)
+    P, I = ctypes.c_void_p, ctypes.c_int
+    lib.csa2c_sink_slots.restype = ctypes.c_longlong
+    lib.csa2c_sink_slots.argtypes = [I, I]
+    lib.csa2c_stream.argtypes = [P, ctypes.c_longlong, P, I, P]
+    lib.csa2c_gather_units.argtypes = [P, P, I, P, I, P]
+    lib.csa2c_gather_rows.argtypes = [P, P, I, P, I, P]
+    lib.csa2c_attn_inputs.argtypes = [P, P, P, P, P, I, P]
+    lib.csa2c_cta_load.argtypes = [P, I, P, P]
+    dev = torch.device("cuda")
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    cur = lambda: P(torch.cuda.current_stream().cuda_stream)   # the capturing stream inside a graph
+    pool_bytes = 4 << 30
+    pool = torch.empty(pool_bytes, dtype=torch.uint8, device=dev)
+    pool.view(torch.int64).random_()
+    rng = np.random.default_rng(11)
+    n_units, n_rows = 65536, 128 * 160     # one Reindex call's pool units; one Reuse launch's rows
+    ids_u = torch.from_numpy(rng.integers(0, pool_bytes // 1024, n_units).astype(np.int32)).to(dev)
+    ids_r = torch.from_numpy(rng.integers(0, pool_bytes // 288, n_rows).astype(np.int32)).to(dev)
+    q = torch.empty(32 * 65536, dtype=torch.uint8, device=dev)
+    q.view(torch.int64).random_()
+    part = torch.empty(128 * 65536, dtype=torch.uint8, device=dev)
+    src = torch.empty(32 * 65536, dtype=torch.uint8, device=dev)
+    src.view(torch.int64).random_()
+    sink = torch.zeros(1 << 20, dtype=torch.int32, device=dev)
+    small = torch.empty(4096, dtype=torch.uint8, device=dev)   # "flush" that leaves L2 as it is
+    ptr = lambda t: P(t.data_ptr())
+
+    def words(t):   # sum of a byte tensor's 32-bit words mod 2^32
+        return int(t.contiguous().view(torch.int32).to(torch.int64).sum().item()) & 0xFFFFFFFF
+
+    def call(rc):
+        if rc != 0:
+            raise RuntimeError(f"ceilings kernel failed: {rc}")
+
+    out = {"note": "kernels that only load (and sum) the bytes of each pattern; flush-subtracted "
+                   "CUDA graphs of 10 launches, L2 flushed before each unless stated"}
+    cases = [
+        ("contiguous_read_64MiB", 64 << 20, 0, 8 * sms,
+         lambda g: lib.csa2c_stream(ptr(pool), (64 << 20) // 16, ptr(sink), g, cur()),
+         lambda: words(pool[: 64 << 20]), flush, "the copy-peak pattern at the pool scorer's size"),
+        ("units_1KiB_random_64MiB", n_units * 1024, 1, 4 * sms,
+         lambda g: lib.csa2c_gather_units(ptr(pool), ptr(ids_u), n_units, ptr(sink), g, cur()),
+         lambda: words(pool.view(-1, 1024)[ids_u.long()]), flush,
+         "one Reindex call's pool scoring: 32 x 2,048 random 1-KiB key units"),
+        ("units_1KiB_random_32MiB", n_units * 512, 1, 4 * sms,
+         lambda g: lib.csa2c_gather_units(ptr(pool), ptr(ids_u), n_units // 2, ptr(sink), g, cur()),
+         lambda: words(pool.view(-1, 1024)[ids_u[: n_units // 2].long()]), flush,
+         "the Full call's block-key scoring size (32 x 1,024 units)"),
+        ("rows_288B_random_5.9MB", n_rows * 288, 2, 4 * sms,
+         lambda g: lib.csa2c_gather_rows(ptr(pool), ptr(ids_r), n_rows, ptr(sink), g, cur()),
+         lambda: words(pool[: pool_bytes // 288 * 288].view(-1, 288)[ids_r.long()]), flush,
+         "one Reuse attention launch's FP4 rows (32 x 640), gathered by warps spread over every SM"),
+        ("attention_inputs", 128 * 65536 + n_rows * 288, 3, 128,
+         lambda g: lib.csa2c_attn_inputs(ptr(q), ptr(pool), ptr(ids_r), None, ptr(sink), 0, cur()),
+         lambda: (4 * words(q) + words(pool[: pool_bytes // 288 * 288].view(-1, 288)[ids_r.long()]))
+         & 0xFFFFFFFF, flush,
+         "the attention's split: 128 CTAs, each its query (64 KiB, shared by 4) and 160 rows"),
+        ("attention_inputs_and_slices", 128 * 65536 * 2 + n_rows * 288, 3, 128,
+         lambda g: lib.csa2c_attn_inputs(ptr(q), ptr(pool), ptr(ids_r), ptr(part), ptr(sink), 1, cur()),
+         lambda: (4 * words(q) + words(pool[: pool_bytes // 288 * 288].view(-1, 288)[ids_r.long()]))
+         & 0xFFFFFFFF, flush, "the same, then each CTA stores a 64-KiB f16 slice (the range merge's store)"),
+        ("topk_score_load_l2", 32 * 65536, 4, 32,
+         lambda g: lib.csa2c_cta_load(ptr(src), g, ptr(sink), cur()),
+         lambda: words(src), small, "32 CTAs x 1,024 threads, 64 KiB of L2-resident scores each (no flush)"),
+    ]
+    for name, nbytes, kernel, grid, launch, expect, fl, what in cases:
+        slots = int(lib.csa2c_sink_slots(kernel, grid))
+        sink.zero_()
+        call(launch(grid))
+        torch.cuda.synchronize()
+        got = int(sink[:slots].to(torch.int64).sum().item()) & 0xFFFFFFFF
+        ms = _graph_ms(lambda: call(launch(grid)), fl, stream, reps=5, n=10)
+        out[name] = {"us": ms * 1e3, "bytes": nbytes, "gbs": nbytes / (ms * 1e-3) / 1e9,
+                     "verified": got == expect(), "pattern": what}
+    a = out["attention_inputs_and_slices"]["us"]
+    out["attention_launch_over_data_floor"] = ms_graph["attention_launch"] * 1e3 / a
+    floor_ri = out["units_1KiB_random_64MiB"]["us"] + out["topk_score_load_l2"]["us"]
+    out["indexer_reindex_over_data_floor"] = ms_graph["indexer_reindex"] * 1e3 / floor_ri
+    del pool, q, part, src, sink, ids_u, ids_r
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_e2e(args, w, step, stream, flush):

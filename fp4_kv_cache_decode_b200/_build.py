@@ -15,6 +15,10 @@ LIB = os.path.join(PKG, "lib", "libcsa2.so")
 # bounded wait run out): loaded only by tests/test_gpu_timeout.py.
 TEST_LIB = os.path.join(PKG, "lib", "libcsa2_test.so")
 TEST_HOOK_SOURCES = ("attention.cu", "score_mma.cu")
+# Access-pattern ceilings (kernels that only move bytes in the CSA2 kernels'
+# patterns): a measurement aid loaded by the benchmark, not part of libcsa2.so.
+CEIL_SRC = os.path.join(PKG, "ceilings", "ceilings.cu")
+CEIL_LIB = os.path.join(PKG, "lib", "libcsa2_ceilings.so")
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",
@@ -34,10 +38,10 @@ def _inputs() -> list[str]:
 
 
 def up_to_date() -> bool:
-    if not os.path.exists(LIB) or not os.path.exists(TEST_LIB):
+    if not all(os.path.exists(p) for p in (LIB, TEST_LIB, CEIL_LIB)):
         return False
-    t = min(os.path.getmtime(LIB), os.path.getmtime(TEST_LIB))
-    return all(os.path.getmtime(p) <= t for p in _inputs())
+    t = min(os.path.getmtime(LIB), os.path.getmtime(TEST_LIB), os.path.getmtime(CEIL_LIB))
+    return all(os.path.getmtime(p) <= t for p in _inputs() + [CEIL_SRC])
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
@@ -73,4 +77,9 @@ def build(force: bool = False, verbose: bool = False) -> str:
         tmp = lib + f".tmp{os.getpid()}"
         subprocess.check_call(["nvcc", "-shared", "-gencode", "arch=compute_100a,code=sm_100a", *objs, "-o", tmp])
         os.replace(tmp, lib)
+    tmp = CEIL_LIB + f".tmp{os.getpid()}"
+    res = subprocess.run(["nvcc", *NVCC_FLAGS, "-shared", CEIL_SRC, "-o", tmp], capture_output=True, text=True)
+    if res.returncode != 0:
+        raise RuntimeError(f"nvcc failed for {CEIL_SRC}:\n{res.stderr}")
+    os.replace(tmp, CEIL_LIB)
     return LIB
